@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""One decode step of absorbed MLA over a compressed latent cache, timed on the GPU.
+
+A step is the whole hot path over one batch: cache append of the new token (a1), query absorption
+(a2), absorbed split-KV decode with its log-sum-exp merge (a3 + a4) and the per-head output
+projection through W_UV (a5). The default workload is the DeepSeek-V2/V3-shaped batch: 64 sequences
+of 4096 cached positions, H=128, d_c=512, d_r=64, bf16 storage, fp32 accumulation.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+N > 1 runs under torch.distributed.run, one process per GPU: every rank runs the full batch on its
+own GPU (independent sequences, weak scaling, no collective in the data path); timing is the max
+over ranks. `--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload
+(rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode cache-positions/s and tokens/s; % of B200 roofline (HBM or TC)"
+UNIT = "positions/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="dsv3_b64_l4096")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="bound on the CPU-baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic counts of the decode kernel (bytes that must move, FLOPs that must be done)
+# ------------------------------------------------------------------------------------------------
+def decode_counts(w, lens):
+    total = int(sum(int(L) for L in lens))
+    e = 2 if w.dtype == "bf16" else 4
+    n_tok = w.B * w.s_q
+    bytes_ = total * (w.d_c + w.d_r) * e + n_tok * w.H * ((w.d_c + w.d_r) + w.d_c) * e + n_tok * w.H * 4
+    visible = sum(int(L) * w.s_q - w.s_q * (w.s_q - 1) // 2 for L in lens)
+    flops = 2 * w.H * (2 * w.d_c + w.d_r) * visible
+    return bytes_, flops, total
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; no setting is touched)
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        0x0000000000000001: "gpu_idle", 0x0000000000000002: "applications_clocks_setting",
+        0x0000000000000004: "sw_power_cap", 0x0000000000000008: "hw_slowdown",
+        0x0000000000000010: "sync_boost", 0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown", 0x0000000000000080: "hw_power_brake_slowdown",
+        0x0000000000000100: "display_clock_setting",
+    }
+
+    def __init__(self, index):
+        self.samples = []
+        self.reasons = set()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as ex:  # noqa: BLE001
+            self.err = repr(ex)
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "nvml")}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+    def rejected(self):
+        bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+        return bool(self.reasons & bad)
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU side: the oracle on a bounded sample (baseline and reference arm)
+# ------------------------------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, seconds, max_seqs=None):
+    """Run the fp64 oracle's decode step (absorb, absorbed decode, W_UV projection) sequence by
+    sequence until `seconds` pass; return (positions, tokens, elapsed, sequences)."""
+    import numpy as np
+    import synth
+    from oracle import mla_oracle as O
+    lens = synth.seq_lengths(w)
+    W = synth.weights(w)
+    step = synth.decode_step_inputs(w)
+    W_UK = W["W_UK"].astype(np.float64)
+    W_UV = W["W_UV"].astype(np.float64)
+    chunks = synth.cache_row_chunks(w, int(lens[: (max_seqs or w.B)].sum()))
+    buf = []
+    pos_done = tok_done = seqs = 0
+    off = 0
+    t0 = time.perf_counter()
+    for b in range(w.B if max_seqs is None else min(w.B, max_seqs)):
+        L = int(lens[b])
+        while sum(len(c) for c, _ in buf) < off + L:
+            _, c, kr = next(chunks)
+            buf.append((c, kr))
+        c = np.concatenate([x for x, _ in buf])[off:off + L].astype(np.float64)
+        kr = np.concatenate([y for _, y in buf])[off:off + L].astype(np.float64)
+        off += L
+        pos = O.token_positions(L, w.s_q)
+        q_abs = O.absorb_query(step["q_nope"][b], step["q_rope_raw"][b], W_UK, pos, w.rope_base)
+        o_lat, _ = O.absorbed_decode(q_abs, c, kr, L, w.sm_scale)
+        O.out_projection(o_lat, W_UV)
+        pos_done += L
+        tok_done += w.s_q
+        seqs += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    return pos_done, tok_done, time.perf_counter() - t0, seqs
+
+
+def run_reference(args, rank, world):
+    import synth
+    if rank != 0:
+        return
+    w = synth.workload(args.workload)
+    per_step_seconds = max(0.5, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, per_step_seconds, max_seqs=1)
+    pos = tok = 0
+    el = 0.0
+    for _ in range(args.steps):
+        p, t, e, s = oracle_sample(w, per_step_seconds, max_seqs=1)
+        pos += p
+        tok += t
+        el += e
+    value = pos / el
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "seq_len": w.lengths[1] if w.lengths[0] == "fixed" else list(w.lengths),
+                   "H": w.H, "d_c": w.d_c, "d_r": w.d_r, "s_q": w.s_q},
+        "tokens_per_s": tok / el,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: sequence 0 of {w.name} ({int(synth.seq_lengths(w)[0])} positions, "
+                                   f"all {w.H} heads), fp64 absorb + absorbed decode + W_UV projection"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+def build_inputs(w, device):
+    import numpy as np
+    import torch
+    import synth
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    lens = synth.seq_lengths(w)
+    table, num_pages = synth.block_table(w, lens)
+    total = int(lens.sum())
+    pool = torch.zeros(num_pages * 64, w.d_c + w.d_r, dtype=tdt, device=device)
+    # logical row r of sequence b -> pool row through the page table
+    idx = np.empty(total, dtype=np.int64)
+    off = 0
+    for b, L in enumerate(lens):
+        p = np.arange(L)
+        idx[off:off + L] = table[b, p // 64].astype(np.int64) * 64 + p % 64
+        off += L
+    for start, c, kr in synth.cache_row_chunks(w, total):
+        n = len(c)
+        rows = torch.from_numpy(np.concatenate([c, kr], axis=1)).to(device=device, dtype=tdt)
+        pool[torch.from_numpy(idx[start:start + n]).to(device)] = rows
+    W = synth.weights(w)
+    step = synth.decode_step_inputs(w)
+    dev = {
+        "pool": pool, "num_pages": num_pages, "lens": lens,
+        "seqlens": torch.from_numpy(lens).to(device), "table": torch.from_numpy(table).to(device),
+        "w_dkv_kr": torch.from_numpy(np.concatenate([W["W_DKV"], W["W_KR"]], 1)).to(device=device, dtype=tdt),
+        "W_UK": torch.from_numpy(W["W_UK"]).to(device=device, dtype=tdt),
+        "W_UV": torch.from_numpy(W["W_UV"]).to(device=device, dtype=tdt),
+        "x_host": torch.from_numpy(step["x"]).to(tdt).pin_memory(),
+        "q_nope_host": torch.from_numpy(step["q_nope"]).to(tdt).pin_memory(),
+        "q_rope_host": torch.from_numpy(step["q_rope_raw"]).to(tdt).pin_memory(),
+    }
+    dev["x"] = dev["x_host"].to(device)
+    dev["q_nope"] = dev["q_nope_host"].to(device)
+    dev["q_rope_raw"] = dev["q_rope_host"].to(device)
+    return dev
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    import synth
+    from mla_compressed_latent_b200 import ops
+    from mla_compressed_latent_b200.ops import Dims, LatentCache
+
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=device)
+
+    w = synth.workload(args.workload)
+    dims = Dims.of(w)
+    dev = build_inputs(w, device)
+    cache = LatentCache(dev["pool"][:, :w.d_c], dev["pool"][:, w.d_c:], dev["num_pages"])
+    n_tok = w.B * w.s_q
+    tdt = dev["pool"].dtype
+    q_abs = torch.empty(w.B, w.s_q, w.H, w.d_c + w.d_r, dtype=tdt, device=device)
+    o_lat = torch.empty(w.B, w.s_q, w.H, w.d_c, dtype=tdt, device=device)
+    lse = torch.empty(w.B, w.s_q, w.H, dtype=torch.float32, device=device)
+    out = torch.empty(w.B, w.s_q, w.H, w.d_v, dtype=tdt, device=device)
+    max_pages = dev["table"].shape[1]
+    ws_dec = torch.empty(max(16, ops.mla_decode_workspace_size(dims, tdt, w.B, w.s_q, max_pages)), dtype=torch.uint8,
+                         device=device)
+    from mla_compressed_latent_b200 import _lib as L
+    import ctypes
+    dc = dims.c()
+    ws_app = torch.empty(max(16, L.load().mla_append_workspace_size(ctypes.byref(dc), w.B, w.s_q, w.C)),
+                         dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    dec_ev = []
+
+    def step(x, q_nope, q_rope, timed_decode=False):
+        ops.mla_append_cache(dims, x, dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache, workspace=ws_app)
+        ops.mla_absorb_q(dims, q_nope, q_rope, dev["W_UK"], dev["seqlens"], q_abs=q_abs)
+        if timed_decode:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+        ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"], o_lat=o_lat, lse=lse, workspace=ws_dec)
+        if timed_decode:
+            b.record(stream)
+            dec_ev.append((a, b))
+        ops.mla_out_proj(dims, o_lat, dev["W_UV"], out=out)
+
+    for _ in range(args.warmup):
+        step(dev["x"], dev["q_nope"], dev["q_rope_raw"])
+    torch.cuda.synchronize()
+    rc = ops.mla_check_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {ops.mla_status_string(rc)}")
+
+    def timed_region():
+        dec_ev.clear()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        n0 = ops.mla_launch_count()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local) as clk:
+            t0.record(stream)
+            for _ in range(args.steps):
+                step(dev["x"], dev["q_nope"], dev["q_rope_raw"], timed_decode=True)
+            t1.record(stream)
+            torch.cuda.synchronize()
+        launches = ops.mla_launch_count() - n0
+        ms = t0.elapsed_time(t1)
+        if world > 1:
+            t = torch.tensor([ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+            dist.barrier()
+        return ms, launches, clk
+
+    ms, launches, clk = timed_region()
+    remeasured = False
+    if clk.rejected():
+        ms, launches, clk = timed_region()
+        remeasured = True
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_ev)
+    assert ops.mla_check_status() == 0
+
+    # end to end through the public API: pinned host inputs in, host result out, every step
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, min(args.steps, 200))
+    e0.record(stream)
+    for _ in range(e_steps):
+        x = dev["x_host"].to(device, non_blocking=True)
+        qn = dev["q_nope_host"].to(device, non_blocking=True)
+        qr = dev["q_rope_host"].to(device, non_blocking=True)
+        step(x, qn, qr)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in (dev["x_host"], dev["q_nope_host"], dev["q_rope_host"]))
+    d2h = out_host.numel() * out_host.element_size()
+
+    bytes_, flops, positions = decode_counts(w, dev["lens"])
+    peaks, peak_kind = load_peaks()
+    step_s = ms / 1e3 / args.steps
+    value = world * positions / step_s
+    achieved_gbs = bytes_ / (dec_ms / 1e3) / 1e9
+    achieved_tf = flops / (dec_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "seq_len": w.lengths[1] if w.lengths[0] == "fixed" else list(w.lengths),
+                   "H": w.H, "D": w.D, "d_c": w.d_c, "d_r": w.d_r, "d_v": w.d_v, "s_q": w.s_q,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2: {positions * (w.d_c + w.d_r) * (2 if w.dtype == 'bf16' else 4) / 1e6:.0f} MB cache read per step"},
+        "tokens_per_s": world * n_tok / step_s,
+        "decode_us": dec_ms * 1e3,
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_kind,
+                     "kernel": "mla_decode_absorbed (decode + split merge)",
+                     "tensor_tflops": achieved_tf, "tensor_frac": achieved_tf / peaks["bf16_tflops"],
+                     "bound_frac": max(bytes_ / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) / (dec_ms / 1e3)},
+        "gpu_launches": int(launches),
+        "clocks": {**clk.summary(), "remeasured": remeasured},
+        "e2e": {"value": world * positions / (e_ms / 1e3 / e_steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e_steps},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        pos, tok, el, seqs = oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": pos / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{seqs} of {w.B} sequences ({pos} positions, all {w.H} heads): fp64 absorb + "
+                                          f"absorbed decode + W_UV projection, {el:.1f} s"}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,174 @@
+/*
+ * mla.h — C ABI of the absorbed Multi-head Latent Attention decode library (libmla.so).
+ *
+ * One decode step of one attention layer whose cache keeps, per position, only a latent row
+ * c = RMSNorm(x·W_DKV) of width d_c and one RoPE key k_r = RoPE(x·W_KR) of width d_r shared by all
+ * heads (« L'attention latente : compresser le cache », sections « L'idée : garder un résumé » and
+ * « L'obstacle : RoPE »). Queries are absorbed into latent space and attend the cached rows
+ * directly (same page, « Ce que DeepSeek fait de plus »; « Résumé technique : GQLA … »,
+ * « Chemin MQA-Absorbé »). The grouped GQA path of the GQLA page (« Chemin GQA ») is also here.
+ *
+ * Conventions shared by every call
+ *  - Pointers named as tensors are DEVICE pointers owned by the caller. The library never
+ *    allocates, frees or synchronises: it validates the arguments on the host, then enqueues
+ *    kernels on `stream` (a cudaStream_t; NULL = the legacy default stream) and returns.
+ *  - Row-major layouts; shapes are written [outer, ..., inner]. Every tensor pointer must be
+ *    16-byte aligned and every row stride a multiple of 16 bytes.
+ *  - dtype is MLA_F32 or MLA_BF16; it is the storage type of the cache, weights, queries and
+ *    outputs of that call. Accumulation, softmax and normalisation are fp32 in every kernel.
+ *  - seqlens[b] counts the cached positions of sequence b INCLUDING this step's s_q new tokens;
+ *    new token t (0 <= t < s_q) sits at position seqlens[b] - s_q + t and attends positions
+ *    0 .. seqlens[b] - s_q + t (causal among the new tokens).
+ *  - Paged cache: position p of sequence b lives in page block_table[b*max_pages + p/page_size],
+ *    slot p % page_size; page_size is 64. Row r = page*64 + slot of a pool starts at
+ *    base + r*stride elements.
+ *  - Return value: MLA_OK, or an error code with nothing launched. Errors found on the device
+ *    (a page id outside the pool, a wait that timed out) are recorded in a per-device status
+ *    word that mla_check_status() reads; the offending access is skipped, never performed.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum mla_status {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer or stride */
+  MLA_ERR_UNSUPPORTED = 2,   /* valid arguments this build has no kernel for (dtype, shape) */
+  MLA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the matching *_workspace_size */
+  MLA_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch error, bad device) */
+  MLA_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel gave up */
+  MLA_ERR_DEVICE_CHECK = 6   /* device: an index read from device memory was out of range */
+};
+
+enum mla_dtype { MLA_F32 = 0, MLA_BF16 = 1 };
+
+/* Shapes of one layer. sm_scale multiplies every score: 1/sqrt(D + d_r) (« L'obstacle : RoPE »). */
+typedef struct mla_dims {
+  int32_t H;          /* query heads */
+  int32_t D;          /* no-RoPE width of a query/key head (qk_nope) */
+  int32_t d_r;        /* width of the decoupled RoPE key, shared by all heads; even */
+  int32_t d_c;        /* latent width */
+  int32_t d_v;        /* value head width */
+  int32_t g;          /* GQLA groups, H % g == 0 (0 when the grouped path is not used) */
+  int32_t page_size;  /* positions per cache page; must be 64 */
+  float sm_scale;     /* score scale */
+  float rms_eps;      /* RMSNorm epsilon: c = z / sqrt(mean(z^2) + rms_eps) * gamma */
+  float rope_base;    /* RoPE: pair (2i, 2i+1) turns by pos * rope_base^(-2i/d_r) */
+} mla_dims_t;
+
+/* Latent cache pool: latent rows [num_pages*64, d_c] and RoPE-key rows [num_pages*64, d_r].
+ * The two may be one interleaved array (rope = latent + d_c, both strides d_c + d_r). */
+typedef struct mla_latent_cache {
+  void* latent;           /* device, dtype */
+  int64_t latent_stride;  /* elements from one row to the next, >= d_c */
+  void* rope;             /* device, dtype */
+  int64_t rope_stride;    /* elements from one row to the next, >= d_r */
+  int32_t num_pages;      /* pages in the pool; page ids must be < num_pages */
+} mla_latent_cache_t;
+
+/* Expanded GQA cache of the grouped path (« Chemin GQA »): per row, keys [g, D], values
+ * [g, d_v] and the shared RoPE key [d_r]. */
+typedef struct mla_gqa_cache {
+  void* k;  int64_t k_stride;     /* [num_pages*64, g, D]; stride = elements between rows */
+  void* v;  int64_t v_stride;     /* [num_pages*64, g, d_v] */
+  void* rope; int64_t rope_stride;/* [num_pages*64, d_r] */
+  int32_t num_pages;
+} mla_gqa_cache_t;
+
+/* ---------------------------------------------------------------------------------------------
+ * a1. Cache append (« L'idée : garder un résumé »; « L'obstacle : RoPE »).
+ * For each new token (b, t): z = x[b,t,:] · W where W = [W_DKV | W_KR] is [C, d_c + d_r];
+ *   c   = z[0:d_c] / sqrt(mean(z[0:d_c]^2) + rms_eps) * gamma      (gamma NULL means all ones)
+ *   k_r = RoPE(z[d_c:d_c+d_r], position)
+ * and writes c and k_r into the cache row of that token's position.
+ *   x       [B, s_q, C] dtype          w_dkv_kr [C, d_c + d_r] dtype      gamma [d_c] dtype or NULL
+ *   seqlens [B] int32                   block_table [B, max_pages] int32
+ * workspace: at least mla_append_workspace_size(...) bytes of device memory (fp32 partial sums);
+ * its contents need not be initialised.
+ * ------------------------------------------------------------------------------------------- */
+size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C);
+int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                     const void* x, int32_t C, const void* w_dkv_kr, const void* gamma,
+                     const int32_t* seqlens, const int32_t* block_table, int32_t max_pages,
+                     const mla_latent_cache_t* cache, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * a2. Query absorption (« Ce que DeepSeek fait de plus »: q·(W_UK c) = (q·W_UK)·c).
+ *   q_abs[b,t,h, 0:d_c]       = q_nope[b,t,h,:] · W_UK[h]            (W_UK[h] is [D, d_c])
+ *   q_abs[b,t,h, d_c:d_c+d_r] = RoPE(q_rope_raw[b,t,h,:], seqlens[b] - s_q + t)
+ *   q_nope [B, s_q, H, D]   q_rope_raw [B, s_q, H, d_r]   w_uk [H, D, d_c]   seqlens [B] int32
+ *   q_abs  [B, s_q, H, d_c + d_r]   (all dtype)
+ * ------------------------------------------------------------------------------------------- */
+int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                 const void* q_nope, const void* q_rope_raw, const void* w_uk,
+                 const int32_t* seqlens, void* q_abs, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * a3 + a4. Absorbed decode over the latent cache, split over the GPU's SMs, with the
+ * log-sum-exp merge of split sequences (« Chemin MQA-Absorbé »; « Le mécanisme d'attention »).
+ * For each (b, t, h), over the visible positions j:
+ *   s_j   = sm_scale * (q_abs[b,t,h,0:d_c] · c_j + q_abs[b,t,h,d_c:] · k_r,j)
+ *   o_lat[b,t,h,:] = sum_j softmax(s)_j * c_j          lse[b,t,h] = log sum_j exp(s_j)
+ *   q_abs [B, s_q, H, d_c + d_r] dtype    o_lat [B, s_q, H, d_c] dtype    lse [B, s_q, H] fp32
+ * workspace: at least mla_decode_workspace_size(...) bytes (split partials); no initialisation
+ * needed. The size depends on the current device's SM count and on max_pages (the longest
+ * sequence the table can describe is max_pages*64 positions).
+ * Requires every seqlens[b] >= s_q (a token always sees itself).
+ * ------------------------------------------------------------------------------------------- */
+size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                                 int32_t max_pages);
+int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                        const void* q_abs, const mla_latent_cache_t* cache,
+                        const int32_t* block_table, int32_t max_pages, const int32_t* seqlens,
+                        void* o_lat, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * a5. Output projection (« Ce que DeepSeek fait de plus »: the weighted latent sum is projected
+ * once by W_UV; « Le code »: the layer's final projection).
+ *   out[b,t,h,:] = o_lat[b,t,h,:] · W_UV[h]                   (W_UV[h] is [d_c, d_v])
+ *   if w_o != NULL: out_model[b,t,:] = concat_h(out[b,t,h,:]) · W_O   (W_O is [H*d_v, C])
+ *   o_lat [B, s_q, H, d_c]  w_uv [H, d_c, d_v]  out [B, s_q, H, d_v]  out_model [B, s_q, C] (dtype)
+ * ------------------------------------------------------------------------------------------- */
+int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                 const void* o_lat, const void* w_uv, void* out,
+                 const void* w_o, int32_t C, void* out_model, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * a6. GQLA grouped decode (« Résumé technique : GQLA … », « Architecture » and « Chemin GQA »).
+ * Head h uses group h / (H/g). For each (b, t, h) over the visible positions j:
+ *   s_j = sm_scale * (q_nope[b,t,h,:] · K[j, g(h), :] + RoPE(q_rope_raw[b,t,h,:], pos_t) · k_r,j)
+ *   out[b,t,h,:] = sum_j softmax(s)_j * V[j, g(h), :]          lse[b,t,h] = log sum_j exp(s_j)
+ *   q_nope [B, s_q, H, D]  q_rope_raw [B, s_q, H, d_r]  out [B, s_q, H, d_v] (dtype)  lse fp32
+ * workspace: at least mla_gqla_workspace_size(...) bytes.
+ * ------------------------------------------------------------------------------------------- */
+size_t mla_gqla_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                               int32_t max_pages);
+int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                            const void* q_nope, const void* q_rope_raw, const mla_gqa_cache_t* cache,
+                            const int32_t* block_table, int32_t max_pages, const int32_t* seqlens,
+                            void* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Status.
+ * mla_check_status: synchronises `stream`, returns the device status word of the current device
+ * (MLA_OK when no kernel recorded an error since the last call) and clears it.
+ * mla_status_string: a static, human-readable name of a status code.
+ * mla_build_info: a static string naming the build (target architecture, kernels compiled in).
+ * mla_launch_count: kernels this process has launched through the library so far (host counter,
+ * incremented at every launch; used to report how many kernels a timed region ran).
+ * ------------------------------------------------------------------------------------------- */
+int mla_check_status(void* stream);
+const char* mla_status_string(int status);
+const char* mla_build_info(void);
+uint64_t mla_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_H_ */

@@ -1,0 +1,78 @@
+// Device helpers shared by every kernel of libmla: storage-type conversion, the per-device status
+// word, RoPE angles and block reductions.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mla.h"
+
+namespace mla {
+
+// Per-device status word: the first error a kernel records wins; mla_check_status() clears it.
+__device__ int g_status;
+
+__device__ __forceinline__ void report(int code) { atomicCAS(&g_status, 0, code); }
+
+// ---- storage types ---------------------------------------------------------------------------
+template <typename T> struct Store;
+template <> struct Store<float> {
+  static __device__ __forceinline__ float load(const float* p) { return *p; }
+  static __device__ __forceinline__ void store(float* p, float v) { *p = v; }
+};
+template <> struct Store<__nv_bfloat16> {
+  static __device__ __forceinline__ float load(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+};
+template <typename T> __device__ __forceinline__ float ld(const T* p) { return Store<T>::load(p); }
+template <typename T> __device__ __forceinline__ void st(T* p, float v) { Store<T>::store(p, v); }
+
+// ---- RoPE ------------------------------------------------------------------------------------
+// Pair (2i, 2i+1) of a d_r vector turns by pos * base^(-2i/d_r). The angle is formed and reduced
+// in double precision: at pos ~ 1e5 an fp32 product would already be off by ~1e-2 rad.
+__device__ __forceinline__ void rope_cos_sin(int pos, int i, int d_r, float base, float* c, float* s) {
+  double theta = pow((double)base, -2.0 * (double)i / (double)d_r);
+  double sn, cs;
+  sincos((double)pos * theta, &sn, &cs);
+  *c = (float)cs;
+  *s = (float)sn;
+}
+
+// ---- reductions --------------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+// Sum over the whole block; `red` needs blockDim.x/32 floats of shared memory.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = (threadIdx.x < (unsigned)nw) ? red[threadIdx.x] : 0.f;
+  if (w == 0) t = warp_sum(t);
+  if (threadIdx.x == 0) red[0] = t;
+  __syncthreads();
+  return red[0];
+}
+
+// Page-table lookup with a range check: returns the pool row of position p, or -1 (and records
+// MLA_ERR_DEVICE_CHECK) when the page id is outside the pool.
+__device__ __forceinline__ int64_t cache_row(const int32_t* table_row, int p, int num_pages) {
+  int page = table_row[p >> 6];
+  if (page < 0 || page >= num_pages) {
+    report(MLA_ERR_DEVICE_CHECK);
+    return -1;
+  }
+  return (int64_t)page * 64 + (p & 63);
+}
+
+}  // namespace mla

@@ -1,0 +1,391 @@
+// Host entry points of libmla: argument validation, kernel selection by dtype and shape, launch.
+// Nothing here allocates, frees or synchronises (except mla_check_status, which reads the
+// device status word after synchronising the stream it is given).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <algorithm>
+#include <atomic>
+#include <utility>
+
+#include "mla.h"
+#include "common.cuh"
+#include "simt.cuh"
+#include "decode_sm100.cuh"
+
+namespace {
+
+using mla::simt::DecodeArgs;
+
+constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_launches{0};
+
+// Every kernel of the library is launched through here, so that the launches can be counted.
+template <typename... KArgs, typename... Args>
+void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  kernel<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+int num_sms() {
+  static int cached[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t esize(int32_t dtype) { return dtype == MLA_F32 ? 4 : 2; }
+inline bool stride_ok(int64_t stride, int32_t dtype, int64_t min_elems) {
+  return stride >= min_elems && ((stride * (int64_t)esize(dtype)) % 16) == 0;
+}
+
+int check_dims(const mla_dims_t* d) {
+  if (!d) return MLA_ERR_INVALID_ARG;
+  if (d->H <= 0 || d->D <= 0 || d->d_r <= 0 || (d->d_r & 1) || d->d_c <= 0 || d->d_v <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (d->page_size != 64) return MLA_ERR_INVALID_ARG;
+  if (!(d->sm_scale > 0.f) || !(d->rms_eps >= 0.f) || !(d->rope_base > 0.f)) return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+int check_dtype(int32_t dtype) { return (dtype == MLA_F32 || dtype == MLA_BF16) ? MLA_OK : MLA_ERR_INVALID_ARG; }
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+template <typename K>
+int set_smem(K kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return MLA_OK;
+  if (bytes > 227 * 1024) return MLA_ERR_UNSUPPORTED;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess
+             ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// ---- a1 split-K choice: enough blocks to cover the SMs about twice ----------------------------
+int append_ksplit(int n_tok, int K, int N) {
+  const int col_blocks = (N + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS;
+  const int tok_blocks = (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK;
+  const int base = col_blocks * tok_blocks;
+  int ks = (2 * num_sms() + base - 1) / base;
+  ks = std::max(1, std::min(ks, std::min(32, (K + 63) / 64)));
+  return ks;
+}
+
+// ---- a3 split choice for the CUDA-core decode ---------------------------------------------------
+struct SimtSplit { int nsplit, chunk; };
+SimtSplit simt_split(int n_tok, int H, int max_pages) {
+  const int max_len = max_pages * 64;
+  const int base = n_tok * (H / mla::simt::DEC_HEADS);
+  int ns = (4 * num_sms() + base - 1) / base;
+  ns = std::max(1, std::min(ns, std::max(1, max_len / 256)));
+  ns = std::min(ns, 64);
+  int chunk = (max_len + ns - 1) / ns;
+  chunk = (chunk + 31) / 32 * 32;
+  ns = (max_len + chunk - 1) / chunk;
+  return {ns, chunk};
+}
+
+size_t simt_decode_ws(int n_tok, int H, int Dv, int max_pages) {
+  SimtSplit s = simt_split(n_tok, H, max_pages);
+  if (s.nsplit <= 1) return 0;
+  const size_t slots = (size_t)n_tok * H * s.nsplit;
+  return slots * Dv * sizeof(float) + slots * sizeof(float) + 256;
+}
+
+template <typename T>
+int launch_decode_simt(DecodeArgs A, int n_tok, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int W = A.Dk + A.d_r;
+  const size_t smem = ((size_t)8 * W + (size_t)32 * (W + 1) + (A.kv_shared ? 0 : (size_t)32 * A.Dv) + 256) * 4 + 32 * 8;
+  int rc = set_smem(mla::simt::decode_simt_kernel<T>, smem);
+  if (rc) return rc;
+  if (A.nsplit > 1) {
+    const size_t slots = (size_t)n_tok * A.H * A.nsplit;
+    if (!ws || ws_bytes < slots * A.Dv * sizeof(float) + slots * sizeof(float)) return MLA_ERR_WORKSPACE;
+    A.part_o = reinterpret_cast<float*>(ws);
+    A.part_lse = A.part_o + slots * A.Dv;
+  }
+  dim3 grid(n_tok, A.H / mla::simt::DEC_HEADS, A.nsplit);
+  launch(mla::simt::decode_simt_kernel<T>, grid, 256, smem, st, A);
+  if (A.nsplit > 1) {
+    launch(mla::simt::merge_splits_kernel<T>, n_tok * A.H, 128, 0, st, 
+        A.part_o, A.part_lse, A.nsplit, A.Dv, reinterpret_cast<T*>(A.out), A.out_head_stride, A.lse);
+  }
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(int s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG: null pointer, bad size, misaligned pointer or stride";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: no kernel for this dtype/shape";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: workspace missing or too small";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA runtime call failed";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: a bounded wait inside a kernel gave up";
+    case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK: an index read on the device was out of range";
+    default: return "unknown mla status";
+  }
+}
+
+uint64_t mla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* mla_build_info(void) {
+  return "libmla: sm_100a; kernels: simt (fp32/bf16 all steps), sm100 absorbed decode (tcgen05/TMA)";
+}
+
+int mla_check_status(void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, mla::g_status, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(mla::g_status, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return v;
+}
+
+// ------------------------------------------------------------------------------------------------
+// a1
+// ------------------------------------------------------------------------------------------------
+size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C) {
+  if (check_dims(dims) || B <= 0 || s_q <= 0 || C <= 0) return 0;
+  const int n_tok = B * s_q, N = dims->d_c + dims->d_r;
+  return (size_t)append_ksplit(n_tok, C, N) * n_tok * N * sizeof(float);
+}
+
+int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x,
+                     int32_t C, const void* w_dkv_kr, const void* gamma, const int32_t* seqlens,
+                     const int32_t* block_table, int32_t max_pages, const mla_latent_cache_t* cache,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (B <= 0 || s_q <= 0 || C <= 0 || max_pages <= 0 || !x || !w_dkv_kr || !seqlens || !block_table || !cache)
+    return MLA_ERR_INVALID_ARG;
+  if (!cache->latent || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_dkv_kr) || (gamma && !aligned16(gamma)) || !aligned16(cache->latent) ||
+      !aligned16(cache->rope) || !aligned16(seqlens) || !aligned16(block_table))
+    return MLA_ERR_INVALID_ARG;
+  if (!stride_ok(cache->latent_stride, dtype, dims->d_c) || !stride_ok(cache->rope_stride, dtype, dims->d_r))
+    return MLA_ERR_INVALID_ARG;
+  const int n_tok = B * s_q, N = dims->d_c + dims->d_r;
+  const int ks = append_ksplit(n_tok, C, N);
+  const size_t need = (size_t)ks * n_tok * N * sizeof(float);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
+  dim3 grid((N + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS,
+            (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK, ks);
+  float* part = reinterpret_cast<float*>(workspace);
+  const size_t fin_smem = (size_t)N * sizeof(float);
+  if (dtype == MLA_F32) {
+    using T = float;
+    launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, 
+        (const T*)x, n_tok, C, (const T*)w_dkv_kr, N, k_chunk, part, nullptr);
+    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
+    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, 
+        part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
+        block_table, max_pages, (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride,
+        cache->num_pages);
+  } else {
+    using T = __nv_bfloat16;
+    launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, 
+        (const T*)x, n_tok, C, (const T*)w_dkv_kr, N, k_chunk, part, nullptr);
+    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
+    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, 
+        part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
+        block_table, max_pages, (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride,
+        cache->num_pages);
+  }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------------------------------------
+// a2
+// ------------------------------------------------------------------------------------------------
+int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_nope,
+                 const void* q_rope_raw, const void* w_uk, const int32_t* seqlens, void* q_abs, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (B <= 0 || s_q <= 0 || !q_nope || !q_rope_raw || !w_uk || !seqlens || !q_abs) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || !aligned16(q_rope_raw) || !aligned16(w_uk) || !aligned16(q_abs) || !aligned16(seqlens))
+    return MLA_ERR_INVALID_ARG;
+  const int n_tok = B * s_q;
+  const int D = dims->D, H = dims->H, d_c = dims->d_c, d_r = dims->d_r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  dim3 grid(H, (n_tok + mla::simt::HG_TOK - 1) / mla::simt::HG_TOK);
+  const size_t smem = (size_t)mla::simt::HG_TOK * D * sizeof(float);
+  if (dtype == MLA_F32) {
+    using T = float;
+    if ((rc = set_smem(mla::simt::head_gemm_kernel<T>, smem))) return rc;
+    launch(mla::simt::head_gemm_kernel<T>, grid, 128, smem, st, 
+        (const T*)q_nope, D, D, (const T*)w_uk, d_c, n_tok, H, (T*)q_abs, d_c + d_r, (const T*)q_rope_raw, d_r,
+        seqlens, s_q, dims->rope_base);
+  } else {
+    using T = __nv_bfloat16;
+    if ((rc = set_smem(mla::simt::head_gemm_kernel<T>, smem))) return rc;
+    launch(mla::simt::head_gemm_kernel<T>, grid, 128, smem, st, 
+        (const T*)q_nope, D, D, (const T*)w_uk, d_c, n_tok, H, (T*)q_abs, d_c + d_r, (const T*)q_rope_raw, d_r,
+        seqlens, s_q, dims->rope_base);
+  }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------------------------------------
+// a3 + a4
+// ------------------------------------------------------------------------------------------------
+size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, int32_t max_pages) {
+  if (check_dims(dims) || check_dtype(dtype) || B <= 0 || s_q <= 0 || max_pages <= 0) return 0;
+  size_t ws = simt_decode_ws(B * s_q, dims->H, dims->d_c, max_pages);
+  ws = std::max(ws, mla::sm100::decode_workspace_bytes(dims, dtype, B, s_q, num_sms()));
+  return ws;
+}
+
+int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_abs,
+                        const mla_latent_cache_t* cache, const int32_t* block_table, int32_t max_pages,
+                        const int32_t* seqlens, void* o_lat, float* lse, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (B <= 0 || s_q <= 0 || max_pages <= 0 || !q_abs || !cache || !block_table || !seqlens || !o_lat || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if (!cache->latent || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_abs) || !aligned16(cache->latent) || !aligned16(cache->rope) || !aligned16(block_table) ||
+      !aligned16(seqlens) || !aligned16(o_lat) || !aligned16(lse) || (workspace && !aligned16(workspace)))
+    return MLA_ERR_INVALID_ARG;
+  if (!stride_ok(cache->latent_stride, dtype, dims->d_c) || !stride_ok(cache->rope_stride, dtype, dims->d_r))
+    return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int n_tok = B * s_q;
+
+  if (mla::sm100::decode_supported(dims, dtype, B, s_q)) {
+    return mla::sm100::launch_decode(dims, B, s_q, q_abs, cache, block_table, max_pages, seqlens, o_lat, lse,
+                                     workspace, ws_bytes, num_sms(), st);
+  }
+
+  if (dims->H % mla::simt::DEC_HEADS || dims->d_c % 32 || dims->d_c > 32 * mla::simt::DEC_MAX_OV)
+    return MLA_ERR_UNSUPPORTED;
+  DecodeArgs A{};
+  A.q = q_abs;
+  A.q_head_stride = dims->d_c + dims->d_r;
+  A.q_rope_raw = nullptr;
+  A.kpart = cache->latent; A.k_stride = cache->latent_stride; A.k_group_off = 0;
+  A.vpart = cache->latent; A.v_stride = cache->latent_stride; A.v_group_off = 0;
+  A.rope = cache->rope; A.rope_stride = cache->rope_stride;
+  A.Dk = dims->d_c; A.Dv = dims->d_c; A.d_r = dims->d_r; A.H = dims->H; A.heads_per_group = dims->H;
+  A.kv_shared = 1;
+  A.block_table = block_table; A.max_pages = max_pages; A.num_pages = cache->num_pages;
+  A.seqlens = seqlens; A.s_q = s_q; A.sm_scale = dims->sm_scale; A.rope_base = dims->rope_base;
+  A.out = o_lat; A.out_head_stride = dims->d_c; A.lse = lse;
+  SimtSplit sp = simt_split(n_tok, dims->H, max_pages);
+  A.nsplit = sp.nsplit; A.chunk = sp.chunk;
+  return dtype == MLA_F32 ? launch_decode_simt<float>(A, n_tok, workspace, ws_bytes, st)
+                          : launch_decode_simt<__nv_bfloat16>(A, n_tok, workspace, ws_bytes, st);
+}
+
+// ------------------------------------------------------------------------------------------------
+// a5
+// ------------------------------------------------------------------------------------------------
+int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* o_lat,
+                 const void* w_uv, void* out, const void* w_o, int32_t C, void* out_model, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (B <= 0 || s_q <= 0 || !o_lat || !w_uv || !out) return MLA_ERR_INVALID_ARG;
+  if (w_o && (C <= 0 || !out_model)) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o_lat) || !aligned16(w_uv) || !aligned16(out) || (w_o && (!aligned16(w_o) || !aligned16(out_model))))
+    return MLA_ERR_INVALID_ARG;
+  const int n_tok = B * s_q;
+  const int H = dims->H, d_c = dims->d_c, d_v = dims->d_v;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  dim3 grid(H, (n_tok + mla::simt::HG_TOK - 1) / mla::simt::HG_TOK);
+  const size_t smem = (size_t)mla::simt::HG_TOK * d_c * sizeof(float);
+  dim3 ogrid((C + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS, (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK, 1);
+  const int K = H * d_v;
+  if (dtype == MLA_F32) {
+    using T = float;
+    if ((rc = set_smem(mla::simt::head_gemm_kernel<T>, smem))) return rc;
+    launch(mla::simt::head_gemm_kernel<T>, grid, 128, smem, st, (const T*)o_lat, d_c, d_c, (const T*)w_uv, d_v, n_tok, H,
+                                                            (T*)out, d_v, nullptr, 0, nullptr, 1, 0.f);
+    if (w_o)
+      launch(mla::simt::proj_partial_kernel<T>, ogrid, mla::simt::PROJ_COLS, 0, st, (const T*)out, n_tok, K, (const T*)w_o,
+                                                                               C, K, nullptr, (T*)out_model);
+  } else {
+    using T = __nv_bfloat16;
+    if ((rc = set_smem(mla::simt::head_gemm_kernel<T>, smem))) return rc;
+    launch(mla::simt::head_gemm_kernel<T>, grid, 128, smem, st, (const T*)o_lat, d_c, d_c, (const T*)w_uv, d_v, n_tok, H,
+                                                            (T*)out, d_v, nullptr, 0, nullptr, 1, 0.f);
+    if (w_o)
+      launch(mla::simt::proj_partial_kernel<T>, ogrid, mla::simt::PROJ_COLS, 0, st, (const T*)out, n_tok, K, (const T*)w_o,
+                                                                               C, K, nullptr, (T*)out_model);
+  }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------------------------------------
+// a6
+// ------------------------------------------------------------------------------------------------
+size_t mla_gqla_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, int32_t max_pages) {
+  if (check_dims(dims) || check_dtype(dtype) || B <= 0 || s_q <= 0 || max_pages <= 0) return 0;
+  return simt_decode_ws(B * s_q, dims->H, dims->d_v, max_pages);
+}
+
+int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_nope,
+                            const void* q_rope_raw, const mla_gqa_cache_t* cache, const int32_t* block_table,
+                            int32_t max_pages, const int32_t* seqlens, void* out, float* lse, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (dims->g <= 0 || dims->H % dims->g) return MLA_ERR_INVALID_ARG;
+  if (B <= 0 || s_q <= 0 || max_pages <= 0 || !q_nope || !q_rope_raw || !cache || !block_table || !seqlens ||
+      !out || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if (!cache->k || !cache->v || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || !aligned16(q_rope_raw) || !aligned16(cache->k) || !aligned16(cache->v) ||
+      !aligned16(cache->rope) || !aligned16(block_table) || !aligned16(seqlens) || !aligned16(out) ||
+      !aligned16(lse) || (workspace && !aligned16(workspace)))
+    return MLA_ERR_INVALID_ARG;
+  const int hpg = dims->H / dims->g;
+  if (!stride_ok(cache->k_stride, dtype, (int64_t)dims->g * dims->D) ||
+      !stride_ok(cache->v_stride, dtype, (int64_t)dims->g * dims->d_v) || !stride_ok(cache->rope_stride, dtype, dims->d_r))
+    return MLA_ERR_INVALID_ARG;
+  if (hpg % mla::simt::DEC_HEADS || dims->d_v % 32 || dims->d_v > 32 * mla::simt::DEC_MAX_OV) return MLA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int n_tok = B * s_q;
+  DecodeArgs A{};
+  A.q = q_nope;
+  A.q_head_stride = dims->D;
+  A.q_rope_raw = q_rope_raw;
+  A.kpart = cache->k; A.k_stride = cache->k_stride; A.k_group_off = dims->D;
+  A.vpart = cache->v; A.v_stride = cache->v_stride; A.v_group_off = dims->d_v;
+  A.rope = cache->rope; A.rope_stride = cache->rope_stride;
+  A.Dk = dims->D; A.Dv = dims->d_v; A.d_r = dims->d_r; A.H = dims->H; A.heads_per_group = hpg;
+  A.kv_shared = 0;
+  A.block_table = block_table; A.max_pages = max_pages; A.num_pages = cache->num_pages;
+  A.seqlens = seqlens; A.s_q = s_q; A.sm_scale = dims->sm_scale; A.rope_base = dims->rope_base;
+  A.out = out; A.out_head_stride = dims->d_v; A.lse = lse;
+  SimtSplit sp = simt_split(n_tok, dims->H, max_pages);
+  A.nsplit = sp.nsplit; A.chunk = sp.chunk;
+  return dtype == MLA_F32 ? launch_decode_simt<float>(A, n_tok, workspace, ws_bytes, st)
+                          : launch_decode_simt<__nv_bfloat16>(A, n_tok, workspace, ws_bytes, st);
+}
+
+}  // extern "C"

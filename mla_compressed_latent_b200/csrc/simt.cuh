@@ -1,0 +1,338 @@
+// CUDA-core kernels (fp32 arithmetic) for every step of one decode step: the fp32 workloads run
+// on them, and so does every shape the tensor-core kernels do not cover.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+namespace simt {
+
+// =============================================================================================
+// Dense projection z = x · W, split over K: part[ks][n][col] = sum_{k in slice ks} x[n][k] W[k][col].
+// One thread per output column, PROJ_TOK tokens per block; W rows are read coalesced.
+// With out != nullptr (and one slice) the result is written in storage type instead.
+// =============================================================================================
+constexpr int PROJ_COLS = 128;
+constexpr int PROJ_TOK = 8;
+constexpr int PROJ_KT = 64;
+
+template <typename T>
+__global__ void __launch_bounds__(PROJ_COLS)
+proj_partial_kernel(const T* __restrict__ x, int n_tok, int K, const T* __restrict__ W, int N,
+                    int k_chunk, float* __restrict__ part, T* __restrict__ out) {
+  __shared__ float xs[PROJ_TOK][PROJ_KT];
+  const int col = blockIdx.x * PROJ_COLS + threadIdx.x;
+  const int tok0 = blockIdx.y * PROJ_TOK;
+  const int ks = blockIdx.z;
+  const int k_lo = ks * k_chunk;
+  const int k_hi = min(K, k_lo + k_chunk);
+  float acc[PROJ_TOK];
+#pragma unroll
+  for (int t = 0; t < PROJ_TOK; ++t) acc[t] = 0.f;
+  for (int kb = k_lo; kb < k_hi; kb += PROJ_KT) {
+    for (int i = threadIdx.x; i < PROJ_TOK * PROJ_KT; i += blockDim.x) {
+      const int tt = i / PROJ_KT, kk = i % PROJ_KT;
+      const int tok = tok0 + tt, k = kb + kk;
+      xs[tt][kk] = (tok < n_tok && k < k_hi) ? ld(x + (int64_t)tok * K + k) : 0.f;
+    }
+    __syncthreads();
+    if (col < N) {
+      const int kn = min(PROJ_KT, k_hi - kb);
+      for (int kk = 0; kk < kn; ++kk) {
+        const float w = ld(W + (int64_t)(kb + kk) * N + col);
+#pragma unroll
+        for (int t = 0; t < PROJ_TOK; ++t) acc[t] = fmaf(xs[t][kk], w, acc[t]);
+      }
+    }
+    __syncthreads();
+  }
+  if (col >= N) return;
+#pragma unroll
+  for (int t = 0; t < PROJ_TOK; ++t) {
+    const int tok = tok0 + t;
+    if (tok >= n_tok) break;
+    if (out) st(out + (int64_t)tok * N + col, acc[t]);
+    else part[((int64_t)ks * n_tok + tok) * N + col] = acc[t];
+  }
+}
+
+// =============================================================================================
+// a1 epilogue: sum the K slices, RMSNorm the latent part, rotate the RoPE part, store the row.
+// One block per new token.
+// =============================================================================================
+template <typename T>
+__global__ void append_finish_kernel(const float* __restrict__ part, int ksplit, int n_tok, int s_q,
+                                     int d_c, int d_r, const T* __restrict__ gamma, float eps,
+                                     float rope_base, const int32_t* __restrict__ seqlens,
+                                     const int32_t* __restrict__ block_table, int max_pages,
+                                     T* latent, int64_t lat_stride, T* rope, int64_t rope_stride,
+                                     int num_pages) {
+  extern __shared__ float z[];
+  __shared__ float red[32];
+  const int tok = blockIdx.x;
+  const int b = tok / s_q, t = tok % s_q;
+  const int N = d_c + d_r;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    float s = 0.f;
+    for (int ks = 0; ks < ksplit; ++ks) s += part[((int64_t)ks * n_tok + tok) * N + i];
+    z[i] = s;
+  }
+  __syncthreads();
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d_c; i += blockDim.x) ss = fmaf(z[i], z[i], ss);
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)d_c + eps);
+  const int pos = seqlens[b] - s_q + t;
+  if (pos < 0 || (pos >> 6) >= max_pages) {
+    if (threadIdx.x == 0) report(MLA_ERR_DEVICE_CHECK);
+    return;
+  }
+  const int64_t row = cache_row(block_table + (int64_t)b * max_pages, pos, num_pages);
+  if (row < 0) return;
+  for (int i = threadIdx.x; i < d_c; i += blockDim.x) {
+    const float gm = gamma ? ld(gamma + i) : 1.f;
+    st(latent + row * lat_stride + i, z[i] * inv * gm);
+  }
+  for (int i = threadIdx.x; i < d_r / 2; i += blockDim.x) {
+    float cs, sn;
+    rope_cos_sin(pos, i, d_r, rope_base, &cs, &sn);
+    const float a = z[d_c + 2 * i], bb = z[d_c + 2 * i + 1];
+    st(rope + row * rope_stride + 2 * i, a * cs - bb * sn);
+    st(rope + row * rope_stride + 2 * i + 1, a * sn + bb * cs);
+  }
+}
+
+// =============================================================================================
+// Per-head small GEMM: y[tok, h, :] = a[tok, h, :] · Wh[h]   (a row K wide, Wh[h] is [K, N]).
+// Used for a2 (a = q_nope, W = W_UK, N = d_c) and a5 (a = o_lat, W = W_UV, N = d_v).
+// Optional RoPE tail for a2: y[tok, h, N + 2i..] = RoPE(r[tok, h, :], pos).
+// =============================================================================================
+constexpr int HG_TOK = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(128)
+head_gemm_kernel(const T* __restrict__ a, int64_t a_head_stride, int K, const T* __restrict__ Wh,
+                 int N, int n_tok, int H, T* __restrict__ y, int64_t y_head_stride,
+                 const T* __restrict__ rope_raw, int d_r, const int32_t* __restrict__ seqlens,
+                 int s_q, float rope_base) {
+  extern __shared__ float as[];  // [HG_TOK][K]
+  const int h = blockIdx.x;
+  const int tok0 = blockIdx.y * HG_TOK;
+  for (int i = threadIdx.x; i < HG_TOK * K; i += blockDim.x) {
+    const int tt = i / K, k = i % K;
+    const int tok = tok0 + tt;
+    as[i] = (tok < n_tok) ? ld(a + ((int64_t)tok * H + h) * a_head_stride + k) : 0.f;
+  }
+  __syncthreads();
+  const T* W = Wh + (int64_t)h * K * N;
+  for (int c = threadIdx.x; c < N; c += blockDim.x) {
+    float acc[HG_TOK];
+#pragma unroll
+    for (int t = 0; t < HG_TOK; ++t) acc[t] = 0.f;
+    for (int k = 0; k < K; ++k) {
+      const float w = ld(W + (int64_t)k * N + c);
+#pragma unroll
+      for (int t = 0; t < HG_TOK; ++t) acc[t] = fmaf(as[t * K + k], w, acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < HG_TOK; ++t) {
+      const int tok = tok0 + t;
+      if (tok < n_tok) st(y + ((int64_t)tok * H + h) * y_head_stride + c, acc[t]);
+    }
+  }
+  if (rope_raw == nullptr) return;
+  const int half = d_r / 2;
+  for (int i = threadIdx.x; i < HG_TOK * half; i += blockDim.x) {
+    const int tt = i / half, p = i % half;
+    const int tok = tok0 + tt;
+    if (tok >= n_tok) continue;
+    const int pos = seqlens[tok / s_q] - s_q + tok % s_q;
+    float cs, sn;
+    rope_cos_sin(pos, p, d_r, rope_base, &cs, &sn);
+    const T* r = rope_raw + ((int64_t)tok * H + h) * d_r;
+    const float x0 = ld(r + 2 * p), x1 = ld(r + 2 * p + 1);
+    T* o = y + ((int64_t)tok * H + h) * y_head_stride + N;
+    st(o + 2 * p, x0 * cs - x1 * sn);
+    st(o + 2 * p + 1, x0 * sn + x1 * cs);
+  }
+}
+
+// =============================================================================================
+// a3 / a6: split-KV flash-decoding on CUDA cores, generic over the absorbed and grouped paths.
+// Key of row j = [kpart_j (Dk) ; rope_j (d_r)], value = vpart_j (Dv). For the absorbed path
+// kpart and vpart are the same latent row (Dk = Dv = d_c) and the query is q_abs; for the grouped
+// path they are the group's K and V rows and the query's RoPE part is rotated here.
+// Block = 8 heads (one warp each) x 32 positions per tile; online softmax per head.
+// =============================================================================================
+constexpr int DEC_HEADS = 8;
+constexpr int DEC_TILE = 32;
+constexpr int DEC_MAX_OV = 16;  // Dv <= 512
+
+struct DecodeArgs {
+  const void* q;           // [n_tok, H, q_head_stride]: Dk query part, then d_r RoPE part (absorbed)
+  int64_t q_head_stride;
+  const void* q_rope_raw;  // grouped path: [n_tok, H, d_r] un-rotated; nullptr for absorbed
+  const void* kpart; int64_t k_stride; int64_t k_group_off;
+  const void* vpart; int64_t v_stride; int64_t v_group_off;
+  const void* rope; int64_t rope_stride;
+  int Dk, Dv, d_r, H, heads_per_group;
+  int kv_shared;           // vpart rows are the kpart rows (absorbed)
+  const int32_t* block_table; int max_pages; int num_pages;
+  const int32_t* seqlens; int s_q;
+  float sm_scale, rope_base;
+  void* out; int64_t out_head_stride; float* lse;
+  float* part_o; float* part_lse; int nsplit; int chunk;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+decode_simt_kernel(DecodeArgs A) {
+  extern __shared__ float sm[];
+  const int W = A.Dk + A.d_r;
+  const int WP = W + 1;  // padded key row: conflict-free column reads
+  float* qs = sm;                              // [8][W]
+  float* ks = qs + DEC_HEADS * W;              // [32][WP]
+  float* vs = A.kv_shared ? ks : ks + DEC_TILE * WP;   // [32][Dv] (or aliases ks)
+  float* ps = ks + DEC_TILE * WP + (A.kv_shared ? 0 : DEC_TILE * A.Dv);  // [8][32]
+  int64_t* rows = reinterpret_cast<int64_t*>(ps + DEC_HEADS * DEC_TILE);  // [32]
+
+  const int tok = blockIdx.x;
+  const int h0 = blockIdx.y * DEC_HEADS;
+  const int split = blockIdx.z;
+  const int b = tok / A.s_q, t = tok % A.s_q;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = h0 + warp;
+  const int grp = h0 / A.heads_per_group;      // all 8 heads of a block share one group
+  const int L = A.seqlens[b];
+  const int n_vis = L - A.s_q + t + 1;
+  const int lo = split * A.chunk;
+  const int hi = min(n_vis, lo + A.chunk);
+  const int32_t* table = A.block_table + (int64_t)b * A.max_pages;
+  if (n_vis < 1 || (L > 0 && ((L - 1) >> 6) >= A.max_pages)) {
+    if (threadIdx.x == 0 && split == 0 && blockIdx.y == 0) report(MLA_ERR_DEVICE_CHECK);
+    return;
+  }
+
+  // query rows of the 8 heads (fp32), RoPE part rotated here for the grouped path
+  const T* q = reinterpret_cast<const T*>(A.q);
+  for (int i = threadIdx.x; i < DEC_HEADS * W; i += blockDim.x) {
+    const int hh = i / W, d = i % W;
+    const int64_t base = ((int64_t)tok * A.H + h0 + hh) * A.q_head_stride;
+    if (A.q_rope_raw == nullptr || d < A.Dk) {
+      qs[i] = ld(q + base + d);
+    } else {
+      const int p = (d - A.Dk) >> 1;
+      const T* r = reinterpret_cast<const T*>(A.q_rope_raw) + ((int64_t)tok * A.H + h0 + hh) * A.d_r;
+      float cs, sn;
+      rope_cos_sin(L - A.s_q + t, p, A.d_r, A.rope_base, &cs, &sn);
+      const float x0 = ld(r + 2 * p), x1 = ld(r + 2 * p + 1);
+      qs[i] = ((d - A.Dk) & 1) ? (x0 * sn + x1 * cs) : (x0 * cs - x1 * sn);
+    }
+  }
+
+  const int nov = A.Dv / 32;
+  float o[DEC_MAX_OV];
+#pragma unroll
+  for (int k = 0; k < DEC_MAX_OV; ++k) o[k] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  const T* kp = reinterpret_cast<const T*>(A.kpart);
+  const T* vp = reinterpret_cast<const T*>(A.vpart);
+  const T* rp = reinterpret_cast<const T*>(A.rope);
+
+  for (int p0 = lo; p0 < hi; p0 += DEC_TILE) {
+    __syncthreads();
+    if (threadIdx.x < DEC_TILE) {
+      const int p = p0 + threadIdx.x;
+      rows[threadIdx.x] = (p < hi) ? cache_row(table, p, A.num_pages) : -1;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < DEC_TILE * W; i += blockDim.x) {
+      const int r = i / W, d = i % W;
+      const int64_t row = rows[r];
+      float v = 0.f;
+      if (row >= 0) {
+        v = (d < A.Dk) ? ld(kp + row * A.k_stride + grp * A.k_group_off + d)
+                       : ld(rp + row * A.rope_stride + (d - A.Dk));
+      }
+      ks[r * WP + d] = v;
+    }
+    if (!A.kv_shared) {
+      for (int i = threadIdx.x; i < DEC_TILE * A.Dv; i += blockDim.x) {
+        const int r = i / A.Dv, d = i % A.Dv;
+        const int64_t row = rows[r];
+        vs[i] = (row >= 0) ? ld(vp + row * A.v_stride + grp * A.v_group_off + d) : 0.f;
+      }
+    }
+    __syncthreads();
+    // score of (head = warp, position = lane)
+    float s = -INFINITY;
+    if (rows[lane] >= 0) {
+      const float* qh = qs + warp * W;
+      const float* kr = ks + lane * WP;
+      float acc = 0.f;
+      for (int d = 0; d < W; ++d) acc = fmaf(qh[d], kr[d], acc);
+      s = acc * A.sm_scale;
+    }
+    const float m_tile = warp_max(s);
+    const float m_new = fmaxf(m_run, m_tile);
+    const float alpha = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);
+    const float pj = (s == -INFINITY) ? 0.f : expf(s - m_new);
+    l_run = l_run * alpha + warp_sum(pj);
+    m_run = m_new;
+    ps[warp * DEC_TILE + lane] = pj;
+    __syncwarp();
+    const int vstride = A.kv_shared ? WP : A.Dv;
+#pragma unroll
+    for (int k = 0; k < DEC_MAX_OV; ++k) {
+      if (k < nov) {
+        float acc = o[k] * alpha;
+        const int d = lane + 32 * k;
+        for (int j = 0; j < DEC_TILE; ++j) acc = fmaf(ps[warp * DEC_TILE + j], vs[j * vstride + d], acc);
+        o[k] = acc;
+      }
+    }
+  }
+
+  const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+  const float lse = (l_run > 0.f) ? m_run + logf(l_run) : -INFINITY;
+  if (A.nsplit == 1) {
+    T* out = reinterpret_cast<T*>(A.out) + ((int64_t)tok * A.H + h) * A.out_head_stride;
+#pragma unroll
+    for (int k = 0; k < DEC_MAX_OV; ++k)
+      if (k < nov) st(out + lane + 32 * k, o[k] * inv_l);
+    if (lane == 0) A.lse[(int64_t)tok * A.H + h] = lse;
+  } else {
+    const int64_t slot = ((int64_t)tok * A.H + h) * A.nsplit + split;
+    float* po = A.part_o + slot * A.Dv;
+#pragma unroll
+    for (int k = 0; k < DEC_MAX_OV; ++k)
+      if (k < nov) po[lane + 32 * k] = o[k] * inv_l;
+    if (lane == 0) A.part_lse[slot] = lse;
+  }
+}
+
+// a4: combine the split partials of every (token, head): weights exp(lse_s - LSE).
+template <typename T>
+__global__ void merge_splits_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                                    int nsplit, int Dv, T* __restrict__ out, int64_t out_head_stride,
+                                    float* __restrict__ lse_out) {
+  const int64_t th = blockIdx.x;  // token * H + head
+  const float* pl = part_lse + th * nsplit;
+  float m = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) m = fmaxf(m, pl[s]);
+  float tot = 0.f;
+  for (int s = 0; s < nsplit; ++s) tot += (pl[s] == -INFINITY) ? 0.f : expf(pl[s] - m);
+  const float inv = 1.f / tot;
+  for (int d = threadIdx.x; d < Dv; d += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+      if (pl[s] == -INFINITY) continue;
+      acc = fmaf(expf(pl[s] - m), part_o[(th * nsplit + s) * Dv + d], acc);
+    }
+    st(out + th * out_head_stride + d, acc * inv);
+  }
+  if (threadIdx.x == 0) lse_out[th] = m + logf(tot);
+}
+
+}  // namespace simt
+}  // namespace mla

@@ -185,13 +185,24 @@ def decode_step_inputs(w: Workload) -> dict:
     """This step's inputs: hidden states of the new tokens and their query parts.
 
     x [B, s_q, C]; q_nope [B, s_q, H, D]; q_rope_raw [B, s_q, H, d_r] (before rotation).
+    q_abs [B, s_q, H, d_c + d_r] is a query already in latent space, for checks of the decode kernel
+    on its own: the latent part is N(0, D/d_c) (the law of q_nope·W_UK[h] for |q_nope|² = D and
+    W_UK ~ N(0, 1/d_c)), the RoPE part N(0, 1). o_lat [B, s_q, H, d_c] ~ N(0, 1) feeds the output
+    projection on its own.
     """
     rng = _rng(SEED_DECODE)
-    return {
+    out = {
         "x": _normal(rng, (w.B, w.s_q, w.C), 1.0),
         "q_nope": _normal(rng, (w.B, w.s_q, w.H, w.D), 1.0),
         "q_rope_raw": _normal(rng, (w.B, w.s_q, w.H, w.d_r), 1.0),
     }
+    rng2 = _rng(SEED_DECODE, 1)
+    q_abs = np.empty((w.B, w.s_q, w.H, w.d_c + w.d_r), dtype=np.float32)
+    q_abs[..., :w.d_c] = _normal(rng2, (w.B, w.s_q, w.H, w.d_c), math.sqrt(w.D / w.d_c))
+    q_abs[..., w.d_c:] = _normal(rng2, (w.B, w.s_q, w.H, w.d_r), 1.0)
+    out["q_abs"] = q_abs
+    out["o_lat"] = _normal(rng2, (w.B, w.s_q, w.H, w.d_c), 1.0)
+    return out
 
 
 def context_hidden_states(w: Workload, L: int, b: int = 0) -> np.ndarray:

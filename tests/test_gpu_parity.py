@@ -1,0 +1,367 @@
+"""GPU parity: every C-ABI call against the fp64 oracle on the same seeded, stored inputs.
+
+Tolerances (the project's numeric bar): fp32 max|Δ| <= 1e-5·max|ref|; bf16 storage with fp32
+accumulation max|Δ| <= 2e-2·max|ref| and |Δ lse| <= 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import mla_oracle as O
+from mla_compressed_latent_b200 import _lib as L
+from mla_compressed_latent_b200 import ops
+from mla_compressed_latent_b200.ops import Dims, LatentCache, GqaCache
+
+from _cases import TOL, Case, max_rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def _cache(dev, case):
+    pool = dev["pool"]
+    d_c = case.w.d_c
+    return LatentCache(pool[:, :d_c], pool[:, d_c:], case.num_pages)
+
+
+def _oracle_absorbed(case, q_abs64, pool=None, heads=None, seqs=None):
+    """fp64 absorbed decode of the given sequences (all by default) and heads."""
+    w = case.w
+    seqs = range(w.B) if seqs is None else seqs
+    o, l = {}, {}
+    for b in seqs:
+        c, kr = case.seq_rows64(b, pool)
+        q = q_abs64[b] if heads is None else q_abs64[b][:, heads]
+        o[b], l[b] = O.absorbed_decode(q, c, kr, int(case.lens[b]), w.sm_scale)
+    return o, l
+
+
+def _assert_close(got, ref, dtype, what, key="out"):
+    err = max_rel_err(got, ref)
+    assert err <= TOL[dtype][key], f"{what}: max|Δ|/max|ref| = {err:.3e}"
+    return err
+
+
+def _assert_lse(got, ref, dtype, what):
+    err = float(np.abs(np.asarray(got, np.float64) - ref).max())
+    bar = TOL[dtype]["lse"] * (1 if dtype == "bf16" else max(1.0, float(np.abs(ref).max())))
+    assert err <= bar, f"{what}: max|Δ lse| = {err:.3e}"
+
+
+# ------------------------------------------------------------------------------------------------
+# a3 + a4 on their own: decode over a stored cache with a stored absorbed query
+# ------------------------------------------------------------------------------------------------
+
+SMALL_DECODE = [
+    # (lens, s_q, pages)
+    ([1], 1, "contiguous"),
+    ([63], 1, "contiguous"),
+    ([64, 65], 1, "random"),
+    ([127, 1000, 3], 1, "random"),
+    ([4096, 129, 2049, 64, 5000], 1, "contiguous"),
+    ([2, 64, 77, 300], 2, "random"),
+    ([4, 513, 1029], 4, "random"),
+]
+
+
+@pytest.mark.parametrize("lens,s_q,pages", SMALL_DECODE)
+def test_decode_absorbed_small(lens, s_q, pages):
+    w = synth.workload("dsv3_b64_l4096", B=len(lens), s_q=s_q, lengths=("list", tuple(lens)), pages=pages)
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    dims = Dims.of(w)
+    o_lat, lse = ops.mla_decode_absorbed(dims, dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    ref_o, ref_l = _oracle_absorbed(case, case.q_abs64)
+    got_o = o_lat.float().cpu().numpy()
+    got_l = lse.cpu().numpy()
+    for b in range(w.B):
+        _assert_close(got_o[b], ref_o[b], "bf16", f"o_lat seq {b}")
+        _assert_lse(got_l[b], ref_l[b], "bf16", f"lse seq {b}")
+
+
+def test_decode_absorbed_fp32_smallem_shapes():
+    w = synth.workload("smallem_fp32", B=3, lengths=("list", (512, 65, 1)))
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    o_lat, lse = ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"])
+    ref_o, ref_l = _oracle_absorbed(case, case.q_abs64)
+    for b in range(w.B):
+        _assert_close(o_lat[b].cpu().numpy(), ref_o[b], "f32", f"o_lat seq {b}")
+        _assert_lse(lse[b].cpu().numpy(), ref_l[b], "f32", f"lse seq {b}")
+
+
+@pytest.mark.parametrize("name", ["dsv3_b64_l4096", "longctx_b8"])
+def test_decode_absorbed_full_size(name):
+    """Full size, the bench's launch configuration; oracle on every sequence (sampled heads for the
+    long-context case, every head otherwise)."""
+    w = synth.workload(name)
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    o_lat, lse = ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    heads = None if name == "dsv3_b64_l4096" else np.random.default_rng(7).choice(w.H, 12, replace=False)
+    ref_o, ref_l = _oracle_absorbed(case, case.q_abs64, heads=heads)
+    got_o = o_lat.float().cpu().numpy()
+    got_l = lse.cpu().numpy()
+    for b in range(w.B):
+        go = got_o[b] if heads is None else got_o[b][:, heads]
+        gl = got_l[b] if heads is None else got_l[b][:, heads]
+        _assert_close(go, ref_o[b], "bf16", f"o_lat seq {b}")
+        _assert_lse(gl, ref_l[b], "bf16", f"lse seq {b}")
+
+
+def test_decode_mtp_random_pages_full_size_sampled():
+    """Multi-token step, random page table, full batch; oracle on a seeded sample of sequences."""
+    w = synth.workload("mtp_sq2_b128")
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    o_lat, lse = ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    seqs = sorted(np.random.default_rng(8).choice(w.B, 6, replace=False).tolist())
+    ref_o, ref_l = _oracle_absorbed(case, case.q_abs64, seqs=seqs)
+    for b in seqs:
+        _assert_close(o_lat[b].float().cpu().numpy(), ref_o[b], "bf16", f"o_lat seq {b}")
+        _assert_lse(lse[b].cpu().numpy(), ref_l[b], "bf16", f"lse seq {b}")
+
+
+# ------------------------------------------------------------------------------------------------
+# a1, a2, a5 on their own
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name,B", [("dsv3_b64_l4096", 64), ("dsv3_b64_l4096", 5), ("smallem_fp32", 1)])
+def test_append_cache(name, B):
+    w = synth.workload(name, B=B, lengths=("list", tuple([4096 - 3 * i for i in range(B)] if B > 1 else [512])))
+    case = Case(w)
+    dev = case.to_device()
+    cache = _cache(dev, case)
+    before = dev["pool"].clone()
+    ops.mla_append_cache(Dims.of(w), dev["x"], dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache)
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    pool = dev["pool"].cpu()
+    pos = (case.lens - 1).astype(np.int64)
+    c_ref, kr_ref = O.latent_rows(case.x64[:, 0], case.W64["W_DKV"], case.W64["W_KR"], pos, None, w.rms_eps, w.rope_base)
+    rows = case.table[np.arange(B), pos // 64].astype(np.int64) * 64 + pos % 64
+    got = pool[torch.from_numpy(rows)].to(torch.float64).numpy()
+    _assert_close(got[:, :w.d_c], c_ref, w.dtype, "appended latent")
+    _assert_close(got[:, w.d_c:], kr_ref, w.dtype, "appended rope key")
+    if w.dtype == "bf16":   # one rounding of an fp32-accurate value: within one bf16 ulp
+        assert np.all(np.abs(got[:, :w.d_c] - c_ref) <= 2.0 ** -8 * np.abs(c_ref) + 1e-3 * np.abs(c_ref).max())
+    # nothing else in the pool moved
+    mask = torch.ones(pool.shape[0], dtype=torch.bool)
+    mask[torch.from_numpy(rows)] = False
+    assert torch.equal(pool[mask], before.cpu()[mask])
+
+
+@pytest.mark.parametrize("name,s_q", [("dsv3_b64_l4096", 1), ("dsv3_b64_l4096", 3), ("smallem_fp32", 1)])
+def test_absorb_q(name, s_q):
+    w = synth.workload(name, s_q=s_q, B=7, lengths=("list", (7, 100, 4096, 65, 64, 9999, 131072)))
+    case = Case(w)
+    dev = case.to_device()
+    q_abs = ops.mla_absorb_q(Dims.of(w), dev["q_nope"], dev["q_rope_raw"], dev["W_UK"], dev["seqlens"])
+    got = q_abs.to(torch.float64).cpu().numpy()
+    for b in range(w.B):
+        pos = O.token_positions(int(case.lens[b]), s_q)
+        ref = O.absorb_query(case.q_nope64[b], case.q_rope_raw64[b], case.W64["W_UK"], pos, w.rope_base)
+        _assert_close(got[b], ref, w.dtype, f"q_abs seq {b}")
+        _assert_close(got[b][..., w.d_c:], ref[..., w.d_c:], w.dtype, f"rotated query seq {b}")
+
+
+@pytest.mark.parametrize("name", ["dsv3_b64_l4096", "smallem_fp32"])
+def test_out_proj(name):
+    w = synth.workload(name, B=5, s_q=2)
+    case = Case(w)
+    dev = case.to_device()
+    out, out_model = ops.mla_out_proj(Dims.of(w), dev["o_lat"], dev["W_UV"], w_o=dev["W_O"])
+    ref = O.out_projection(case.o_lat64.reshape(-1, w.H, w.d_c), case.W64["W_UV"])
+    _assert_close(out.to(torch.float64).cpu().numpy().reshape(ref.shape), ref, w.dtype, "out heads")
+    ref_m = O.out_projection(case.o_lat64.reshape(-1, w.H, w.d_c), case.W64["W_UV"], case.W64["W_O"])
+    # the model projection consumes the stored (rounded) head outputs on the GPU side
+    _assert_close(out_model.to(torch.float64).cpu().numpy().reshape(ref_m.shape), ref_m, w.dtype, "out model")
+
+
+# ------------------------------------------------------------------------------------------------
+# whole step through the C ABI against the expanded definition
+# ------------------------------------------------------------------------------------------------
+
+def _gpu_step(w, case, dev):
+    dims = Dims.of(w)
+    cache = _cache(dev, case)
+    ops.mla_append_cache(dims, dev["x"], dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache)
+    q_abs = ops.mla_absorb_q(dims, dev["q_nope"], dev["q_rope_raw"], dev["W_UK"], dev["seqlens"])
+    o_lat, lse = ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"])
+    out, out_model = ops.mla_out_proj(dims, o_lat, dev["W_UV"], w_o=dev["W_O"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    return out, out_model, lse
+
+
+def test_smallem_layer_fp32_from_hidden_states():
+    """The Smallem-scale layer in fp32: every position's row appended from x by the GPU (511 as one
+    prefill call, the new token as a decode step), then absorb -> decode -> out_proj, against the
+    expanded definition of the oracle built from the same x."""
+    w = synth.workload("smallem_fp32")
+    L = 512
+    case = Case(w)
+    dev = case.to_device()
+    dims = Dims.of(w)
+    x_all = synth.context_hidden_states(w, L)
+    xt = torch.from_numpy(x_all).float().cuda()
+    cache = _cache(dev, case)
+    prefill_len = torch.tensor([L - 1], dtype=torch.int32, device="cuda")
+    ops.mla_append_cache(dims, xt[None, :L - 1], dev["w_dkv_kr"], None, prefill_len, dev["table"], cache)
+    ops.mla_append_cache(dims, xt[None, L - 1:], dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache)
+    q_abs = ops.mla_absorb_q(dims, dev["q_nope"], dev["q_rope_raw"], dev["W_UK"], dev["seqlens"])
+    o_lat, lse = ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"])
+    out, out_model = ops.mla_out_proj(dims, o_lat, dev["W_UV"], w_o=dev["W_O"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    c, kr = O.latent_rows(x_all.astype(np.float64), case.W64["W_DKV"], case.W64["W_KR"], np.arange(L))
+    got_rows = dev["pool"][:L].double().cpu().numpy()
+    _assert_close(got_rows[:, :w.d_c], c, "f32", "latent rows")
+    _assert_close(got_rows[:, w.d_c:], kr, "f32", "rope rows")
+    pos = np.array([L - 1])
+    q_rot = O.rope(case.q_rope_raw64[0], pos[:, None] * np.ones((1, w.H)))
+    ref, ref_lse = O.expanded_decode(case.q_nope64[0], q_rot, c, kr, case.W64["W_UK"], case.W64["W_UV"], L, w.sm_scale)
+    _assert_close(out[0].double().cpu().numpy(), ref, "f32", "head outputs")
+    _assert_lse(lse[0].cpu().numpy(), ref_lse, "f32", "lse")
+    ref_model = ref.reshape(1, -1) @ case.W64["W_O"]
+    _assert_close(out_model[0].double().cpu().numpy(), ref_model, "f32", "layer output")
+
+
+def test_full_step_dsv3_against_oracle():
+    """configs' DeepSeek shape, full size: append -> absorb -> decode -> out_proj on the GPU; the
+    absorbed fp64 oracle on every sequence, the expanded definition on a sample."""
+    w = synth.workload("dsv3_b64_l4096")
+    case = Case(w)
+    dev = case.to_device()
+    out, out_model, lse = _gpu_step(w, case, dev)
+    # oracle: its own new rows (stored in the cache's type), its own absorption
+    pos = (case.lens - 1).astype(np.int64)
+    c_new, kr_new = O.latent_rows(case.x64[:, 0], case.W64["W_DKV"], case.W64["W_KR"], pos)
+    pool = case.pool.clone()
+    rows = case.table[np.arange(w.B), pos // 64].astype(np.int64) * 64 + pos % 64
+    pool[torch.from_numpy(rows)] = torch.from_numpy(np.concatenate([c_new, kr_new], 1)).to(pool.dtype)
+    got = out.double().cpu().numpy()
+    got_lse = lse.cpu().numpy()
+    sample = [(0, None), (17, None), (63, None)]
+    for b in range(w.B):
+        c, kr = case.seq_rows64(b, pool)
+        L = int(case.lens[b])
+        pb = O.token_positions(L, 1)
+        q_abs = O.absorb_query(case.q_nope64[b], case.q_rope_raw64[b], case.W64["W_UK"], pb)
+        o_lat, l = O.absorbed_decode(q_abs, c, kr, L, w.sm_scale)
+        ref = O.out_projection(o_lat, case.W64["W_UV"])
+        _assert_close(got[b], ref, "bf16", f"out seq {b}")
+        _assert_lse(got_lse[b], l, "bf16", f"lse seq {b}")
+    heads = [0, 5, 77, 127]
+    for b, _ in sample:
+        c, kr = case.seq_rows64(b, pool)
+        L = int(case.lens[b])
+        q_rot = O.rope(case.q_rope_raw64[b][:, heads], np.full((1, len(heads)), L - 1))
+        ref, _ = O.expanded_decode(case.q_nope64[b][:, heads], q_rot, c, kr, case.W64["W_UK"][heads],
+                                   case.W64["W_UV"][heads], L, w.sm_scale)
+        _assert_close(got[b][:, heads], ref, "bf16", f"expanded definition seq {b}")
+
+
+# ------------------------------------------------------------------------------------------------
+# a6: GQLA grouped path
+# ------------------------------------------------------------------------------------------------
+
+def test_gqla_grouped_equals_absorbed_on_same_weights():
+    """Expanded group caches are built by the oracle from the latent rows (stored bf16); the GPU
+    grouped path, the GPU absorbed path on group-shared weights and the oracle must agree."""
+    w = synth.workload("gqla_g8_b32_l8192", B=3, lengths=("list", (100, 1025, 64)), pages="random")
+    case = Case(w)
+    dev = case.to_device()
+    dims = Dims.of(w)
+    W_UK_g, W_UV_g = case.W64["W_UK_g"], case.W64["W_UV_g"]
+    rows = case.pool.to(torch.float64).numpy()
+    K, V = O.gqla_expand(rows[:, :w.d_c], W_UK_g, W_UV_g)
+    Kt = torch.from_numpy(K).to(torch.bfloat16).cuda()
+    Vt = torch.from_numpy(V).to(torch.bfloat16).cuda()
+    gcache = GqaCache(Kt, Vt, dev["pool"][:, w.d_c:], case.num_pages)
+    out, lse = ops.mla_decode_gqla_grouped(dims, dev["q_nope"], dev["q_rope_raw"], gcache, dev["table"], dev["seqlens"])
+    # absorbed path on identical (group-shared) weights
+    W_UK = torch.from_numpy(O.group_weights_per_head(W_UK_g, w.H)).to(torch.bfloat16).cuda()
+    W_UV = torch.from_numpy(O.group_weights_per_head(W_UV_g, w.H)).to(torch.bfloat16).cuda()
+    q_abs = ops.mla_absorb_q(dims, dev["q_nope"], dev["q_rope_raw"], W_UK, dev["seqlens"])
+    o_lat, lse_a = ops.mla_decode_absorbed(dims, q_abs, _cache(dev, case), dev["table"], dev["seqlens"])
+    out_a = ops.mla_out_proj(dims, o_lat, W_UV)
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    Ks = torch.from_numpy(K).to(torch.bfloat16).double().numpy()
+    Vs = torch.from_numpy(V).to(torch.bfloat16).double().numpy()
+    for b in range(w.B):
+        L = int(case.lens[b])
+        p = np.arange(L)
+        idx = case.table[b, p // 64].astype(np.int64) * 64 + p % 64
+        q_rot = O.rope(case.q_rope_raw64[b], np.full((1, w.H), L - 1))
+        ref, ref_l = O.gqla_grouped_decode(case.q_nope64[b], q_rot, Ks[idx], Vs[idx], rows[idx, w.d_c:], L,
+                                           w.sm_scale, w.g)
+        _assert_close(out[b].double().cpu().numpy(), ref, "bf16", f"grouped seq {b}")
+        _assert_lse(lse[b].cpu().numpy(), ref_l, "bf16", f"grouped lse seq {b}")
+        _assert_close(out_a[b].double().cpu().numpy(), ref, "bf16", f"absorbed on group weights seq {b}")
+        _assert_lse(lse_a[b].cpu().numpy(), ref_l, "bf16", f"absorbed lse seq {b}")
+
+
+def test_gqla_full_size_sampled():
+    w = synth.workload("gqla_g8_b32_l8192")
+    lens = synth.seq_lengths(w)
+    table, num_pages = synth.block_table(w, lens)
+    n = num_pages * 64
+    K = torch.empty(n, w.g, w.D, dtype=torch.bfloat16)
+    V = torch.empty(n, w.g, w.d_v, dtype=torch.bfloat16)
+    R = torch.empty(n, w.d_r, dtype=torch.bfloat16)
+    for start, k, v, r in synth.gqla_cache_chunks(w, n):
+        K[start:start + len(k)] = torch.from_numpy(k)
+        V[start:start + len(k)] = torch.from_numpy(v)
+        R[start:start + len(k)] = torch.from_numpy(r)
+    step = synth.decode_step_inputs(w)
+    qn = torch.from_numpy(step["q_nope"]).to(torch.bfloat16)
+    qr = torch.from_numpy(step["q_rope_raw"]).to(torch.bfloat16)
+    gcache = GqaCache(K.cuda(), V.cuda(), R.cuda(), num_pages)
+    out, lse = ops.mla_decode_gqla_grouped(Dims.of(w), qn.cuda(), qr.cuda(), gcache, torch.from_numpy(table).cuda(),
+                                           torch.from_numpy(lens).cuda())
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    Kd, Vd, Rd = K.double().numpy(), V.double().numpy(), R.double().numpy()
+    heads = [0, 15, 16, 64, 127]
+    for b in [0, 13, 31]:
+        L = int(lens[b])
+        p = np.arange(L)
+        idx = table[b, p // 64].astype(np.int64) * 64 + p % 64
+        q_rot = O.rope(qr[b].double().numpy(), np.full((1, w.H), L - 1))
+        ref, ref_l = O.gqla_grouped_decode(qn[b].double().numpy(), q_rot, Kd[idx], Vd[idx], Rd[idx], L, w.sm_scale, w.g)
+        _assert_close(out[b][:, heads].double().cpu().numpy(), ref[:, heads], "bf16", f"grouped seq {b}")
+        _assert_lse(lse[b][:, heads].cpu().numpy(), ref_l[:, heads], "bf16", f"grouped lse seq {b}")
+
+
+# ------------------------------------------------------------------------------------------------
+# errors
+# ------------------------------------------------------------------------------------------------
+
+def test_page_id_outside_pool_is_reported_not_read():
+    w = synth.workload("dsv3_b64_l4096", B=2, lengths=("list", (200, 70)))
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    bad = dev["table"].clone()
+    bad[1, 0] = case.num_pages + 5          # outside the pool: the kernel must skip it and report
+    ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), bad, dev["seqlens"])
+    assert ops.mla_check_status() == L.MLA_ERR_DEVICE_CHECK
+    assert ops.mla_check_status() == 0       # cleared by the previous read
+
+
+def test_invalid_arguments_raise():
+    w = synth.workload("dsv3_b64_l4096", B=1, lengths=("list", (64,)))
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    with pytest.raises(ops.MlaError):
+        ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"],
+                                o_lat=torch.empty(1, 1, 128, 512, dtype=torch.bfloat16, device="cuda")[..., 1:])
