@@ -6,9 +6,23 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+#include <atomic>
+#include <utility>
+
 #include "mla.h"
 
 namespace mla {
+
+// Host-side count of kernel launches made by the library (reported by mla_launch_count).
+inline std::atomic<uint64_t> g_launches{0};
+
+// Every kernel of the library is launched through here, so that the launches can be counted.
+template <typename... KArgs, typename... Args>
+void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  kernel<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
 
 // Per-device status word: the first error a kernel records wins; mla_check_status() clears it.
 __device__ int g_status;

@@ -7,8 +7,6 @@
 #include <stdio.h>
 
 #include <algorithm>
-#include <atomic>
-#include <utility>
 
 #include "mla.h"
 #include "common.cuh"
@@ -21,14 +19,7 @@ using mla::simt::DecodeArgs;
 
 constexpr int kMaxDevices = 64;
 
-std::atomic<uint64_t> g_launches{0};
-
-// Every kernel of the library is launched through here, so that the launches can be counted.
-template <typename... KArgs, typename... Args>
-void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
-  kernel<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-}
+using mla::launch;
 
 int num_sms() {
   static int cached[kMaxDevices] = {0};
@@ -141,7 +132,7 @@ const char* mla_status_string(int s) {
   }
 }
 
-uint64_t mla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+uint64_t mla_launch_count(void) { return mla::g_launches.load(std::memory_order_relaxed); }
 
 const char* mla_build_info(void) {
   return "libmla: sm_100a; kernels: simt (fp32/bf16 all steps), sm100 absorbed decode (tcgen05/TMA)";

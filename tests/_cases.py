@@ -86,6 +86,12 @@ class Case:
         return d
 
 
+def as_stored(a64, dtype: str):
+    """The oracle's own value rounded to the storage type the boundary keeps it in (q_abs and o_lat
+    are bf16 tensors between calls in a bf16 pipeline). Nothing here comes from the GPU."""
+    return torch.from_numpy(np.asarray(a64, np.float64)).to(TORCH_DT[dtype]).to(torch.float64).numpy()
+
+
 def max_rel_err(got, ref):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
