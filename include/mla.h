@@ -99,6 +99,24 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
                      const mla_latent_cache_t* cache, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * a1 without a workspace. The pages have no counterpart to this call: it exists for callers that
+ * cannot allocate device memory — code running inside a framework whose memory pool owns the
+ * device and forbids side allocations, plugins that only receive the tensors of the call, or a
+ * serving process that must not call cudaMalloc once it is running. Same arguments and result as
+ * mla_append_cache, minus the workspace: the split-K partial sums go to a 4 MiB buffer that is
+ * part of the library's device image (every GPU that loads the library holds it until exit).
+ * Nothing is allocated or freed. Limit: B * s_q * (d_c + d_r) <= 1,048,576, else
+ * MLA_ERR_WORKSPACE is returned and nothing is launched. The first call on each device looks up
+ * the buffer's device address (with that device current) and caches it; make that first call
+ * before any stream capture. All calls share the buffer: calls that overlap on the GPU (streams
+ * with no ordering between them) race on it. Nothing in it needs to start at zero.
+ * ------------------------------------------------------------------------------------------- */
+int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                             const void* x, int32_t C, const void* w_dkv_kr, const void* gamma,
+                             const int32_t* seqlens, const int32_t* block_table, int32_t max_pages,
+                             const mla_latent_cache_t* cache, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * a2. Query absorption (« Ce que DeepSeek fait de plus »: q·(W_UK c) = (q·W_UK)·c).
  *   q_abs[b,t,h, 0:d_c]       = q_nope[b,t,h,:] · W_UK[h]            (W_UK[h] is [D, d_c])
  *   q_abs[b,t,h, d_c:d_c+d_r] = RoPE(q_rope_raw[b,t,h,:], seqlens[b] - s_q + t)

@@ -7,6 +7,7 @@
 #include <stdio.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "mla.h"
 #include "common.cuh"
@@ -380,3 +381,91 @@ int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, in
 }
 
 }  // extern "C"
+
+// ================================================================================================
+// Cache append for callers that cannot allocate device memory.
+//
+// Some callers have no way to hand the library a workspace: code that runs inside a framework
+// whose memory pool owns every byte of the device and forbids side allocations, plugins that only
+// receive the tensors of the call, or processes that must not call cudaMalloc once serving has
+// started. mla_append_cache_noalloc serves them: its split-K partial sums live in a fixed buffer
+// that is part of this library's device image (g_append_scratch, 4 MiB). The caller still passes
+// every input and output; nothing is allocated or freed, by this call or by any library it calls.
+//
+// In host code g_append_scratch is only a host-side stand-in for the device array: its device
+// address is looked up once per device with cudaGetSymbolAddress (with that device current) and
+// cached; that set-up happens in the first call made on each device. Every call shares the one
+// buffer, which keeps the previous call's contents; nothing in it needs to start at zero (each
+// call writes every partial sum it later reads). Calls that overlap on the GPU (different streams
+// without ordering between them) race on the buffer.
+// ================================================================================================
+namespace {
+
+constexpr size_t kAppendScratchFloats = size_t(1) << 20;   // 4 MiB of fp32 partial sums
+__device__ __align__(256) float g_append_scratch[kAppendScratchFloats];
+
+std::mutex g_append_scratch_mu;
+float* g_append_scratch_dev[kMaxDevices] = {nullptr};
+
+// Device address of g_append_scratch on the current device (looked up once per device).
+int append_scratch_address(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_append_scratch_mu);
+  if (g_append_scratch_dev[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_append_scratch) != cudaSuccess || ptr == nullptr) return MLA_ERR_CUDA;
+    g_append_scratch_dev[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_append_scratch_dev[dev];
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x,
+                                        int32_t C, const void* w_dkv_kr, const void* gamma, const int32_t* seqlens,
+                                        const int32_t* block_table, int32_t max_pages, const mla_latent_cache_t* cache,
+                                        void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (B <= 0 || s_q <= 0 || C <= 0 || max_pages <= 0 || !x || !w_dkv_kr || !seqlens || !block_table || !cache)
+    return MLA_ERR_INVALID_ARG;
+  if (!cache->latent || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_dkv_kr) || (gamma && !aligned16(gamma)) || !aligned16(cache->latent) ||
+      !aligned16(cache->rope) || !aligned16(seqlens) || !aligned16(block_table))
+    return MLA_ERR_INVALID_ARG;
+  if (!stride_ok(cache->latent_stride, dtype, dims->d_c) || !stride_ok(cache->rope_stride, dtype, dims->d_r))
+    return MLA_ERR_INVALID_ARG;
+  const int n_tok = B * s_q, N = dims->d_c + dims->d_r;
+  // as many K slices as the built-in buffer holds, at most the number the workspace path uses
+  const size_t per_slice = (size_t)n_tok * N;
+  if (per_slice > kAppendScratchFloats) return MLA_ERR_WORKSPACE;   // B*s_q*(d_c+d_r) > 1,048,576
+  const int ks = std::min(append_ksplit(n_tok, C, N), (int)(kAppendScratchFloats / per_slice));
+  float* part = nullptr;
+  if ((rc = append_scratch_address(&part))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
+  dim3 grid((N + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS,
+            (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK, ks);
+  const size_t fin_smem = (size_t)N * sizeof(float);
+  if (dtype == MLA_F32) {
+    using T = float;
+    launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, (const T*)x, n_tok, C,
+           (const T*)w_dkv_kr, N, k_chunk, part, (T*)nullptr);
+    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
+    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)part, ks, n_tok, s_q,
+           dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
+           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);
+  } else {
+    using T = __nv_bfloat16;
+    launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, (const T*)x, n_tok, C,
+           (const T*)w_dkv_kr, N, k_chunk, part, (T*)nullptr);
+    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
+    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)part, ks, n_tok, s_q,
+           dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
+           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);
+  }
+  return launch_status();
+}
