@@ -45,7 +45,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     if not force and up_to_date():
         return LIB
     cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC,
-           "-o", LIB + ".tmp", os.path.join(CSRC, "mla_api.cu"), "-lcuda"]
+           "-o", LIB + ".tmp", os.path.join(CSRC, "mla_api.cu")]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     res = subprocess.run(cmd, capture_output=True, text=True)
