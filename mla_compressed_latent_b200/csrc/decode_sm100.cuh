@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "ptx_sm100.cuh"
+#include "tmap.cuh"
 
 namespace mla {
 namespace sm100 {
@@ -874,34 +875,8 @@ inline size_t decode_workspace_bytes(const mla_dims_t* d, int32_t dtype, int32_t
   return slots * kH * kDC * sizeof(float) + slots * kH * sizeof(float) + 256;
 }
 
-// The tensor-map encoder is a driver entry point; it is resolved at run time through the runtime
-// so that the library does not link against libcuda (and loads on machines without a driver).
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-inline EncodeTiledFn encode_tiled_fn() {
-  static EncodeTiledFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      p = nullptr;
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
 inline bool make_tmap(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t stride_elems) {
-  const EncodeTiledFn encode = encode_tiled_fn();
-  if (!encode) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)stride_elems * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)kTile};
-  const cuuint32_t estr[2] = {1, 1};
-  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return tmap::make_bf16_sw128(m, base, cols, rows, stride_elems, kTile);
 }
 
 inline int active_pairs(int num_sms) {

@@ -1,0 +1,234 @@
+// Per-head "activations times weights" GEMM on the sm_100a tensor cores, for the projections of a
+// decode step: query absorption (q_nope · W_UK[h]), the output projection (o_lat · W_UV[h]) and the
+// cache-append projection (x · [W_DKV | W_KR], split over K). At decode batch sizes all three are
+// bound by reading the weights once, so the kernel streams weight tiles with TMA into a ring of
+// shared-memory stages and keeps one tcgen05 MMA chain fed from it.
+//
+//   Y[tok, h, m] = sum_k X[tok, h, k] · W[h, k, m]
+// is computed transposed, D[m, tok] = A[m, k] · B[tok, k], with A = W[h]ᵀ (the weights' row-major
+// [k, m] layout is MN-major for A, so they are read as stored) and B = X[:, h, :] (K-major). One
+// CTA owns one head, 128 output features (MMA M) and up to 128 tokens (MMA N), and a range of K in
+// chunks of 64. The fp32 accumulator lives in TMEM; four epilogue warps read it back (one TMEM lane
+// = one output feature) and write bf16 rows or fp32 split-K partial sums.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "ptx_sm100.cuh"
+#include "tmap.cuh"
+
+namespace mla {
+namespace gemm {
+
+constexpr int kBM = 128;         // output features per CTA (MMA M)
+constexpr int kBK = 64;          // K per stage: one 128-byte swizzle row of bf16
+constexpr int kMaxStages = 4;
+constexpr int kThreads = 256;    // warp 0 TMA producer, 1 MMA issuer, 2 TMEM owner, 4-7 epilogue
+constexpr int kABytes = kBK * 128 * 2;   // two boxes of 64 k-rows x 64 features
+constexpr int kBarBytes = 1024;          // barriers + TMEM address slot, ahead of the stages
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+struct Params {
+  int M, K;                // output features per head, reduction length per head (K % 64 == 0)
+  int n_tok;               // rows of X
+  int chunks_per_split;    // K chunks (of 64) per blockIdx.z
+  int tn;                  // tokens per CTA = MMA N: 32, 64 or 128
+  int stages;              // ring depth, 1..kMaxStages
+  // mode 0: bf16 Y[tok * y_tok_stride + h * y_head_stride + m]
+  // mode 1: fp32 part[(split * n_tok + tok) * M + m]   (one head)
+  int mode;
+  __nv_bfloat16* y;
+  int64_t y_tok_stride, y_head_stride;
+  float* part;
+  // Optional rotated tail (query absorption): the m-tile-0 CTA of head h also writes
+  // Y[tok, h, M + 2i], Y[tok, h, M + 2i + 1] = RoPE of rope_in[tok, h, 2i .. 2i + 1] at the token's
+  // position seqlens[tok / s_q] - s_q + tok % s_q.
+  const __nv_bfloat16* rope_in;
+  int d_r, H, s_q;
+  const int32_t* seqlens;
+  float rope_base;
+};
+
+__host__ __device__ constexpr int stage_bytes(int tn) { return kABytes + tn * 128; }
+__host__ __device__ constexpr int smem_bytes(int tn, int stages) { return 1024 + kBarBytes + stages * stage_bytes(tn); }
+
+__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = 0;
+  for (uint32_t n = 0;; ++n) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((n & 15u) == 15u) {
+      const uint64_t now = ptx::globaltimer();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kTimeoutNs) { report(MLA_ERR_TIMEOUT); return false; }
+    }
+  }
+}
+
+// grid: x = head * m_tiles + m_tile, y = token block, z = K split
+__global__ void __launch_bounds__(kThreads, 1)
+head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (p.M + kBM - 1) / kBM;
+  const int h = blockIdx.x / m_tiles, mt = blockIdx.x % m_tiles;
+  const int tok0 = blockIdx.y * p.tn;
+  const int split = blockIdx.z;
+  const int kc0 = split * p.chunks_per_split;
+  const int nk = max(0, min(p.K / kBK, kc0 + p.chunks_per_split) - kc0);
+  const int S = p.stages;
+  const uint32_t full0 = base, empty0 = base + 8u * kMaxStages, done = base + 16u * kMaxStages;
+  const uint32_t slot = done + 8u;
+  const uint32_t ring = base + kBarBytes;
+  const uint32_t sbytes = (uint32_t)stage_bytes(p.tn);
+  const uint32_t tmem_cols = p.tn <= 32 ? 32u : (p.tn <= 64 ? 64u : 128u);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { ptx::mbar_init(full0 + 8u * s, 1); ptx::mbar_init(empty0 + 8u * s, 1); }
+    ptx::mbar_init(done, 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tm_w);
+    ptx::prefetch_tmap(&tm_x);
+  }
+  if (warp == 2) { ptx::tmem_alloc(slot, tmem_cols); ptx::tmem_relinquish(); }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + (slot - raw));
+
+  if (warp == 0 && lane == 0) {
+    // ---- TMA producer: per K chunk two weight boxes (64 k x 64 features) and one token box
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % S;
+      if (!wait(empty0 + 8u * s, ((i / S) & 1u) ^ 1u)) break;
+      const uint32_t st = ring + s * sbytes;
+      const int k = h * p.K + (kc0 + i) * kBK;
+      ptx::mbar_arrive_expect_tx(full0 + 8u * s, sbytes);
+      ptx::tma_load_2d(st, &tm_w, mt * kBM, k, full0 + 8u * s);
+      ptx::tma_load_2d(st + kABytes / 2, &tm_w, mt * kBM + 64, k, full0 + 8u * s);
+      ptx::tma_load_2d(st + kABytes, &tm_x, k, tok0, full0 + 8u * s);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer: M = 128, N = tn, four K = 16 steps per chunk
+    const uint32_t idesc = ptx::idesc_bf16_f32_ab(kBM, p.tn, true, false);
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % S;
+      if (!wait(full0 + 8u * s, (i / S) & 1u)) break;
+      ptx::tc_fence_after();
+      const uint32_t st = ring + s * sbytes;
+      // A, MN-major: 8-row K groups 1024 B apart (SBO), the two 64-feature halves one box apart (LBO).
+      // B, K-major: 8-token groups 1024 B apart; a K step of 16 moves 32 B inside the swizzle row.
+      const uint64_t ad = ptx::smem_desc_sw128(st, kABytes / 2, 1024);
+      const uint64_t bd = ptx::smem_desc_sw128(st + kABytes, 16, 1024);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        ptx::mma_ss(tmem, ad + (uint64_t)(k * (2048 >> 4)), bd + (uint64_t)(2 * k), idesc, (i | k) ? 1u : 0u);
+      ptx::mma_commit(empty0 + 8u * s);
+    }
+    ptx::mma_commit(done);
+  } else if (warp >= 4) {
+    // ---- epilogue: thread = output feature (TMEM lane), 32 tokens (TMEM columns) per load
+    const int row = threadIdx.x - 128;
+    const int m = mt * kBM + row;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const bool ok = __all_sync(0xffffffffu, wait(done, 0));
+    ptx::tc_fence_after();
+    if (ok) {
+      for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tmem + lane_off + (uint32_t)c, r);
+        ptx::tmem_wait_ld();
+        if (m >= p.M) continue;
+        const int kn = min(32, p.n_tok - tok0 - c);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          if (k >= kn) break;
+          const int tok = tok0 + c + k;
+          const float v = nk > 0 ? __uint_as_float(r[k]) : 0.f;
+          if (p.mode == 0)
+            p.y[(int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + m] = __float2bfloat16_rn(v);
+          else
+            p.part[((int64_t)split * p.n_tok + tok) * p.M + m] = v;
+        }
+      }
+    }
+    if (p.rope_in != nullptr && mt == 0) {
+      const int half = p.d_r / 2;
+      for (int i = row; i < p.tn * half; i += 128) {
+        const int tok = tok0 + i / half, q = i % half;
+        if (tok >= p.n_tok) continue;
+        const int pos = p.seqlens[tok / p.s_q] - p.s_q + tok % p.s_q;
+        float cs, sn;
+        rope_cos_sin(pos, q, p.d_r, p.rope_base, &cs, &sn);
+        const __nv_bfloat16* r = p.rope_in + ((int64_t)tok * p.H + h) * p.d_r;
+        const float x0 = __bfloat162float(r[2 * q]), x1 = __bfloat162float(r[2 * q + 1]);
+        __nv_bfloat16* o = p.y + (int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + p.M;
+        o[2 * q] = __float2bfloat16_rn(x0 * cs - x1 * sn);
+        o[2 * q + 1] = __float2bfloat16_rn(x0 * sn + x1 * cs);
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+// ---- host ----------------------------------------------------------------------------------------
+// Shapes the kernel takes: K a multiple of 64 (whole chunks), M a multiple of 8 (16-byte weight rows).
+inline bool supported(int K, int M) { return K > 0 && K % kBK == 0 && M > 0 && M % 8 == 0; }
+
+inline int tokens_per_cta(int n_tok) { return n_tok <= 32 ? 32 : (n_tok <= 64 ? 64 : 128); }
+
+// Split of K for mode 1: about one CTA per SM, every split non-empty. Returns the number of splits.
+inline int plan_splits(int M, int K, int n_tok, int num_sms, int max_splits) {
+  const int chunks = K / kBK;
+  const int base = ((M + kBM - 1) / kBM) * ((n_tok + tokens_per_cta(n_tok) - 1) / tokens_per_cta(n_tok));
+  int ks = std::max(1, std::min({(num_sms + base - 1) / base, chunks, max_splits}));
+  const int per = (chunks + ks - 1) / ks;
+  return (chunks + per - 1) / per;
+}
+
+struct Problem {
+  const void* w;             // [H * K, M] row-major bf16 (W[h] = rows h*K .. h*K + K - 1)
+  const void* x;             // [n_tok, H * K] row-major bf16
+  int H, K, M, n_tok;
+  int splits;                // 1 for mode 0
+};
+
+// Launches on `st`; returns MLA_OK, or an error status with nothing launched.
+inline int run(const Problem& pr, Params p, cudaStream_t st) {
+  if (!supported(pr.K, pr.M) || pr.n_tok <= 0 || pr.H <= 0 || pr.splits <= 0) return MLA_ERR_UNSUPPORTED;
+  p.M = pr.M;
+  p.K = pr.K;
+  p.n_tok = pr.n_tok;
+  p.H = pr.H;
+  p.tn = tokens_per_cta(pr.n_tok);
+  const int chunks = pr.K / kBK;
+  p.chunks_per_split = (chunks + pr.splits - 1) / pr.splits;
+  p.stages = std::min(kMaxStages, p.chunks_per_split);
+  CUtensorMap tm_w, tm_x;
+  if (!tmap::make_bf16_sw128(&tm_w, pr.w, pr.M, (int64_t)pr.H * pr.K, pr.M, kBK)) return MLA_ERR_INVALID_ARG;
+  if (!tmap::make_bf16_sw128(&tm_x, pr.x, (int64_t)pr.H * pr.K, pr.n_tok, (int64_t)pr.H * pr.K, p.tn))
+    return MLA_ERR_INVALID_ARG;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+    if (cudaFuncSetAttribute(head_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_bytes(128, kMaxStages)) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    if (dev >= 0 && dev < 64) attr_done[dev] = true;
+  }
+  const dim3 grid(pr.H * ((pr.M + kBM - 1) / kBM), (pr.n_tok + p.tn - 1) / p.tn, pr.splits);
+  mla::launch(head_gemm_kernel, grid, dim3(kThreads), (size_t)smem_bytes(p.tn, p.stages), st, tm_w, tm_x, p);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace gemm
+}  // namespace mla

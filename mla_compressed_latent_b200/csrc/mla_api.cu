@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "decode_sm100.cuh"
+#include "gemm_sm100.cuh"
 
 namespace {
 
@@ -73,6 +74,10 @@ int append_ksplit(int n_tok, int K, int N) {
   ks = std::max(1, std::min(ks, std::min(32, (K + 63) / 64)));
   return ks;
 }
+
+// The tensor-core projection takes bf16 with whole 64-wide K chunks and 16-byte weight rows.
+bool append_on_tc(int32_t dtype, int C, int N) { return dtype == MLA_BF16 && mla::gemm::supported(C, N); }
+int append_tc_splits(int n_tok, int C, int N) { return mla::gemm::plan_splits(N, C, n_tok, num_sms(), 64); }
 
 // ---- a3 split choice for the CUDA-core decode ---------------------------------------------------
 struct SimtSplit { int nsplit, chunk; };
@@ -136,7 +141,7 @@ const char* mla_status_string(int s) {
 uint64_t mla_launch_count(void) { return mla::g_launches.load(std::memory_order_relaxed); }
 
 const char* mla_build_info(void) {
-  return "libmla: sm_100a; kernels: simt (fp32/bf16 all steps), sm100 absorbed decode (tcgen05/TMA)";
+  return "libmla: sm_100a; kernels: simt (fp32/bf16 all steps), sm100 absorbed decode and per-head projections (tcgen05/TMA)";
 }
 
 int mla_check_status(void* stream) {
@@ -157,7 +162,9 @@ int mla_check_status(void* stream) {
 size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C) {
   if (check_dims(dims) || B <= 0 || s_q <= 0 || C <= 0) return 0;
   const int n_tok = B * s_q, N = dims->d_c + dims->d_r;
-  return (size_t)append_ksplit(n_tok, C, N) * n_tok * N * sizeof(float);
+  int ks = append_ksplit(n_tok, C, N);
+  if (mla::gemm::supported(C, N)) ks = std::max(ks, append_tc_splits(n_tok, C, N));
+  return (size_t)ks * n_tok * N * sizeof(float);
 }
 
 int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x,
@@ -176,10 +183,24 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
   if (!stride_ok(cache->latent_stride, dtype, dims->d_c) || !stride_ok(cache->rope_stride, dtype, dims->d_r))
     return MLA_ERR_INVALID_ARG;
   const int n_tok = B * s_q, N = dims->d_c + dims->d_r;
-  const int ks = append_ksplit(n_tok, C, N);
+  const bool tc = append_on_tc(dtype, C, N);
+  const int ks = tc ? append_tc_splits(n_tok, C, N) : append_ksplit(n_tok, C, N);
   const size_t need = (size_t)ks * n_tok * N * sizeof(float);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (tc) {
+    using T = __nv_bfloat16;
+    mla::gemm::Params p{};
+    p.mode = 1;
+    p.part = reinterpret_cast<float*>(workspace);
+    if ((rc = mla::gemm::run({w_dkv_kr, x, 1, C, N, n_tok, ks}, p, st))) return rc;
+    const size_t fin_smem = (size_t)N * sizeof(float);
+    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
+    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)p.part, ks, n_tok, s_q,
+           dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
+           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);
+    return launch_status();
+  }
   const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
   dim3 grid((N + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS,
             (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK, ks);
@@ -221,6 +242,19 @@ int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
   const int n_tok = B * s_q;
   const int D = dims->D, H = dims->H, d_c = dims->d_c, d_r = dims->d_r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == MLA_BF16 && mla::gemm::supported(D, d_c)) {
+    mla::gemm::Params p{};
+    p.mode = 0;
+    p.y = reinterpret_cast<__nv_bfloat16*>(q_abs);
+    p.y_tok_stride = (int64_t)H * (d_c + d_r);
+    p.y_head_stride = d_c + d_r;
+    p.rope_in = reinterpret_cast<const __nv_bfloat16*>(q_rope_raw);
+    p.d_r = d_r;
+    p.s_q = s_q;
+    p.seqlens = seqlens;
+    p.rope_base = dims->rope_base;
+    return mla::gemm::run({w_uk, q_nope, H, D, d_c, n_tok, 1}, p, st);
+  }
   dim3 grid(H, (n_tok + mla::simt::HG_TOK - 1) / mla::simt::HG_TOK);
   const size_t smem = (size_t)mla::simt::HG_TOK * D * sizeof(float);
   if (dtype == MLA_F32) {
@@ -311,6 +345,20 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
   const size_t smem = (size_t)mla::simt::HG_TOK * d_c * sizeof(float);
   dim3 ogrid((C + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS, (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK, 1);
   const int K = H * d_v;
+  if (dtype == MLA_BF16 && mla::gemm::supported(d_c, d_v)) {
+    mla::gemm::Params p{};
+    p.mode = 0;
+    p.y = reinterpret_cast<__nv_bfloat16*>(out);
+    p.y_tok_stride = (int64_t)H * d_v;
+    p.y_head_stride = d_v;
+    if ((rc = mla::gemm::run({w_uv, o_lat, H, d_c, d_v, n_tok, 1}, p, st))) return rc;
+    if (w_o) {
+      using T = __nv_bfloat16;
+      launch(mla::simt::proj_partial_kernel<T>, ogrid, mla::simt::PROJ_COLS, 0, st, (const T*)out, n_tok, K,
+             (const T*)w_o, C, K, nullptr, (T*)out_model);
+    }
+    return launch_status();
+  }
   if (dtype == MLA_F32) {
     using T = float;
     if ((rc = set_smem(mla::simt::head_gemm_kernel<T>, smem))) return rc;

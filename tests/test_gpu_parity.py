@@ -192,6 +192,53 @@ def test_out_proj(name):
     _assert_close(out_model.to(torch.float64).cpu().numpy().reshape(ref_m.shape), ref_m, w.dtype, "out model")
 
 
+def _within_one_rounding(got, ref, what):
+    """bf16 result of an fp32-accumulated sum: one rounding (2^-8 relative) plus a little slack for
+    the accumulation order, relative to the largest reference value."""
+    got = np.asarray(got, np.float64)
+    bad = np.abs(got - ref) > 2.0 ** -8 * np.abs(ref) + 1e-3 * np.abs(ref).max()
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond one bf16 rounding"
+
+
+@pytest.mark.parametrize("B", [33, 100, 300])
+def test_projections_across_token_blocks(B):
+    """a1, a2 and a5 at token counts that take each token width of the tensor-core projection
+    (32, 64, 128 per CTA), several token blocks and a ragged last block."""
+    lens = tuple(65 + (7 * i) % 200 for i in range(B))
+    w = synth.workload("dsv3_b64_l4096", B=B, lengths=("list", lens))
+    case = Case(w)
+    dev = case.to_device()
+    dims = Dims.of(w)
+    q_abs = ops.mla_absorb_q(dims, dev["q_nope"], dev["q_rope_raw"], dev["W_UK"], dev["seqlens"])
+    out = ops.mla_out_proj(dims, dev["o_lat"], dev["W_UV"])
+    cache = _cache(dev, case)
+    before = dev["pool"].clone()
+    ops.mla_append_cache(dims, dev["x"], dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache)
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    got = q_abs.to(torch.float64).cpu().numpy()
+    for b in range(B):
+        ref = O.absorb_query(case.q_nope64[b], case.q_rope_raw64[b], case.W64["W_UK"],
+                             O.token_positions(int(case.lens[b]), 1), w.rope_base)
+        _assert_close(got[b], ref, "bf16", f"q_abs seq {b}")
+        _within_one_rounding(got[b], ref, f"q_abs seq {b}")
+    ref = O.out_projection(case.o_lat64.reshape(-1, w.H, w.d_c), case.W64["W_UV"])
+    got = out.to(torch.float64).cpu().numpy().reshape(ref.shape)
+    _assert_close(got, ref, "bf16", "out heads")
+    _within_one_rounding(got, ref, "out heads")
+    pos = (case.lens - 1).astype(np.int64)
+    c_ref, kr_ref = O.latent_rows(case.x64[:, 0], case.W64["W_DKV"], case.W64["W_KR"], pos, None, w.rms_eps,
+                                  w.rope_base)
+    rows = case.table[np.arange(B), pos // 64].astype(np.int64) * 64 + pos % 64
+    pool = dev["pool"].cpu()
+    got = pool[torch.from_numpy(rows)].to(torch.float64).numpy()
+    _within_one_rounding(got[:, :w.d_c], c_ref, "appended latent")
+    _within_one_rounding(got[:, w.d_c:], kr_ref, "appended rope key")
+    mask = torch.ones(pool.shape[0], dtype=torch.bool)
+    mask[torch.from_numpy(rows)] = False
+    assert torch.equal(pool[mask], before.cpu()[mask])
+
+
 # ------------------------------------------------------------------------------------------------
 # whole step through the C ABI against the expanded definition
 # ------------------------------------------------------------------------------------------------
