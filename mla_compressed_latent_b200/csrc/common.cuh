@@ -43,14 +43,24 @@ template <typename T> __device__ __forceinline__ float ld(const T* p) { return S
 template <typename T> __device__ __forceinline__ void st(T* p, float v) { Store<T>::store(p, v); }
 
 // ---- RoPE ------------------------------------------------------------------------------------
-// Pair (2i, 2i+1) of a d_r vector turns by pos * base^(-2i/d_r). The angle is formed and reduced
-// in double precision: at pos ~ 1e5 an fp32 product would already be off by ~1e-2 rad.
+// Pair (2i, 2i+1) of a d_r vector turns by pos * base^(-2i/d_r). The angle is formed in double
+// precision (at pos ~ 1e5 an fp32 product would already be off by ~1e-2 rad), reduced modulo 2π
+// in double by the Cody-Waite method with 2π split into a double head and tail, and the remainder
+// (|r| <= π) is evaluated with fp32 sincosf.
+__device__ __forceinline__ double rope_inv_freq(int i, int d_r, float base) {
+  return exp2(-(2.0 * (double)i / (double)d_r) * log2((double)base));
+}
+__device__ __forceinline__ void rope_cos_sin_at(int pos, double inv_freq, float* c, float* s) {
+  constexpr double kTwoPiHi = 6.283185307179586;        // 2π rounded to double
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;   // 2π minus kTwoPiHi
+  constexpr double kInvTwoPi = 0.15915494309189535;
+  const double a = (double)pos * inv_freq;
+  const double k = rint(a * kInvTwoPi);
+  const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
+  sincosf((float)r, s, c);
+}
 __device__ __forceinline__ void rope_cos_sin(int pos, int i, int d_r, float base, float* c, float* s) {
-  double theta = pow((double)base, -2.0 * (double)i / (double)d_r);
-  double sn, cs;
-  sincos((double)pos * theta, &sn, &cs);
-  *c = (float)cs;
-  *s = (float)sn;
+  rope_cos_sin_at(pos, rope_inv_freq(i, d_r, base), c, s);
 }
 
 // ---- reductions --------------------------------------------------------------------------------

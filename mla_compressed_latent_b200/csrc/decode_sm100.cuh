@@ -822,44 +822,46 @@ merge_kernel(const int32_t* __restrict__ seqlens, int B, int max_tiles, int npai
   if (tb == 0 || T == 0) return;
   const int p0 = pair_of(off, T, npairs), p1 = pair_of(off + tb - 1, T, npairs);
   if (p0 == p1) return;                       // written whole by one pair
-  // heads of this block: 32 per blockIdx.y, 4 per warp; lanes cover 16 columns each
-  for (int hh = 0; hh < 4; ++hh) {
-    const int h = blockIdx.y * 32 + warp * 4 + hh;
-    float mx = -INFINITY;
-    for (int q = p0; q <= p1; ++q) {
-      const long long start_q = (long long)q * T / npairs;
-      if ((long long)(q + 1) * T / npairs <= start_q) continue;   // a pair with an empty range wrote nothing
-      const int idx = q * 2 + (start_q < off ? 1 : 0);
-      mx = fmaxf(mx, part_lse[(size_t)idx * kH + h]);
-    }
-    float tot = 0.f;
-    float acc[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    for (int q = p0; q <= p1; ++q) {
-      const long long start_q = (long long)q * T / npairs;
-      if ((long long)(q + 1) * T / npairs <= start_q) continue;
-      const int idx = q * 2 + (start_q < off ? 1 : 0);
-      const float wgt = exp2f((part_lse[(size_t)idx * kH + h] - mx) * 1.4426950408889634f);
-      tot += wgt;
-      const float4* src = reinterpret_cast<const float4*>(part_o + ((size_t)idx * kH + h) * kDC + lane * 16);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 v = src[k];
-        acc[4 * k] = fmaf(wgt, v.x, acc[4 * k]);
-        acc[4 * k + 1] = fmaf(wgt, v.y, acc[4 * k + 1]);
-        acc[4 * k + 2] = fmaf(wgt, v.z, acc[4 * k + 2]);
-        acc[4 * k + 3] = fmaf(wgt, v.w, acc[4 * k + 3]);
-      }
-    }
-    const float inv = 1.f / tot;
-    uint4* dst = reinterpret_cast<uint4*>(o_lat + ((size_t)b * kH + h) * kDC + lane * 16);
-    dst[0] = make_uint4(ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv), ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                        ptx::pack_bf16x2(acc[4] * inv, acc[5] * inv), ptx::pack_bf16x2(acc[6] * inv, acc[7] * inv));
-    dst[1] = make_uint4(ptx::pack_bf16x2(acc[8] * inv, acc[9] * inv), ptx::pack_bf16x2(acc[10] * inv, acc[11] * inv),
-                        ptx::pack_bf16x2(acc[12] * inv, acc[13] * inv), ptx::pack_bf16x2(acc[14] * inv, acc[15] * inv));
-    if (lane == 0) lse[(size_t)b * kH + h] = mx + logf(tot);
+  // one head per warp; lanes cover 16 columns each. A pair with an empty range wrote nothing.
+  const int h = blockIdx.y * 8 + warp;
+  auto slot = [&](int q) -> int {
+    const long long start_q = (long long)q * T / npairs;
+    if ((long long)(q + 1) * T / npairs <= start_q) return -1;
+    return q * 2 + (start_q < off ? 1 : 0);
+  };
+  float mx = -INFINITY;
+  for (int q0 = p0; q0 <= p1; q0 += 32) {     // the partials' lse values, one lane each
+    const int q = q0 + lane;
+    const int idx = q <= p1 ? slot(q) : -1;
+    mx = fmaxf(mx, warp_max(idx >= 0 ? part_lse[(size_t)idx * kH + h] : -INFINITY));
   }
+  float tot = 0.f;
+  float acc[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+#pragma unroll 2
+  for (int q = p0; q <= p1; ++q) {
+    const int idx = slot(q);
+    if (idx < 0) continue;
+    const float wgt = exp2f((part_lse[(size_t)idx * kH + h] - mx) * 1.4426950408889634f);
+    tot += wgt;
+    const float4* src = reinterpret_cast<const float4*>(part_o + ((size_t)idx * kH + h) * kDC + lane * 16);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = src[k];
+      acc[4 * k] = fmaf(wgt, v.x, acc[4 * k]);
+      acc[4 * k + 1] = fmaf(wgt, v.y, acc[4 * k + 1]);
+      acc[4 * k + 2] = fmaf(wgt, v.z, acc[4 * k + 2]);
+      acc[4 * k + 3] = fmaf(wgt, v.w, acc[4 * k + 3]);
+    }
+  }
+  const float inv = 1.f / tot;
+  uint4* dst = reinterpret_cast<uint4*>(o_lat + ((size_t)b * kH + h) * kDC + lane * 16);
+  dst[0] = make_uint4(ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv), ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                      ptx::pack_bf16x2(acc[4] * inv, acc[5] * inv), ptx::pack_bf16x2(acc[6] * inv, acc[7] * inv));
+  dst[1] = make_uint4(ptx::pack_bf16x2(acc[8] * inv, acc[9] * inv), ptx::pack_bf16x2(acc[10] * inv, acc[11] * inv),
+                      ptx::pack_bf16x2(acc[12] * inv, acc[13] * inv), ptx::pack_bf16x2(acc[14] * inv, acc[15] * inv));
+  if (lane == 0) lse[(size_t)b * kH + h] = mx + logf(tot);
 }
 
 // ---- host side -----------------------------------------------------------------------------------------
@@ -932,7 +934,7 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   prm.part_lse = prm.part_o + (size_t)2 * max_pairs(num_sms) * kH * kDC;
   prm.sm_scale_log2 = d->sm_scale * 1.4426950408889634f;
   launch(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
-  launch(merge_kernel, dim3(B, kH / 32), dim3(256), 0, st, seqlens, (int)B, (int)max_pages, P, (const float*)prm.part_o,
+  launch(merge_kernel, dim3(B, kH / 8), dim3(256), 0, st, seqlens, (int)B, (int)max_pages, P, (const float*)prm.part_o,
          (const float*)prm.part_lse, prm.o_lat, lse);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

@@ -134,6 +134,23 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     const int row = threadIdx.x - 128;
     const int m = mt * kBM + row;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    if (p.rope_in != nullptr) {
+      // the rotated tail does not depend on the GEMM: done while the main loop runs, the token
+      // block's tokens dealt out over the head's m-tiles (token j of the block goes to m-tile j % m_tiles)
+      const int half = p.d_r / 2;
+      const int my_tok = (p.tn - mt + m_tiles - 1) / m_tiles;
+      for (int i = row; i < my_tok * half; i += 128) {
+        const int tok = tok0 + (i / half) * m_tiles + mt, q = i % half;
+        if (tok >= p.n_tok) continue;
+        const int pos = p.seqlens[tok / p.s_q] - p.s_q + tok % p.s_q;
+        float cs, sn;
+        rope_cos_sin(pos, q, p.d_r, p.rope_base, &cs, &sn);
+        const __nv_bfloat162 r2 = *reinterpret_cast<const __nv_bfloat162*>(p.rope_in + ((int64_t)tok * p.H + h) * p.d_r + 2 * q);
+        const float x0 = __low2float(r2), x1 = __high2float(r2);
+        __nv_bfloat16* o = p.y + (int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + p.M;
+        *reinterpret_cast<__nv_bfloat162*>(o + 2 * q) = __floats2bfloat162_rn(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+      }
+    }
     const bool ok = __all_sync(0xffffffffu, wait(done, 0));
     ptx::tc_fence_after();
     if (ok) {
@@ -153,21 +170,6 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
           else
             p.part[((int64_t)split * p.n_tok + tok) * p.M + m] = v;
         }
-      }
-    }
-    if (p.rope_in != nullptr && mt == 0) {
-      const int half = p.d_r / 2;
-      for (int i = row; i < p.tn * half; i += 128) {
-        const int tok = tok0 + i / half, q = i % half;
-        if (tok >= p.n_tok) continue;
-        const int pos = p.seqlens[tok / p.s_q] - p.s_q + tok % p.s_q;
-        float cs, sn;
-        rope_cos_sin(pos, q, p.d_r, p.rope_base, &cs, &sn);
-        const __nv_bfloat16* r = p.rope_in + ((int64_t)tok * p.H + h) * p.d_r;
-        const float x0 = __bfloat162float(r[2 * q]), x1 = __bfloat162float(r[2 * q + 1]);
-        __nv_bfloat16* o = p.y + (int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + p.M;
-        o[2 * q] = __float2bfloat16_rn(x0 * cs - x1 * sn);
-        o[2 * q + 1] = __float2bfloat16_rn(x0 * sn + x1 * cs);
       }
     }
   }
