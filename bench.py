@@ -294,16 +294,22 @@ def main():
     dec_ev = []
 
     def step(x, q_nope, q_rope, timed_decode=False):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if timed_decode else None
+        if ev:
+            ev[0].record(stream)
         ops.mla_append_cache(dims, x, dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache, workspace=ws_app)
+        if ev:
+            ev[1].record(stream)
         ops.mla_absorb_q(dims, q_nope, q_rope, dev["W_UK"], dev["seqlens"], q_abs=q_abs)
-        if timed_decode:
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
+        if ev:
+            ev[2].record(stream)
         ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"], o_lat=o_lat, lse=lse, workspace=ws_dec)
-        if timed_decode:
-            b.record(stream)
-            dec_ev.append((a, b))
+        if ev:
+            ev[3].record(stream)
         ops.mla_out_proj(dims, o_lat, dev["W_UV"], out=out)
+        if ev:
+            ev[4].record(stream)
+            dec_ev.append(ev)
 
     for _ in range(args.warmup):
         step(dev["x"], dev["q_nope"], dev["q_rope_raw"])
@@ -339,7 +345,9 @@ def main():
     if clk.rejected():
         ms, launches, clk = timed_region()
         remeasured = True
-    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_ev)
+    calls = ("append", "absorb_q", "decode", "out_proj")
+    breakdown = {c: statistics.mean(ev[i].elapsed_time(ev[i + 1]) for ev in dec_ev) * 1e3 for i, c in enumerate(calls)}
+    dec_ms = breakdown["decode"] / 1e3
     assert ops.mla_check_status() == 0
 
     # end to end through the public API: pinned host inputs in, host result out, every step
@@ -382,6 +390,7 @@ def main():
                    "l2": f"inputs larger than L2: {positions * (w.d_c + w.d_r) * (2 if w.dtype == 'bf16' else 4) / 1e6:.0f} MB cache read per step"},
         "tokens_per_s": world * n_tok / step_s,
         "decode_us": dec_ms * 1e3,
+        "step_breakdown_us": breakdown,
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_kind,
                      "kernel": "mla_decode_absorbed (decode + split merge)",

@@ -8,11 +8,13 @@
 // Why a pair: the fp32 accumulator O = 128 heads x 512 latent columns fills all 512 TMEM columns of
 // one SM, leaving no room for the scores. So the two CTAs of a cluster split the work by operand:
 //   CTA 0 ("score CTA") keeps Q̃ [128 x 576] bf16 in TMEM (288 columns) as the A operand and
-//         computes S = Q̃ · [c;k_r]ᵀ for 64-position tiles into three TMEM buffers; its softmax
-//         warps turn S into bf16 P and write P straight into CTA 1's shared memory (DSMEM).
-//   CTA 1 ("output CTA") holds O in TMEM and issues O += P · C for each tile; its warps rescale
-//         O rows when the running maximum moved (lazily: only past 2^8) and run the epilogue.
-// No FLOP is done twice. Each CTA TMA-loads the rows it needs (the second read hits L2).
+//         computes S = Q̃ · [c;k_r]ᵀ for 64-position tiles into three TMEM buffers.
+//   CTA 1 ("output CTA") holds O in TMEM and issues O += P · C for each tile.
+// The score CTA's eight row warps turn S into bf16 P (two softmax warps per SM sub-partition: one
+// alone is bound by its own latency) and each tile's P crosses to the output CTA as one bulk DSMEM
+// copy; the output CTA's row warps rescale their rows of O when a running maximum moved (lazily: only
+// past 2^8) and run the epilogue. No FLOP is done twice; each CTA TMA-loads the rows it needs (the
+// second read hits L2).
 // Work: the tiles of all sequences are laid end to end and cut into one contiguous range per
 // pair; a sequence cut between pairs is written as fp32 partials and merged afterwards.
 // Every wait is bounded in time; on expiry the kernel records MLA_ERR_TIMEOUT and drains.
@@ -35,7 +37,10 @@ __device__ long long g_prof[148][2][12][16];
 #define PROF_ADD(i, from) (prof_[i] += clock64() - (from))
 #define PROF_SAVE(its) do { if (pair < 148) { for (int k_ = 0; k_ < 14; ++k_) g_prof[pair][rank][warp][k_] = prof_[k_]; \
     g_prof[pair][rank][warp][14] = clock64() - prof_t0_; g_prof[pair][rank][warp][15] = (its); } } while (0)
+__device__ unsigned long long g_ptime[148][2][16];
+#define PROF_TIME(k) do { if (pair < 148) g_ptime[pair][rank][k] = ptx::globaltimer(); } while (0)
 #else
+#define PROF_TIME(k) do {} while (0)
 #define PROF_DECL() do {} while (0)
 #define PROF_MARK(v) do {} while (0)
 #define PROF_ADD(i, from) do {} while (0)
@@ -51,59 +56,67 @@ constexpr int kGroupChunks = 3;                       // score CTA: a ring of 3-
 constexpr int kGroupsPerTile = kKChunks / kGroupChunks;// 3 per tile, each released as soon as its
 constexpr int kRing = 7;                               // 12 MMAs are done
 constexpr int kGroupBytes = kGroupChunks * kChunkBytes;// 24576
-constexpr int kPrefetchAhead = 3;                      // tiles fetched into L2 ahead of the ring loads
 constexpr int kQGroups = 6;                            // a sequence's Q̃ travels the ring first: 18 boxes of
                                                        // 64 heads x 64 columns in 6 groups
 constexpr int kVStages = 2;                            // output CTA: whole-tile stages
 constexpr int kVStageBytes = kVChunks * kChunkBytes;   // 65536
-constexpr int kPSlots = 4;                             // P tiles in flight to the output CTA
-constexpr int kStaging = 2;                            // P tiles assembled on the score CTA
-constexpr int kPBytes = kH * kTile * 2;                // 16384: P tile, bf16, 128-byte swizzle
-constexpr int kPSlotStride = 17408;                    // P, then rescale factor per row, then 4 flags
-constexpr int kPCopyBytes = kPBytes + kH * 4 + 16;     // 16912: one bulk copy per tile
 constexpr int kSBufs = 3;
 constexpr int kQCols = kRow / 2;                       // 288 TMEM columns hold Q̃ as bf16 pairs
 constexpr int kSCol0 = kQCols;                         // S buffers at 288, 352, 416
 constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;                   // lazy rescale threshold (log2 units)
-constexpr int kThreads = 384;                          // 4 control warps + 8 softmax / epilogue warps
-constexpr int kGroup = 256;                            // threads of the softmax / epilogue warps
+constexpr int kThreads = 384;                          // 4 control warps + 8 row warps
+constexpr int kGroup = 256;                            // threads of the row warps (4-11)
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
+// Per-tile geometry of the row warps (4..11): warp w owns rows [32 q + 16 u, +16) with q = w % 4 (its
+// TMEM lane quarter, which only sub-partition q can reach) and u = (w - 4) / 4; lane t holds rows
+// +t/4 and +t/4+8, columns 8j + 2 (t % 4) + {0, 1} (the tcgen05 16x256b shape). Two softmax warps per
+// sub-partition: one alone is bound by its own latency, two keep the exponential unit near its rate.
+constexpr int kPBytes = kH * kTile * 2;                // 16384: a P tile, bf16, K-major 128-byte swizzle
+// Rescale factors alpha: per row, 1 unless the row's running maximum moved at this tile.
+// staging buffer (score CTA) and P slot (output CTA) alike: P [128 rows] | alpha [128]
+constexpr int kAlphaOff = kPBytes;
+constexpr int kCopyBytes = kPBytes + kH * 4;           // 16896: one bulk copy per tile
+constexpr int kStgStride = kCopyBytes;
+constexpr int kSlotStride = 17408;                     // a multiple of 1024 (the swizzle repeat)
+constexpr int kPSlots = 4;                             // P tiles in flight on the output CTA
+constexpr int kStaging = 2;                            // P tiles assembled on the score CTA
+static_assert(kCopyBytes <= kSlotStride && kSlotStride % 1024 == 0 && kCopyBytes % 16 == 0, "P slot layout");
+
 // shared memory map (offsets from a 1024-byte aligned base)
-//   score CTA:  K group ring [7] | P staging [2]  | row-maximum and row-sum exchange
-//   output CTA: V stages [2] | P slots [4]        | 1/l per row | mailbox
+//   score CTA:  K group ring [7] | staging [2]
+//   output CTA: V stages [2] | P slots [4] | epilogue transpose buffers [8 x 2 KB]
+//   both:       1/l per row (two segments) | barriers | TMEM address | abort flag | work range
 constexpr int kOffK = 0;
 constexpr int kOffStaging = kRing * kGroupBytes;                       // 172032
+constexpr int kRegion0 = kOffStaging + kStaging * kStgStride;         // 205824
 constexpr int kOffV = 0;
 constexpr int kOffPSlots = kVStages * kVStageBytes;                    // 131072
-constexpr int kRegion0 = kOffStaging + kStaging * kPSlotStride;       // 206848
-constexpr int kRegion1 = kOffPSlots + kPSlots * kPSlotStride;         // 200704
+constexpr int kOffEpi = kOffPSlots + kPSlots * kSlotStride;           // 200704
+constexpr int kEpiWarpBytes = 2048;
+constexpr int kRegion1 = kOffEpi + 8 * kEpiWarpBytes;                 // 217088
 constexpr int kRegion = kRegion0 > kRegion1 ? kRegion0 : kRegion1;
-constexpr int kOffStats = kRegion;                     // float [128] 1/l            (output CTA)
-constexpr int kOffXmax = kOffStats + kH * 4;           // float [2][2][128] partial maxima (score CTA)
-constexpr int kOffXsum = kOffXmax + 2 * 2 * kH * 4;    // float [2][128] partial sums     (score CTA)
-constexpr int kOffMail = kOffXsum + 2 * kH * 4;        // int [4] request to the correction warps
-constexpr int kOffBar = kOffMail + 16;
-// Barriers. Score CTA: K_*, S_*, Q_FULL, P_EMPTY, STATS_EMPTY. Output CTA: V_*, P_FULL, REQ*,
-// RS_READY, SEG_DONE, O_FREE, STATS_FULL. Arrivals from the other CTA reach P_EMPTY, STATS_EMPTY
-// (score CTA) and P_FULL, STATS_FULL (output CTA).
+constexpr int kOffStats = kRegion;                     // float [2][128] 1/l per row   (output CTA)
+constexpr int kOffBar = kOffStats + 2 * kH * 4;
+// Barriers. Score CTA: K_*, S_*, Q_FULL, P_EMPTY, P_WRITTEN, STG_FREE, STATS_EMPTY. Output CTA:
+// V_*, P_FULL, P_LOCAL, P_EMPTY, STATS_FULL. P_EMPTY[slot] completes in both CTAs when the O MMAs
+// of the slot's tile are done (one multicast commit). Arrivals from the other CTA reach P_EMPTY,
+// STG_FREE, STATS_EMPTY (score CTA) and P_FULL, STATS_FULL (output CTA).
 enum Bar : int {
   K_FULL = 0, K_EMPTY = K_FULL + kRing, S_FULL = K_EMPTY + kRing, S_EMPTY = S_FULL + kSBufs,
   Q_FULL = S_EMPTY + kSBufs, P_EMPTY = Q_FULL + 1, P_WRITTEN = P_EMPTY + kPSlots,
   STG_FREE = P_WRITTEN + kStaging, STATS_EMPTY = STG_FREE + kStaging,
   V_FULL = STATS_EMPTY + 1, V_EMPTY = V_FULL + kVStages, P_FULL = V_EMPTY + kVStages,
-  REQ = P_FULL + kPSlots, REQ_DONE = REQ + 1, RS_READY = REQ_DONE + 1, SEG_DONE = RS_READY + 1,
-  O_FREE = SEG_DONE + 1, STATS_FULL = O_FREE + 1, NUM_BARS = STATS_FULL + 1
+  P_LOCAL = P_FULL + kPSlots, STATS_FULL = P_LOCAL + kPSlots, NUM_BARS = STATS_FULL + 1
 };
-enum Mail : int { MAIL_RESCALE = 1, MAIL_EPILOGUE = 2, MAIL_STOP = 3 };
 constexpr int kOffTmemSlot = kOffBar + NUM_BARS * 8;
 constexpr int kOffAbort = kOffTmemSlot + 8;
 constexpr int kOffWork = kOffAbort + 8;                // long long start, end, off_b, b
 constexpr int kSmemUsed = kOffWork + 32;
 constexpr int kSmemBytes = kSmemUsed + 1024;           // + alignment slack of the dynamic base
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert((kOffBar % 8) == 0 && (kOffWork % 8) == 0, "alignment");
+static_assert((kOffBar % 8) == 0 && (kOffWork % 8) == 0 && (kOffEpi % 1024) == 0 && (kOffStaging % 16) == 0, "alignment");
 
 constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 64, false);   // S = Q̃ · Kᵀ   (K-major B)
 constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, 256, true);   // O += P · C   (MN-major B)
@@ -122,6 +135,83 @@ struct Params {
   float* part_lse;             // [2 * pairs, 128]
   float sm_scale_log2;         // sm_scale * log2(e)
 };
+
+// One tile of the online softmax for rows r0 and r0 + 8 of a thread (register layout of the 16x256b
+// shape, see above): the rows' maxima over the tile's valid columns (the 4 threads of a row meet by
+// shuffles), the lazy update of the running maxima m (rescale factors al, 1 when m did not move), and
+// the exponentials packed as bf16 pairs (pk0 row r0, pk1 row r1; column block j) with their sums in l.
+// kMask: the tile has fewer than 64 valid columns (the last page of a sequence).
+template <bool kMask>
+__device__ __forceinline__ void softmax_rows(const uint32_t (&sr)[32], int valid, int t4, float scale2, float& m0,
+                                             float& m1, float& l0, float& l1, float& al0, float& al1,
+                                             uint32_t (&pk0)[8], uint32_t (&pk1)[8]) {
+  float a0 = -INFINITY, a1 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int c = 8 * j + 2 * t4;
+    if (!kMask || c < valid) {
+      a0 = fmaxf(a0, __uint_as_float(sr[4 * j]));
+      a1 = fmaxf(a1, __uint_as_float(sr[4 * j + 2]));
+    }
+    if (!kMask || c + 1 < valid) {
+      a0 = fmaxf(a0, __uint_as_float(sr[4 * j + 1]));
+      a1 = fmaxf(a1, __uint_as_float(sr[4 * j + 3]));
+    }
+  }
+  a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
+  a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+  a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 2));
+  a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
+  // lazy rescale: the running maximum moves only when the tile's exceeds it by 2^kRescaleLog2
+  al0 = 1.f;
+  al1 = 1.f;
+  const float mt0 = a0 * scale2, mt1 = a1 * scale2;
+  if (mt0 > m0 + kRescaleLog2) {
+    al0 = (m0 == -INFINITY) ? 0.f : ptx::ex2_approx(m0 - mt0);
+    l0 *= al0;
+    m0 = mt0;
+  }
+  if (mt1 > m1 + kRescaleLog2) {
+    al1 = (m1 == -INFINITY) ? 0.f : ptx::ex2_approx(m1 - mt1);
+    l1 *= al1;
+    m1 = mt1;
+  }
+  float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int c = 8 * j + 2 * t4;
+    const float e00 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j]), scale2, -m0)) : 0.f;
+    const float e01 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 1]), scale2, -m0)) : 0.f;
+    const float e10 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 2]), scale2, -m1)) : 0.f;
+    const float e11 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 3]), scale2, -m1)) : 0.f;
+    if (j & 1) {
+      ls1 += e00 + e01;
+      ls3 += e10 + e11;
+    } else {
+      ls0 += e00 + e01;
+      ls2 += e10 + e11;
+    }
+    pk0[j] = ptx::pack_bf16x2(e00, e01);
+    pk1[j] = ptx::pack_bf16x2(e10, e11);
+  }
+  l0 += ls0 + ls1;
+  l1 += ls2 + ls3;
+}
+
+// The P words of rows r0, r1 into a P tile at `ptile` (K-major, 128-byte swizzle: row r at
+// (r / 8) * 1024 + (r % 8) * 128, 16-byte chunk j at (j ^ (r % 8)) * 16; word t4 in the chunk).
+__device__ __forceinline__ void store_p_rows(uint32_t ptile, int r0, int t4, const uint32_t (&pk0)[8],
+                                             const uint32_t (&pk1)[8]) {
+  const int r1 = r0 + 8;
+  const uint32_t sw = (uint32_t)(r0 & 7);
+  const uint32_t o0 = ptile + (uint32_t)(r0 >> 3) * 1024u + (uint32_t)(r0 & 7) * 128u + 4u * t4;
+  const uint32_t o1 = ptile + (uint32_t)(r1 >> 3) * 1024u + (uint32_t)(r1 & 7) * 128u + 4u * t4;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    ptx::st_shared_u32(o0 + (((uint32_t)j ^ sw) << 4), pk0[j]);
+    ptx::st_shared_u32(o1 + (((uint32_t)j ^ sw) << 4), pk1[j]);
+  }
+}
 
 // ---- work split -----------------------------------------------------------------------------------
 __device__ __forceinline__ int tiles_of(int L, int max_tiles) { return L > 0 ? min((L + kTile - 1) / kTile, max_tiles) : 0; }
@@ -227,13 +317,13 @@ __device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, uin
 }
 
 // ---- the kernel ------------------------------------------------------------------------------------
-// Warp roles.  Score CTA: 0 TMA producer (+ L2 prefetch ahead) | 1 S-MMA issuer for even tiles, and
-// lane 0 of warp 2 for odd tiles (one issuing thread cannot keep the tensor core busy at N = 64) |
-// 2 TMEM | 3 copier (one bulk copy of each finished P tile into the output CTA) | 4-11 softmax
-// (warps 4-7 columns 0-31 of a tile, warps 8-11 columns 32-63).
+// Warp roles.  Score CTA: 0 TMA producer | 1 S-MMA issuer for even tiles, and lane 0 of warp 2 for odd
+// tiles (one issuing thread cannot keep the tensor core busy at N = 64) | 2 TMEM | 3 copier (one bulk
+// copy per tile into the output CTA) | 4-11 row warps: softmax of their 16 rows each; all of them
+// copy Q̃ into TMEM at a segment start.
 // Output CTA: 0 TMA producer | 1 O-MMA issuer | 2 TMEM, then receiver (returns the score CTA's
-// staging buffers as P tiles land) | 4-11 correction and epilogue (warps 4-7 latent columns 0-255,
-// warps 8-11 columns 256-511).
+// staging buffers as tiles land) | 4-11 row warps: rescale of their own rows of O when a running
+// maximum moved, and the epilogue.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
               const __grid_constant__ CUtensorMap tm_q, const Params p) {
@@ -248,22 +338,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
   auto bar = [&](int i) -> uint32_t { return base + kOffBar + 8u * (uint32_t)i; };
   const uint32_t abort_addr = base + kOffAbort;
   long long* work = reinterpret_cast<long long*>(gbase + kOffWork);
+  if (threadIdx.x == 0) PROF_TIME(0);
 
   if (threadIdx.x == 0) {
     // arrival counts: TMA producers and tcgen05.commit arrive once; thread groups one by one
     for (int i = 0; i < kRing; ++i) { ptx::mbar_init(bar(K_FULL + i), 1); ptx::mbar_init(bar(K_EMPTY + i), 1); }
     for (int i = 0; i < kSBufs; ++i) { ptx::mbar_init(bar(S_FULL + i), 1); ptx::mbar_init(bar(S_EMPTY + i), kGroup); }
     ptx::mbar_init(bar(Q_FULL), kGroup);
-    for (int i = 0; i < kPSlots; ++i) { ptx::mbar_init(bar(P_EMPTY + i), 1); ptx::mbar_init(bar(P_FULL + i), 1); }
+    for (int i = 0; i < kPSlots; ++i) {
+      ptx::mbar_init(bar(P_EMPTY + i), 1);
+      ptx::mbar_init(bar(P_FULL + i), 1);
+      ptx::mbar_init(bar(P_LOCAL + i), kGroup);
+    }
     for (int i = 0; i < kStaging; ++i) { ptx::mbar_init(bar(P_WRITTEN + i), kGroup); ptx::mbar_init(bar(STG_FREE + i), 1); }
     ptx::mbar_init(bar(STATS_EMPTY), kGroup);
     for (int i = 0; i < kVStages; ++i) { ptx::mbar_init(bar(V_FULL + i), 1); ptx::mbar_init(bar(V_EMPTY + i), 1); }
-    ptx::mbar_init(bar(REQ), 1);
-    ptx::mbar_init(bar(REQ_DONE), kGroup);
-    ptx::mbar_init(bar(RS_READY), 1);
-    ptx::mbar_init(bar(SEG_DONE), 1);
-    ptx::mbar_init(bar(O_FREE), kGroup);
-    ptx::mbar_init(bar(STATS_FULL), kH);
+    ptx::mbar_init(bar(STATS_FULL), kH / 2);   // one arrival per score-CTA row thread with t % 4 = 0
     *reinterpret_cast<volatile int*>(gbase + kOffAbort) = 0;
     ptx::fence_mbar_init();
   }
@@ -282,8 +372,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
   ptx::cluster_sync();      // the peer's barriers are initialised before any remote arrive
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffTmemSlot);
+  if (threadIdx.x == 0) PROF_TIME(1);
   SegIter segs{work[0], work[1], work[2], (int)work[3]};
   int b, t_lo, t_hi, tiles_b;
+  // row-warp geometry (warps 4-11)
+  const int qd = warp & 3, sub = (warp - 4) >> 2, t4 = lane & 3;
+  const int r0 = 32 * qd + 16 * sub + (lane >> 2);                       // and r0 + 8
+  const uint32_t s_lane = (uint32_t)(32 * qd + 16 * sub) << 16;          // TMEM lane field of the warp
+  const float scale2 = p.sm_scale_log2;
 
   if (rank == 0) {
     // ============================== score CTA ==============================
@@ -291,22 +387,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
       if (lane == 0) {   // ---- TMA producer: [c (8 chunks) ; k_r (1 chunk)] of each tile
         uint32_t it = 0;
         bool ok = true;
-        // a second walk over the same tiles, kPrefetchAhead ahead, pulls them into L2 (and the
-        // next sequence's query block when it starts)
-        SegIter ahead = segs;
-        int ab = -1, at = 0, a_hi = 0, ax = 0;
-        auto prefetch_next = [&]() {
-          if (at >= a_hi) {
-            if (!ahead.next(p.seqlens, p.B, p.max_tiles, ab, at, a_hi, ax)) { ab = -1; return; }
-          }
-          int pg = p.block_table[(long long)ab * p.max_pages + at];
-          if (pg >= 0 && pg < p.num_pages) {
-            for (int j = 0; j < kVChunks; ++j) ptx::tma_prefetch_2d(&tm_lat, 64 * j, pg * kTile);
-            ptx::tma_prefetch_2d(&tm_rope, 0, pg * kTile);
-          }
-          ++at;
-        };
-        for (int k = 0; k < kPrefetchAhead; ++k) prefetch_next();
         uint32_t gi = 0;
         while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
           // the sequence's absorbed query first: box (column block cb, head half rh)
@@ -320,7 +400,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             }
           }
           for (int t = t_lo; t < t_hi && ok; ++t, ++it) {
-            if (ab >= 0 || at < a_hi) prefetch_next();
             int page = p.block_table[(long long)b * p.max_pages + t];   // issued before the wait
             for (int q = 0; q < kGroupsPerTile && ok; ++q, ++gi) {
               const uint32_t s = gi % kRing;
@@ -336,13 +415,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             }
           }
         }
+        PROF_TIME(2);
         // loads still in flight must land before the CTA may exit
         const uint32_t ng = gi;
         for (uint32_t k = (ng > (uint32_t)kRing ? ng - kRing : 0); k < ng; ++k)
           wait_bar(bar(K_FULL + k % kRing), (k / kRing) & 1u, abort_addr, false, false);
       }
     } else if (warp == 3) {
-      if (lane == 0) {   // ---- copier: each P tile the softmax warps finished goes to the output CTA
+      if (lane == 0) {   // ---- copier: each finished staging buffer goes to the output CTA's slot
         const uint32_t slot_remote0 = ptx::map_to_cta(base + kOffPSlots, 1);
         uint32_t it = 0;
         bool ok = true;
@@ -354,13 +434,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             if (!(ok = wait_bar(bar(P_WRITTEN + stg), (it / kStaging) & 1u, abort_addr, false))) break;
             PROF_ADD(0, c0);
             PROF_MARK(c1);
-            // the slot on the output CTA is free once its MMAs of tile it - kPSlots are done
+            // the slot is free once the output CTA's MMAs of tile it - kPSlots are done
             if (!(ok = wait_bar(bar(P_EMPTY + slot), ((it / kPSlots) & 1u) ^ 1u, abort_addr, true))) break;
             PROF_ADD(1, c1);
             PROF_MARK(c2);
             const uint32_t full = ptx::map_to_cta(bar(P_FULL + slot), 1);
-            ptx::mbar_arrive_expect_tx_remote(bar(P_FULL + slot), 1, kPCopyBytes);
-            ptx::bulk_copy_to_cta(slot_remote0 + slot * kPSlotStride, base + kOffStaging + stg * kPSlotStride, kPCopyBytes, full);
+            const uint32_t src = base + kOffStaging + stg * kStgStride, dst = slot_remote0 + slot * kSlotStride;
+            ptx::mbar_arrive_expect_tx_remote(bar(P_FULL + slot), 1, kCopyBytes);
+            ptx::bulk_copy_to_cta(dst, src, kCopyBytes, full);
             PROF_ADD(2, c2);
           }
         }
@@ -382,6 +463,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           PROF_MARK(q0);
           if (!(ok = wait_bar(bar(Q_FULL), seg & 1u, abort_addr, false))) break;
           PROF_ADD(4, q0);
+          if (parity == 0)   // every row-warp thread has copied its part of the query out of the ring
+            for (int qg = 0; qg < kQGroups; ++qg) ptx::mbar_arrive(bar(K_EMPTY + (gq + qg) % kRing));
           ++seg;
           gq += kQGroups;
           for (int t = t_lo; t < t_hi && ok; ++t, ++it, gq += kGroupsPerTile) {
@@ -389,9 +472,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             PROF_MARK(c0);
             const uint32_t sb = it % kSBufs;
             const uint32_t g0 = gq;
-            // probe, then block on whichever is not there yet
-            const bool se = ptx::mbar_try_wait(bar(S_EMPTY + sb), ((it / kSBufs) & 1u) ^ 1u);
-            if (!se && !(ok = wait_bar(bar(S_EMPTY + sb), ((it / kSBufs) & 1u) ^ 1u, abort_addr, false))) break;
+            if (!(ok = wait_bar(bar(S_EMPTY + sb), ((it / kSBufs) & 1u) ^ 1u, abort_addr, false))) break;
             const uint32_t d = tmem + kSCol0 + 64u * sb;
             PROF_ADD(0, c0);
 #pragma unroll
@@ -421,19 +502,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
         PROF_SAVE(it);
       }
     } else if (warp >= 4) {
-      // ---- softmax: thread = (head h = TMEM lane, column half g of the tile)
-      const int g = (warp - 4) >> 2;
+      // ---- row warps: the softmax of their 16 rows
+      const int g = (warp - 4) >> 2;                      // Q̃ copy: head h, column half g
       const int h = ((warp & 3) << 5) | lane;
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const uint32_t stats_remote = ptx::map_to_cta(base + kOffStats, 1);
-      float* xmax = reinterpret_cast<float*>(gbase + kOffXmax);
-      float* xsum = reinterpret_cast<float*>(gbase + kOffXsum);
-      const float scale2 = p.sm_scale_log2;
       uint32_t it = 0, seg = 0, gq = 0;
       bool ok = true;
       PROF_DECL();
       while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
         const int L = p.seqlens[b];
+        if (threadIdx.x == 128) PROF_TIME(12);
         PROF_MARK(q0);
         // Q̃ of this sequence into TMEM columns [0, 288), from the 6 ring groups that carry it (the
         // previous segment's S MMAs are done: their last result was read below). Half g fills
@@ -442,38 +521,36 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           bool qok = true;
           for (int qg = 0; qg < kQGroups; ++qg)
             qok = qok && wait_bar_warp(bar(K_FULL + (gq + qg) % kRing), ((gq + qg) / kRing) & 1u, abort_addr, false);
-          if (qok) {
-            const int r = h & 63, rh = h >> 6;
+          if (!qok) { ok = false; break; }
+          const int r = h & 63, rh = h >> 6;
 #pragma unroll 1
-            for (int cb = g ? 5 : 0; cb < (g ? 9 : 5); ++cb) {
-              const int qc = 2 * cb + rh, qg = qc / kGroupChunks, j = qc % kGroupChunks;
-              const uint32_t row = base + kOffK + ((gq + qg) % kRing) * kGroupBytes + j * kChunkBytes + r * 128;
-              uint32_t v[32];
+          for (int cb = g ? 5 : 0; cb < (g ? 9 : 5); ++cb) {
+            const int qc = 2 * cb + rh, qg = qc / kGroupChunks, j = qc % kGroupChunks;
+            const uint32_t row = base + kOffK + ((gq + qg) % kRing) * kGroupBytes + j * kChunkBytes + r * 128;
+            uint32_t v[32];
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const uint4 x = ptx::ld_shared_v4(row + ((uint32_t)(k ^ (r & 7)) << 4));
-                v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
-              }
-              ptx::tmem_st32(tmem + lane_off + 32u * cb, v);
+            for (int k = 0; k < 8; ++k) {
+              const uint4 x = ptx::ld_shared_v4(row + ((uint32_t)(k ^ (r & 7)) << 4));
+              v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
             }
-            ptx::tmem_wait_st();
+            ptx::tmem_st32(tmem + lane_off + 32u * cb, v);
           }
-          // the query groups go back to the producer once every thread has read its part
-          if (ptx::named_bar_or(4, kGroup, !qok)) { ok = false; break; }
-          if (threadIdx.x == 128)
-            for (int qg = 0; qg < kQGroups; ++qg) ptx::mbar_arrive(bar(K_EMPTY + (gq + qg) % kRing));
+          ptx::tmem_wait_st();
+          // Q_FULL completes once every thread has stored its part in TMEM; the S-MMA issuer of even
+          // tiles then hands the query groups back to the producer
           gq += kQGroups;
           ptx::tc_fence_before();
           ptx::mbar_arrive(bar(Q_FULL));
         }
         PROF_ADD(7, q0);
+        if (threadIdx.x == 128) PROF_TIME(13);
         int nb = -1;
         {
           SegIter peek = segs;
           int x0, x1, x2;
           if (!peek.next(p.seqlens, p.B, p.max_tiles, nb, x0, x1, x2)) nb = -1;
         }
-        float m = -INFINITY, l = 0.f;
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         gq += kGroupsPerTile * (t_hi - t_lo);
         for (int t = t_lo; t < t_hi; ++t, ++it) {
           const uint32_t s = it % kSBufs, stg = it % kStaging;
@@ -481,71 +558,41 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             const char* nq = reinterpret_cast<const char*>(p.q_abs + ((size_t)nb * kH + h) * kRow);
             for (int k = g ? 5 : 0; k < (g ? 9 : 5); ++k) ptx::prefetch_l2(nq + 128 * k);
           }
-          // probe this tile's staging buffer now; the answer is used after the softmax arithmetic
-          bool stg_free = ptx::mbar_test_wait_cluster(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u);
+          // probe this tile's staging buffer now; the answer is used after the arithmetic
+          const bool stg_free = ptx::mbar_test_wait_cluster(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u);
           PROF_MARK(c0);
-          bool good = wait_bar_warp(bar(S_FULL + s), (it / kSBufs) & 1u, abort_addr, false);
+          if (!wait_bar_warp(bar(S_FULL + s), (it / kSBufs) & 1u, abort_addr, false)) { ok = false; break; }
           PROF_ADD(0, c0);
           PROF_MARK(c1);
           uint32_t sr[32];
-          const int valid = min(kTile, L - t * kTile) - 32 * g;     // valid columns of this half
-          float pm = -INFINITY;
-          if (good) {
-            ptx::tc_fence_after();
-            ptx::tmem_ld32(tmem + lane_off + kSCol0 + 64u * s + 32u * g, sr);
-            ptx::tmem_wait_ld();
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(bar(S_EMPTY + s));
-            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < valid) mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(sr[j]));
-            pm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            xmax[((it & 1) * 2 + g) * kH + h] = pm;
-          }
+          ptx::tc_fence_after();
+          ptx::tmem_ld_16x256b_x8(tmem + s_lane + kSCol0 + 64u * s, sr);
+          ptx::tmem_wait_ld();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar(S_EMPTY + s));
           PROF_ADD(1, c1);
-          PROF_MARK(c2);
-          // all 256 threads meet here every tile and agree whether to stop
-          if (ptx::named_bar_or(1, kGroup, !good)) { ok = false; break; }
-          PROF_ADD(2, c2);
           PROF_MARK(c3);
-          const float m_tile = fmaxf(pm, xmax[((it & 1) * 2 + (g ^ 1)) * kH + h]) * scale2;
-          float alpha = 1.f;
-          if (m_tile > m + kRescaleLog2) {
-            alpha = (m == -INFINITY) ? 0.f : ptx::ex2_approx(m - m_tile);
-            l *= alpha;
-            m = m_tile;
-          }
-          uint32_t pk[16];
-          float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float e0 = (j < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[j]), scale2, -m)) : 0.f;
-            const float e1 = (j + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[j + 1]), scale2, -m)) : 0.f;
-            ls[(j >> 1) & 3] += e0 + e1;
-            pk[j / 2] = ptx::pack_bf16x2(e0, e1);
-          }
-          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          uint32_t pk0[8], pk1[8];
+          float al0 = 1.f, al1 = 1.f;
+          const int valid = L - t * kTile;
+          if (valid >= kTile) softmax_rows<false>(sr, kTile, t4, scale2, m0, m1, l0, l1, al0, al1, pk0, pk1);
+          else softmax_rows<true>(sr, valid, t4, scale2, m0, m1, l0, l1, al0, al1, pk0, pk1);
           PROF_ADD(3, c3);
           PROF_MARK(c4);
           // this tile's staging buffer must have been copied out (tile it - kStaging)
           if (!__all_sync(0xffffffffu, stg_free) &&
-              !wait_bar_warp(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u, abort_addr, true))
-            continue;
+              !wait_bar_warp(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u, abort_addr, true)) {
+            ok = false;
+            break;
+          }
           PROF_ADD(4, c4);
           PROF_MARK(c5);
-          const uint32_t st0 = base + kOffStaging + stg * kPSlotStride;
-          const uint32_t row = st0 + (uint32_t)(h >> 3) * 1024u + (uint32_t)(h & 7) * 128u;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int c = 4 * g + k;
-            ptx::st_shared_v4(row + ((uint32_t)(c ^ (h & 7)) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-          }
-          if (g == 0) {
-            reinterpret_cast<float*>(gbase + kOffStaging + stg * kPSlotStride + kPBytes)[h] = alpha;
-            const bool rescaled = __any_sync(0xffffffffu, alpha != 1.f);
-            if (lane == 0)
-              reinterpret_cast<int*>(gbase + kOffStaging + stg * kPSlotStride + kPBytes + kH * 4)[warp & 3] = rescaled ? 1 : 0;
+          const uint32_t st0 = base + kOffStaging + stg * kStgStride;
+          store_p_rows(st0, r0, t4, pk0, pk1);
+          if (t4 == 0) {
+            float* alpha_s = reinterpret_cast<float*>(gbase + kOffStaging + stg * kStgStride + kAlphaOff);
+            alpha_s[r0] = al0;
+            alpha_s[r0 + 8] = al1;
           }
           // visible to the bulk copy (async proxy), then handed to the copier
           ptx::fence_proxy_async_smem();
@@ -553,35 +600,35 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           PROF_ADD(5, c5);
         }
         if (!ok) break;
-        // segment end: combine the two halves' row sums; 1/l to the output CTA, lse to memory
-        xsum[g * kH + h] = l;
-        if (ptx::named_bar_or(2, kGroup, false)) { ok = false; break; }
-        l = xsum[h] + xsum[kH + h];
-        bool fail = false;
-        if (g == 0) {
-          if (!wait_bar_warp(bar(STATS_EMPTY), (seg & 1u) ^ 1u, abort_addr, true)) {
-            fail = true;
-          } else {
+        {
+          // segment end: each row's sum over its four threads; 1/l to the output CTA, lse to memory
+          l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+          l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+          l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+          l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+          if (!wait_bar_warp(bar(STATS_EMPTY), (seg & 1u) ^ 1u, abort_addr, true)) { ok = false; break; }
+          if (t4 == 0) {
             const bool partial = !(t_lo == 0 && t_hi == tiles_b);
-            const float lse = (m + log2f(l)) * 0.69314718055994531f;
-            if (partial) p.part_lse[((size_t)pair * 2 + (seg > 0)) * kH + h] = lse;
-            else p.lse[(size_t)b * kH + h] = lse;
-            ptx::st_cluster_f32(stats_remote + h * 4u, 1.f / l);
+            float* lse_dst = partial ? p.part_lse + ((size_t)pair * 2 + (seg > 0)) * kH : p.lse + (size_t)b * kH;
+            lse_dst[r0] = (m0 + log2f(l0)) * 0.69314718055994531f;
+            lse_dst[r0 + 8] = (m1 + log2f(l1)) * 0.69314718055994531f;
+            const uint32_t st = stats_remote + ((seg & 1u) * kH) * 4u;
+            ptx::st_cluster_f32(st + r0 * 4u, 1.f / l0);
+            ptx::st_cluster_f32(st + (r0 + 8) * 4u, 1.f / l1);
             ptx::mbar_arrive_remote(bar(STATS_FULL), 1);
           }
         }
-        // both halves leave together if either failed (the next segment meets at named barriers)
-        if (ptx::named_bar_or(3, kGroup, fail)) { ok = false; break; }
         ++seg;
       }
       PROF_SAVE(it);
+      if (threadIdx.x == 128) PROF_TIME(3);
       // before leaving: the output CTA's last release of the stats must have landed here
-      if (g == 0 && seg > 0) wait_bar(bar(STATS_EMPTY), (seg - 1) & 1u, abort_addr, true, false);
+      if (t4 == 0 && seg > 0) wait_bar(bar(STATS_EMPTY), (seg - 1) & 1u, abort_addr, true, false);
     }
   } else {
     // ============================== output CTA ==============================
     if (warp == 2) {
-      if (lane == 0) {   // ---- receiver: as each P tile lands, the score CTA may reuse that staging buffer
+      if (lane == 0) {   // ---- receiver: as each tile lands, the score CTA may reuse that staging buffer
         uint32_t it = 0;
         bool ok = true;
         while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
@@ -611,37 +658,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
       }
     } else if (warp == 1) {
       // ---- MMA issuer (lane 0) with the warp's help for masking: O += P · C, K = 64 positions in
-      // 4 steps of 16, N = 512 in 2 halves
+      // 4 steps of 16, N = 512 in 2 halves. A tile's P is complete (and O rescaled for it) once the
+      // row warps arrived on P_LOCAL.
       const uint64_t v_desc0 = ptx::smem_desc_sw128(base + kOffV, kChunkBytes, 1024);
       const uint64_t p_desc0 = ptx::smem_desc_sw128(base + kOffPSlots, 16, 1024);
-      volatile int* mail = reinterpret_cast<volatile int*>(gbase + kOffMail);
-      uint32_t it = 0, seg = 0, nresc = 0;
+      uint32_t it = 0;
       bool ok = true;
       PROF_DECL();
       while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
         const int L = p.seqlens[b];
-        // the previous segment's epilogue has read O out of TMEM
-        PROF_MARK(f0);
-        if (!(ok = wait_bar_warp(bar(O_FREE), (seg & 1u) ^ 1u, abort_addr, false))) break;
-        PROF_ADD(4, f0);
         for (int t = t_lo; t < t_hi; ++t, ++it) {
           const uint32_t slot = it % kPSlots, s = it % kVStages;
           PROF_MARK(c0);
-          if (!(ok = wait_bar_warp(bar(P_FULL + slot), (it / kPSlots) & 1u, abort_addr, true))) break;
+          if (!(ok = wait_bar_warp(bar(P_LOCAL + slot), (it / kPSlots) & 1u, abort_addr, false))) break;
           PROF_ADD(0, c0);
-          const volatile int* flags = reinterpret_cast<const volatile int*>(gbase + kOffPSlots + slot * kPSlotStride + kPBytes + kH * 4);
-          const bool resc = (t > t_lo) && (flags[0] | flags[1] | flags[2] | flags[3]);
-          if (resc) {
-            // some rows' maximum moved: the correction warps rescale O once the MMAs so far are done
-            if (lane == 0) {
-              ptx::mma_commit(bar(RS_READY));
-              mail[0] = MAIL_RESCALE;
-              mail[1] = (int)slot;
-              ptx::mbar_arrive(bar(REQ));
-            }
-            if (!(ok = wait_bar_warp(bar(REQ_DONE), nresc & 1u, abort_addr, false))) break;
-            ++nresc;
-          }
           PROF_MARK(c2);
           if (!(ok = wait_bar_warp(bar(V_FULL + s), (it / kVStages) & 1u, abort_addr, false))) break;
           PROF_ADD(1, c2);
@@ -666,7 +696,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           if (lane == 0) {
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_after();
-            const uint64_t pd = p_desc0 + (uint64_t)(slot * (kPSlotStride >> 4));
+            const uint64_t pd = p_desc0 + (uint64_t)(slot * (kSlotStride >> 4));
             const uint64_t vd = v_desc0 + (uint64_t)(s * (kVStageBytes >> 4));
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk) {
@@ -677,116 +707,150 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
               }
             }
             ptx::mma_commit(bar(V_EMPTY + s));
-            ptx::mma_commit_mc(bar(P_EMPTY + slot), (uint16_t)0x1);
+            ptx::mma_commit_mc(bar(P_EMPTY + slot), (uint16_t)0x3);
           }
           __syncwarp();
           PROF_ADD(2, c3);
         }
-        if (!ok) break;
-        // segment complete once its MMAs are: hand O to the epilogue
-        if (lane == 0) {
-          ptx::mma_commit(bar(SEG_DONE));
-          mail[0] = MAIL_EPILOGUE;
-          mail[1] = (int)seg;
-          ptx::mbar_arrive(bar(REQ));
-        }
-        ++seg;
       }
       if (lane == 0) PROF_SAVE(it);
-      if (lane == 0) {
-        // let the correction warps leave (after the last epilogue has freed O)
-        if (seg > 0) wait_bar(bar(O_FREE), (seg - 1) & 1u, abort_addr, false, false);
-        mail[0] = MAIL_STOP;
-        ptx::mbar_arrive(bar(REQ));
-      }
+      if (lane == 0) PROF_TIME(4);
     } else if (warp >= 4) {
-      // ---- correction + epilogue: thread = (head h = TMEM lane, latent half g). Serves the
-      // requests of the MMA warp in order: rescale O rows, or write out a finished segment.
-      const int g = (warp - 4) >> 2;
+      // ---- row warps: rescale of the warp's own 16 rows of O before a tile whose P was computed
+      // against a larger maximum, and the segment epilogue
+      const int g = (warp - 4) >> 2;                      // epilogue: head h, latent half g
       const int h = ((warp & 3) << 5) | lane;
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const uint32_t col0 = 256u * g;
-      const volatile float* stats_s = reinterpret_cast<const volatile float*>(gbase + kOffStats);
-      const volatile int* mail = reinterpret_cast<const volatile int*>(gbase + kOffMail);
-      uint32_t nreq = 0, nresc = 0, seg = 0;
-      while (true) {
-        if (!wait_bar_warp(bar(REQ), nreq & 1u, abort_addr, false)) break;
-        ++nreq;
-        const int kind = mail[0], arg = mail[1];
-        if (kind == MAIL_STOP) break;
-        if (kind == MAIL_RESCALE) {
-          if (!wait_bar_warp(bar(RS_READY), nresc & 1u, abort_addr, false)) break;
-          ++nresc;
-          ptx::tc_fence_after();
-          const float alpha = reinterpret_cast<const volatile float*>(gbase + kOffPSlots + arg * kPSlotStride + kPBytes)[h];
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      float* stats = reinterpret_cast<float*>(gbase + kOffStats);
+      uint32_t it = 0, seg = 0;
+      bool ok = true;
+      PROF_DECL();
+      while (segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
+        for (int t = t_lo; t < t_hi; ++t, ++it) {
+          if (!ok) continue;   // after a failure: skip to the segment end, where all row warps meet
+          const uint32_t slot = it % kPSlots;
+          PROF_MARK(c0);
+          if (!wait_bar_warp(bar(P_FULL + slot), (it / kPSlots) & 1u, abort_addr, true)) { ok = false; continue; }
+          PROF_ADD(0, c0);
+          PROF_MARK(c1);
+          const float* alpha_s = reinterpret_cast<const float*>(gbase + kOffPSlots + slot * kSlotStride + kAlphaOff);
+          const float al0 = alpha_s[r0], al1 = alpha_s[r0 + 8];
+          PROF_ADD(1, c1);
+          PROF_MARK(c2);
+          // O rows of this warp computed against an older maximum: scale them once the MMAs of the
+          // previous tile are done (16x256b: rows r0, r0 + 8, 8 columns per 256-bit chunk). The slot's
+          // phase before that one (tile it - 1 - kPSlots) completed before tile it - 1's P_FULL, so the
+          // parity test cannot mistake it.
+          if (t > t_lo && __any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+            const uint32_t pt = it - 1;
+            if (!wait_bar_warp(bar(P_EMPTY + pt % kPSlots), (pt / kPSlots) & 1u, abort_addr, false)) { ok = false; continue; }
+            ptx::tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < kDC / 2; c += 32) {
+            for (int c = 0; c < kDC; c += 64) {
               uint32_t r[32];
-              ptx::tmem_ld32(tmem + lane_off + col0 + c, r);
+              ptx::tmem_ld_16x256b_x8(tmem + s_lane + c, r);
               ptx::tmem_wait_ld();
 #pragma unroll
-              for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-              ptx::tmem_st32(tmem + lane_off + col0 + c, r);
+              for (int j = 0; j < 8; ++j) {
+                r[4 * j] = __float_as_uint(__uint_as_float(r[4 * j]) * al0);
+                r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) * al0);
+                r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) * al1);
+                r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) * al1);
+              }
+              ptx::tmem_st_16x256b_x8(tmem + s_lane + c, r);
             }
             ptx::tmem_wait_st();
           }
+          PROF_ADD(2, c2);
           ptx::tc_fence_before();
-          ptx::mbar_arrive(bar(REQ_DONE));
-          continue;
+          ptx::mbar_arrive(bar(P_LOCAL + slot));
         }
-        // MAIL_EPILOGUE: O / l  ->  o_lat (bf16) or an fp32 partial
-        if (!segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) break;
-        if (!wait_bar_warp(bar(SEG_DONE), seg & 1u, abort_addr, false)) break;
-        if (!wait_bar_warp(bar(STATS_FULL), seg & 1u, abort_addr, true)) break;
+        // segment end: O / l out, 1/l from the score CTA
+        if (threadIdx.x == 128) PROF_TIME(8);
+        if (ok && !wait_bar_warp(bar(P_EMPTY + (it - 1) % kPSlots), ((it - 1) / kPSlots) & 1u, abort_addr, false)) ok = false;
+        if (threadIdx.x == 128) PROF_TIME(9);
+        if (ok && !wait_bar_warp(bar(STATS_FULL), seg & 1u, abort_addr, true)) ok = false;
+        if (threadIdx.x == 128) PROF_TIME(10);
+        // every row warp meets here once per segment and agrees whether to go on
+        if (ptx::named_bar_or(1, kGroup, !ok)) break;
         ptx::tc_fence_after();
-        const float inv_l = stats_s[h];
+        const float inv_l = stats[(seg & 1u) * kH + h];
         const bool partial = !(t_lo == 0 && t_hi == tiles_b);
-        if (partial) {
-          float* dst = p.part_o + (((size_t)pair * 2 + (seg > 0)) * kH + h) * kDC + col0;
-#pragma unroll 1
-          for (int c = 0; c < kDC / 2; c += 32) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tmem + lane_off + col0 + c, r);
-            ptx::tmem_wait_ld();
-            float4* d4 = reinterpret_cast<float4*>(dst + c);
+        // 32 columns of the warp's 32 rows at a time: each thread (row) scales its values and puts
+        // them in the warp's buffer as one 64-byte row (16-byte chunks XOR-swizzled by row / 2, so
+        // both phases are free of bank conflicts); read back as (row 8i + lane / 4, chunk lane % 4),
+        // every 16-byte store instruction writes eight 64-byte row pieces.
+        const uint32_t ebuf = base + kOffEpi + (uint32_t)(warp - 4) * kEpiWarpBytes;
+        const uint32_t wrow = ebuf + (uint32_t)lane * 64u;
+        const uint32_t sw = (uint32_t)(lane >> 1) & 3u;
+        const int c4 = lane & 3, rsub = lane >> 2;
+        const int row0 = (warp & 3) * 32;
+        auto flush = [&](char* dst0, size_t row_bytes) {   // the buffer's 32 rows to dst0 + row * row_bytes
+          __syncwarp();
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              d4[k] = make_float4(__uint_as_float(r[4 * k]) * inv_l, __uint_as_float(r[4 * k + 1]) * inv_l,
-                                  __uint_as_float(r[4 * k + 2]) * inv_l, __uint_as_float(r[4 * k + 3]) * inv_l);
+          for (int i = 0; i < 4; ++i) {
+            const int rr = 8 * i + rsub;
+            const uint4 v = ptx::ld_shared_v4(ebuf + rr * 64u + (((uint32_t)c4 ^ (((uint32_t)rr >> 1) & 3u)) << 4));
+            *reinterpret_cast<uint4*>(dst0 + (size_t)(row0 + rr) * row_bytes + c4 * 16) = v;
           }
-        } else {
-          __nv_bfloat16* dst = p.o_lat + ((size_t)b * kH + h) * kDC + col0;
+          __syncwarp();
+        };
 #pragma unroll 1
-          for (int c = 0; c < kDC / 2; c += 32) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tmem + lane_off + col0 + c, r);
-            ptx::tmem_wait_ld();
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+        for (int c = 0; c < kDC / 2; c += 32) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tmem + lane_off + col0 + c, r);
+          ptx::tmem_wait_ld();
+          if (partial) {
+            float* dst = p.part_o + ((size_t)pair * 2 + (seg > 0)) * kH * kDC + col0 + c;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              d4[k] = make_uint4(ptx::pack_bf16x2(__uint_as_float(r[8 * k]) * inv_l, __uint_as_float(r[8 * k + 1]) * inv_l),
-                                 ptx::pack_bf16x2(__uint_as_float(r[8 * k + 2]) * inv_l, __uint_as_float(r[8 * k + 3]) * inv_l),
-                                 ptx::pack_bf16x2(__uint_as_float(r[8 * k + 4]) * inv_l, __uint_as_float(r[8 * k + 5]) * inv_l),
-                                 ptx::pack_bf16x2(__uint_as_float(r[8 * k + 6]) * inv_l, __uint_as_float(r[8 * k + 7]) * inv_l));
+            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int j = 16 * half + 4 * k;
+                ptx::st_shared_v4(wrow + ((k ^ sw) << 4), __float_as_uint(__uint_as_float(r[j]) * inv_l),
+                                  __float_as_uint(__uint_as_float(r[j + 1]) * inv_l),
+                                  __float_as_uint(__uint_as_float(r[j + 2]) * inv_l),
+                                  __float_as_uint(__uint_as_float(r[j + 3]) * inv_l));
+              }
+              flush(reinterpret_cast<char*>(dst + 16 * half), kDC * sizeof(float));
+            }
+          } else {
+            __nv_bfloat16* dst = p.o_lat + (size_t)b * kH * kDC + col0 + c;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int j = 8 * k;
+              ptx::st_shared_v4(wrow + ((k ^ sw) << 4),
+                                ptx::pack_bf16x2(__uint_as_float(r[j]) * inv_l, __uint_as_float(r[j + 1]) * inv_l),
+                                ptx::pack_bf16x2(__uint_as_float(r[j + 2]) * inv_l, __uint_as_float(r[j + 3]) * inv_l),
+                                ptx::pack_bf16x2(__uint_as_float(r[j + 4]) * inv_l, __uint_as_float(r[j + 5]) * inv_l),
+                                ptx::pack_bf16x2(__uint_as_float(r[j + 6]) * inv_l, __uint_as_float(r[j + 7]) * inv_l));
+            }
+            flush(reinterpret_cast<char*>(dst), kDC * sizeof(__nv_bfloat16));
           }
         }
+        if (threadIdx.x == 128) PROF_TIME(11);
+        // O may be overwritten by the next segment's first MMA once every row warp arrived on its
+        // P_LOCAL (after this point, in program order); the score CTA may write the next 1/l values
         ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(O_FREE));
         ptx::mbar_arrive_remote(bar(STATS_EMPTY), 0);
         ++seg;
       }
+      PROF_SAVE(it);
+      if (threadIdx.x == 128) PROF_TIME(5);
     }
   }
 
   // teardown: TMEM back, then leave together so no remote access can target an exited CTA
   ptx::tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) PROF_TIME(6);
   if (warp == 2) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
   ptx::cluster_sync();
+  if (threadIdx.x == 0) PROF_TIME(7);
 }
 
 // ---- merge of split sequences ------------------------------------------------------------------------
