@@ -24,6 +24,31 @@ void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaSt
   g_launches.fetch_add(1, std::memory_order_relaxed);
 }
 
+// Same, with programmatic dependent launch allowed: the kernel may be scheduled while the previous
+// kernel of the stream is still running, and runs its prologue (barrier setup, TMEM allocation) in
+// its shadow. Such a kernel calls grid_dependency_wait() before it touches global memory and
+// allow_dependents() once its own successor may be scheduled.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+// Waits until the kernels this one depends on have completed and their writes are visible.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel of the stream be scheduled (it still waits for this one in its own
+// grid_dependency_wait before reading anything).
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Per-device status word: the first error a kernel records wins; mla_check_status() clears it.
 __device__ int g_status;
 

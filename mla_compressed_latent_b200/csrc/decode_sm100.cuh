@@ -198,18 +198,19 @@ __device__ __forceinline__ void softmax_rows(const uint32_t (&sr)[32], int valid
   l1 += ls2 + ls3;
 }
 
-// The P words of rows r0, r1 into a P tile at `ptile` (K-major, 128-byte swizzle: row r at
-// (r / 8) * 1024 + (r % 8) * 128, 16-byte chunk j at (j ^ (r % 8)) * 16; word t4 in the chunk).
-__device__ __forceinline__ void store_p_rows(uint32_t ptile, int r0, int t4, const uint32_t (&pk0)[8],
+// A warp's P rows into a P tile at `ptile` (K-major, 128-byte swizzle: row r at (r / 8) * 1024 +
+// (r % 8) * 128, 16-byte chunk j at (j ^ (r % 8)) * 16). The warp's rows are [rw, rw + 16); pk0[j] /
+// pk1[j] are the thread's element pairs of the 8x8 blocks (rows rw + [0, 8) / rw + [8, 16), chunk j),
+// which is exactly the stmatrix fragment layout: four stmatrix.x4 store all sixteen blocks.
+__device__ __forceinline__ void store_p_rows(uint32_t ptile, int rw, int lane, const uint32_t (&pk0)[8],
                                              const uint32_t (&pk1)[8]) {
-  const int r1 = r0 + 8;
-  const uint32_t sw = (uint32_t)(r0 & 7);
-  const uint32_t o0 = ptile + (uint32_t)(r0 >> 3) * 1024u + (uint32_t)(r0 & 7) * 128u + 4u * t4;
-  const uint32_t o1 = ptile + (uint32_t)(r1 >> 3) * 1024u + (uint32_t)(r1 & 7) * 128u + 4u * t4;
+  const int m = lane >> 3, row = rw + (lane & 7) + 8 * (m & 1);
+  const uint32_t row_addr = ptile + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
+  const uint32_t sw = (uint32_t)(row & 7);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    ptx::st_shared_u32(o0 + (((uint32_t)j ^ sw) << 4), pk0[j]);
-    ptx::st_shared_u32(o1 + (((uint32_t)j ^ sw) << 4), pk1[j]);
+  for (int j = 0; j < 8; j += 2) {
+    const uint32_t chunk = (uint32_t)(j + (m >> 1));
+    ptx::stmatrix_x4(row_addr + ((chunk ^ sw) << 4), pk0[j], pk1[j], pk0[j + 1], pk1[j + 1]);
   }
 }
 
@@ -366,9 +367,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
     ptx::tmem_alloc(base + kOffTmemSlot, kTmemCols);
     ptx::tmem_relinquish();
   }
+  // nothing above touched global memory; from here on the previous kernel's results are needed
+  grid_dependency_wait();
   if (warp == 3) plan_range(p.seqlens, p.B, p.max_tiles, pair, npairs, work);
   ptx::tc_fence_before();
   __syncthreads();
+  // (no early allow_dependents(): the merge that follows would park its blocks on these SMs)
   ptx::cluster_sync();      // the peer's barriers are initialised before any remote arrive
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffTmemSlot);
@@ -588,7 +592,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           PROF_ADD(4, c4);
           PROF_MARK(c5);
           const uint32_t st0 = base + kOffStaging + stg * kStgStride;
-          store_p_rows(st0, r0, t4, pk0, pk1);
+          store_p_rows(st0, 32 * qd + 16 * sub, lane, pk0, pk1);
           if (t4 == 0) {
             float* alpha_s = reinterpret_cast<float*>(gbase + kOffStaging + stg * kStgStride + kAlphaOff);
             alpha_s[r0] = al0;
@@ -863,6 +867,8 @@ merge_kernel(const int32_t* __restrict__ seqlens, int B, int max_tiles, int npai
   __shared__ long long sh[3];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  grid_dependency_wait();
+  allow_dependents();
   if (warp == 0) {
     const int per = (B + 31) / 32;
     const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
@@ -997,8 +1003,8 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   prm.part_o = reinterpret_cast<float*>(workspace);
   prm.part_lse = prm.part_o + (size_t)2 * max_pairs(num_sms) * kH * kDC;
   prm.sm_scale_log2 = d->sm_scale * 1.4426950408889634f;
-  launch(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
-  launch(merge_kernel, dim3(B, kH / 8), dim3(256), 0, st, seqlens, (int)B, (int)max_pages, P, (const float*)prm.part_o,
+  launch_pdl(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
+  launch_pdl(merge_kernel, dim3(B, kH / 8), dim3(256), 0, st, seqlens, (int)B, (int)max_pages, P, (const float*)prm.part_o,
          (const float*)prm.part_lse, prm.o_lat, lse);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

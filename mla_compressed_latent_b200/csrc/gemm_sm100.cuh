@@ -94,8 +94,10 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     ptx::prefetch_tmap(&tm_x);
   }
   if (warp == 2) { ptx::tmem_alloc(slot, tmem_cols); ptx::tmem_relinquish(); }
+  grid_dependency_wait();   // the inputs may come from the previous kernel of the stream
   ptx::tc_fence_before();
   __syncthreads();
+  allow_dependents();
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + (slot - raw));
 
@@ -228,7 +230,7 @@ inline int run(const Problem& pr, Params p, cudaStream_t st) {
     if (dev >= 0 && dev < 64) attr_done[dev] = true;
   }
   const dim3 grid(pr.H * ((pr.M + kBM - 1) / kBM), (pr.n_tok + p.tn - 1) / p.tn, pr.splits);
-  mla::launch(head_gemm_kernel, grid, dim3(kThreads), (size_t)smem_bytes(p.tn, p.stages), st, tm_w, tm_x, p);
+  mla::launch_pdl(head_gemm_kernel, grid, dim3(kThreads), (size_t)smem_bytes(p.tn, p.stages), st, tm_w, tm_x, p);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -196,7 +196,7 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     if ((rc = mla::gemm::run({w_dkv_kr, x, 1, C, N, n_tok, ks}, p, st))) return rc;
     const size_t fin_smem = (size_t)N * sizeof(float);
     if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
-    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)p.part, ks, n_tok, s_q,
+    mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(256), fin_smem, st, (const float*)p.part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
            (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);
     return launch_status();

@@ -69,6 +69,8 @@ __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit,
                                      int num_pages) {
   extern __shared__ float z[];
   __shared__ float red[32];
+  grid_dependency_wait();   // launched with programmatic dependent launch after the projection
+  allow_dependents();
   const int tok = blockIdx.x;
   const int b = tok / s_q, t = tok % s_q;
   const int N = d_c + d_r;
