@@ -16,7 +16,9 @@
 // past 2^8) and run the epilogue. No FLOP is done twice; each CTA TMA-loads the rows it needs (the
 // second read hits L2).
 // Work: the tiles of all sequences are laid end to end and cut into one contiguous range per
-// pair; a sequence cut between pairs is written as fp32 partials and merged afterwards.
+// pair; a sequence cut between pairs is written as fp32 partials and merged afterwards. When the
+// batch has no more sequences than pairs and they are close in length, each pair takes one whole
+// sequence instead.
 // Every wait is bounded in time; on expiry the kernel records MLA_ERR_TIMEOUT and drains.
 #pragma once
 
@@ -65,6 +67,7 @@ constexpr int kQCols = kRow / 2;                       // 288 TMEM columns hold 
 constexpr int kSCol0 = kQCols;                         // S buffers at 288, 352, 416
 constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;                   // lazy rescale threshold (log2 units)
+constexpr bool kExpHalf2 = true;                       // softmax exponentials two per SFU op (f16x2)
 constexpr int kThreads = 384;                          // 4 control warps + 8 row warps
 constexpr int kGroup = 256;                            // threads of the row warps (4-11)
 constexpr uint64_t kTimeoutNs = 2000000000ull;
@@ -112,8 +115,8 @@ enum Bar : int {
 };
 constexpr int kOffTmemSlot = kOffBar + NUM_BARS * 8;
 constexpr int kOffAbort = kOffTmemSlot + 8;
-constexpr int kOffWork = kOffAbort + 8;                // long long start, end, off_b, b
-constexpr int kSmemUsed = kOffWork + 32;
+constexpr int kOffWork = kOffAbort + 8;                // long long start, end, off_b, b, total tiles
+constexpr int kSmemUsed = kOffWork + 40;
 constexpr int kSmemBytes = kSmemUsed + 1024;           // + alignment slack of the dynamic base
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert((kOffBar % 8) == 0 && (kOffWork % 8) == 0 && (kOffEpi % 1024) == 0 && (kOffStaging % 16) == 0, "alignment");
@@ -180,10 +183,23 @@ __device__ __forceinline__ void softmax_rows(const uint32_t (&sr)[32], int valid
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int c = 8 * j + 2 * t4;
-    const float e00 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j]), scale2, -m0)) : 0.f;
-    const float e01 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 1]), scale2, -m0)) : 0.f;
-    const float e10 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 2]), scale2, -m1)) : 0.f;
-    const float e11 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 3]), scale2, -m1)) : 0.f;
+    float e00, e01, e10, e11;
+    if constexpr (kExpHalf2) {
+      // two exponentials per SFU operation: arguments (at most 2^kRescaleLog2) rounded to f16
+      // (relative error of the result at most about 2^-8, the order of P's own bf16 rounding),
+      // a masked column's argument is -inf, whose exponential is 0
+      const float x00 = (!kMask || c < valid) ? fmaf(__uint_as_float(sr[4 * j]), scale2, -m0) : -INFINITY;
+      const float x01 = (!kMask || c + 1 < valid) ? fmaf(__uint_as_float(sr[4 * j + 1]), scale2, -m0) : -INFINITY;
+      const float x10 = (!kMask || c < valid) ? fmaf(__uint_as_float(sr[4 * j + 2]), scale2, -m1) : -INFINITY;
+      const float x11 = (!kMask || c + 1 < valid) ? fmaf(__uint_as_float(sr[4 * j + 3]), scale2, -m1) : -INFINITY;
+      ptx::ex2_half2(x00, x01, e00, e01);
+      ptx::ex2_half2(x10, x11, e10, e11);
+    } else {
+      e00 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j]), scale2, -m0)) : 0.f;
+      e01 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 1]), scale2, -m0)) : 0.f;
+      e10 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 2]), scale2, -m1)) : 0.f;
+      e11 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 3]), scale2, -m1)) : 0.f;
+    }
     if (j & 1) {
       ls1 += e00 + e01;
       ls3 += e10 + e11;
@@ -240,26 +256,53 @@ struct SegIter {
   }
 };
 
-// One warp: total tiles T, this pair's range [pair*T/P, (pair+1)*T/P), and the sequence holding its
-// first tile. Lane l scans sequences [l*per, (l+1)*per).
+// The work split. Default: the tiles of all sequences laid end to end and cut into one contiguous
+// range per pair (balanced to a tile), pair p taking [p*T/P, (p+1)*T/P). A sequence cut between pairs
+// costs its pairs a segment switch, fp32 partials and the merge; so when there are no more sequences
+// than pairs and the longest is within kSplitSlack tiles of the balanced share, each pair takes one
+// whole sequence instead (pair p takes sequence p; nothing is cut). Both the decode and the merge
+// kernel decide it the same way from seqlens.
+constexpr int kSplitSlack = 12;
+__device__ __forceinline__ bool whole_sequences(int B, int npairs, long long T, int max_tb) {
+  return B <= npairs && (long long)max_tb <= (T + npairs - 1) / npairs + kSplitSlack;
+}
+
+// One warp: total tiles T, this pair's range, and the sequence holding its first tile. Lane l scans
+// sequences [l*per, (l+1)*per).
 __device__ void plan_range(const int32_t* seqlens, int B, int max_tiles, int pair, int npairs, long long* out) {
   const int lane = threadIdx.x & 31;
   const int per = (B + 31) / 32;
   const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
   long long local = 0;
+  int max_tb = 0;
   for (int b = b0; b < b1; ++b) {
     const int L = seqlens[b];
     if (L < 1 || (L + kTile - 1) / kTile > max_tiles) report(MLA_ERR_DEVICE_CHECK);
-    local += tiles_of(L, max_tiles);
+    const int tb = tiles_of(L, max_tiles);
+    local += tb;
+    max_tb = max(max_tb, tb);
   }
   long long incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const long long v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
+    max_tb = max(max_tb, __shfl_xor_sync(0xffffffffu, max_tb, o));
   }
   const long long T = __shfl_sync(0xffffffffu, incl, 31);
   const long long excl = incl - local;
+  if (lane == 0) out[4] = T;
+  if (whole_sequences(B, npairs, T, max_tb)) {
+    // pair p: sequence p whole
+    if (pair >= B) {
+      if (lane == 0) { out[0] = 0; out[1] = 0; out[2] = 0; out[3] = B; }
+    } else if (pair >= b0 && pair < b1) {
+      long long off = excl;
+      for (int b = b0; b < pair; ++b) off += tiles_of(seqlens[b], max_tiles);
+      out[0] = off; out[1] = off + tiles_of(seqlens[pair], max_tiles); out[2] = off; out[3] = pair;
+    }
+    return;
+  }
   const long long start = (long long)pair * T / npairs;
   const long long end = (long long)(pair + 1) * T / npairs;
   if (start < end && start >= excl && start < incl) {
@@ -861,46 +904,47 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
 // pair p covers global tiles [p*T/P, (p+1)*T/P); the pair holding tile x is floor(((x+1)*P - 1) / T).
 __device__ __forceinline__ int pair_of(long long x, long long T, int P) { return (int)(((x + 1) * P - 1) / T); }
 
-__global__ void __launch_bounds__(256)
+// One warp per (sequence, head), 4 heads per block of 128 threads (about 1.4 waves at 48 registers).
+// Each warp finds the sequence's tile range itself (no block barrier), then issues all its
+// partial loads before combining them.
+constexpr int kMergeHeads = 4;
+__global__ void __launch_bounds__(32 * kMergeHeads)
 merge_kernel(const int32_t* __restrict__ seqlens, int B, int max_tiles, int npairs, const float* __restrict__ part_o,
              const float* __restrict__ part_lse, __nv_bfloat16* __restrict__ o_lat, float* __restrict__ lse) {
-  __shared__ long long sh[3];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   grid_dependency_wait();
   allow_dependents();
-  if (warp == 0) {
-    const int per = (B + 31) / 32;
-    const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
-    long long local = 0, before = 0;
-    for (int x = b0; x < b1; ++x) {
-      const int tb = tiles_of(seqlens[x], max_tiles);
-      if (x < b) before += tb;
-      local += tb;
-    }
-    long long incl = local, incl_b = before;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long v = __shfl_up_sync(0xffffffffu, incl, o);
-      const long long w = __shfl_up_sync(0xffffffffu, incl_b, o);
-      if (lane >= o) { incl += v; incl_b += w; }
-    }
-    if (lane == 31) { sh[0] = incl; sh[1] = incl_b; sh[2] = tiles_of(seqlens[b], max_tiles); }
+  // global tile offset of sequence b and the total: lane l sums sequences [l*per, (l+1)*per)
+  const int per = (B + 31) / 32;
+  const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
+  long long local = 0, before = 0;
+  int max_tb = 0;
+  for (int x = b0; x < b1; ++x) {
+    const int tb = tiles_of(__ldg(seqlens + x), max_tiles);
+    if (x < b) before += tb;
+    local += tb;
+    max_tb = max(max_tb, tb);
   }
-  __syncthreads();
-  const long long T = sh[0], off = sh[1], tb = sh[2];
-  if (tb == 0 || T == 0) return;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    local += __shfl_xor_sync(0xffffffffu, local, o);
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    max_tb = max(max_tb, __shfl_xor_sync(0xffffffffu, max_tb, o));
+  }
+  const long long T = local, off = before, tb = tiles_of(__ldg(seqlens + b), max_tiles);
+  if (tb == 0 || T == 0 || whole_sequences(B, npairs, T, max_tb)) return;   // nothing was cut
   const int p0 = pair_of(off, T, npairs), p1 = pair_of(off + tb - 1, T, npairs);
   if (p0 == p1) return;                       // written whole by one pair
-  // one head per warp; lanes cover 16 columns each. A pair with an empty range wrote nothing.
-  const int h = blockIdx.y * 8 + warp;
+  const int h = blockIdx.y * kMergeHeads + warp;
+  // a pair with an empty range wrote nothing; the others' parts in order, lane q holds part p0 + q's lse
   auto slot = [&](int q) -> int {
     const long long start_q = (long long)q * T / npairs;
     if ((long long)(q + 1) * T / npairs <= start_q) return -1;
     return q * 2 + (start_q < off ? 1 : 0);
   };
   float mx = -INFINITY;
-  for (int q0 = p0; q0 <= p1; q0 += 32) {     // the partials' lse values, one lane each
+  for (int q0 = p0; q0 <= p1; q0 += 32) {
     const int q = q0 + lane;
     const int idx = q <= p1 ? slot(q) : -1;
     mx = fmaxf(mx, warp_max(idx >= 0 ? part_lse[(size_t)idx * kH + h] : -INFINITY));
@@ -909,28 +953,34 @@ merge_kernel(const int32_t* __restrict__ seqlens, int B, int max_tiles, int npai
   float acc[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-#pragma unroll 2
-  for (int q = p0; q <= p1; ++q) {
-    const int idx = slot(q);
-    if (idx < 0) continue;
-    const float wgt = exp2f((part_lse[(size_t)idx * kH + h] - mx) * 1.4426950408889634f);
-    tot += wgt;
-    const float4* src = reinterpret_cast<const float4*>(part_o + ((size_t)idx * kH + h) * kDC + lane * 16);
+  // lane covers columns [4 lane + 128 k, +4) for k < 4: every load instruction reads 512 contiguous bytes
+  for (int q = p0; q <= p1; q += 2) {
+    const int i0 = slot(q), i1 = q + 1 <= p1 ? slot(q + 1) : -1;
+    float4 x0[4], x1[4];
+    const float w0 = i0 >= 0 ? exp2f((part_lse[(size_t)i0 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
+    const float w1 = i1 >= 0 ? exp2f((part_lse[(size_t)i1 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
+    const float4* s0 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i0, 0) * kH + h) * kDC) + lane;
+    const float4* s1 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i1, 0) * kH + h) * kDC) + lane;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const float4 v = src[k];
-      acc[4 * k] = fmaf(wgt, v.x, acc[4 * k]);
-      acc[4 * k + 1] = fmaf(wgt, v.y, acc[4 * k + 1]);
-      acc[4 * k + 2] = fmaf(wgt, v.z, acc[4 * k + 2]);
-      acc[4 * k + 3] = fmaf(wgt, v.w, acc[4 * k + 3]);
+      x0[k] = i0 >= 0 ? s0[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+      x1[k] = i1 >= 0 ? s1[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    tot += w0 + w1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc[4 * k] += w0 * x0[k].x + w1 * x1[k].x;
+      acc[4 * k + 1] += w0 * x0[k].y + w1 * x1[k].y;
+      acc[4 * k + 2] += w0 * x0[k].z + w1 * x1[k].z;
+      acc[4 * k + 3] += w0 * x0[k].w + w1 * x1[k].w;
     }
   }
   const float inv = 1.f / tot;
-  uint4* dst = reinterpret_cast<uint4*>(o_lat + ((size_t)b * kH + h) * kDC + lane * 16);
-  dst[0] = make_uint4(ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv), ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                      ptx::pack_bf16x2(acc[4] * inv, acc[5] * inv), ptx::pack_bf16x2(acc[6] * inv, acc[7] * inv));
-  dst[1] = make_uint4(ptx::pack_bf16x2(acc[8] * inv, acc[9] * inv), ptx::pack_bf16x2(acc[10] * inv, acc[11] * inv),
-                      ptx::pack_bf16x2(acc[12] * inv, acc[13] * inv), ptx::pack_bf16x2(acc[14] * inv, acc[15] * inv));
+  uint2* dst = reinterpret_cast<uint2*>(o_lat + ((size_t)b * kH + h) * kDC) + lane;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    dst[32 * k] = make_uint2(ptx::pack_bf16x2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
+                             ptx::pack_bf16x2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
   if (lane == 0) lse[(size_t)b * kH + h] = mx + logf(tot);
 }
 
@@ -1004,7 +1054,7 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   prm.part_lse = prm.part_o + (size_t)2 * max_pairs(num_sms) * kH * kDC;
   prm.sm_scale_log2 = d->sm_scale * 1.4426950408889634f;
   launch_pdl(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
-  launch_pdl(merge_kernel, dim3(B, kH / 8), dim3(256), 0, st, seqlens, (int)B, (int)max_pages, P, (const float*)prm.part_o,
+  launch_pdl(merge_kernel, dim3(B, kH / kMergeHeads), dim3(32 * kMergeHeads), 0, st, seqlens, (int)B, (int)max_pages, P, (const float*)prm.part_o,
          (const float*)prm.part_lse, prm.o_lat, lse);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

@@ -26,7 +26,8 @@ constexpr int kBK = 64;          // K per stage: one 128-byte swizzle row of bf1
 constexpr int kMaxStages = 4;
 constexpr int kThreads = 256;    // warp 0 TMA producer, 1 MMA issuer, 2 TMEM owner, 4-7 epilogue
 constexpr int kABytes = kBK * 128 * 2;   // two boxes of 64 k-rows x 64 features
-constexpr int kBarBytes = 1024;          // barriers + TMEM address slot, ahead of the stages
+constexpr int kBarBytes = 1024;          // barriers, TMEM address slot, RoPE inverse frequencies
+constexpr int kInvFreqOff = 512;         // double [d_r / 2 <= 64] inside the barrier area
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 struct Params {
@@ -138,15 +139,19 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     if (p.rope_in != nullptr) {
       // the rotated tail does not depend on the GEMM: done while the main loop runs, the token
-      // block's tokens dealt out over the head's m-tiles (token j of the block goes to m-tile j % m_tiles)
+      // block's tokens dealt out over the head's m-tiles (token j of the block goes to m-tile j % m_tiles);
+      // the pairs' inverse frequencies are computed once, into shared memory
       const int half = p.d_r / 2;
+      double* inv_freq = reinterpret_cast<double*>(smem_raw + (base + kInvFreqOff - raw));
+      if (row < half) inv_freq[row] = rope_inv_freq(row, p.d_r, p.rope_base);
+      ptx::named_bar_sync(1, 128);
       const int my_tok = (p.tn - mt + m_tiles - 1) / m_tiles;
       for (int i = row; i < my_tok * half; i += 128) {
         const int tok = tok0 + (i / half) * m_tiles + mt, q = i % half;
         if (tok >= p.n_tok) continue;
         const int pos = p.seqlens[tok / p.s_q] - p.s_q + tok % p.s_q;
         float cs, sn;
-        rope_cos_sin(pos, q, p.d_r, p.rope_base, &cs, &sn);
+        rope_cos_sin_at(pos, inv_freq[q], &cs, &sn);
         const __nv_bfloat162 r2 = *reinterpret_cast<const __nv_bfloat162*>(p.rope_in + ((int64_t)tok * p.H + h) * p.d_r + 2 * q);
         const float x0 = __low2float(r2), x1 = __high2float(r2);
         __nv_bfloat16* o = p.y + (int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + p.M;
@@ -186,6 +191,8 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
 // ---- host ----------------------------------------------------------------------------------------
 // Shapes the kernel takes: K a multiple of 64 (whole chunks), M a multiple of 8 (16-byte weight rows).
 inline bool supported(int K, int M) { return K > 0 && K % kBK == 0 && M > 0 && M % 8 == 0; }
+// The rotated tail of the absorbed query keeps one inverse frequency per pair in the barrier area.
+inline bool supported_rope(int d_r) { return d_r > 0 && d_r <= 128; }
 
 inline int tokens_per_cta(int n_tok) { return n_tok <= 32 ? 32 : (n_tok <= 64 ? 64 : 128); }
 

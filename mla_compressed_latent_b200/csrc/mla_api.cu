@@ -196,7 +196,8 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     if ((rc = mla::gemm::run({w_dkv_kr, x, 1, C, N, n_tok, ks}, p, st))) return rc;
     const size_t fin_smem = (size_t)N * sizeof(float);
     if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
-    mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(256), fin_smem, st, (const float*)p.part, ks, n_tok, s_q,
+    const int fin_threads = std::min(1024, (N + 31) / 32 * 32);   // one thread per output column
+    mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)p.part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
            (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);
     return launch_status();
@@ -242,7 +243,7 @@ int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
   const int n_tok = B * s_q;
   const int D = dims->D, H = dims->H, d_c = dims->d_c, d_r = dims->d_r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == MLA_BF16 && mla::gemm::supported(D, d_c)) {
+  if (dtype == MLA_BF16 && mla::gemm::supported(D, d_c) && mla::gemm::supported_rope(d_r)) {
     mla::gemm::Params p{};
     p.mode = 0;
     p.y = reinterpret_cast<__nv_bfloat16*>(q_abs);

@@ -74,19 +74,19 @@ __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit,
   const int tok = blockIdx.x;
   const int b = tok / s_q, t = tok % s_q;
   const int N = d_c + d_r;
+  // the K slices of a column are summed 32 at a time, all 32 loads in flight together
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
     const float* src = part + (int64_t)tok * N + i;
     const int64_t step = (int64_t)n_tok * N;
-    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-    int ks = 0;
-    for (; ks + 4 <= ksplit; ks += 4) {
-      s0 += src[ks * step];
-      s1 += src[(ks + 1) * step];
-      s2 += src[(ks + 2) * step];
-      s3 += src[(ks + 3) * step];
+    float s = 0.f;
+    for (int ks = 0; ks < ksplit; ks += 32) {
+      float v[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) v[k] = (ks + k < ksplit) ? src[(ks + k) * step] : 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; k += 4) s += (v[k] + v[k + 1]) + (v[k + 2] + v[k + 3]);
     }
-    for (; ks < ksplit; ++ks) s0 += src[ks * step];
-    z[i] = (s0 + s1) + (s2 + s3);
+    z[i] = s;
   }
   __syncthreads();
   float ss = 0.f;

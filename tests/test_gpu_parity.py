@@ -89,6 +89,29 @@ def test_decode_absorbed_small(lens, s_q, pages):
         _assert_lse(got_l[b], ref_l[b], "bf16", f"lse seq {b}")
 
 
+def test_decode_workspace_reused_across_calls():
+    """One zero-filled workspace for several calls whose sequences are cut between worker pairs in
+    different places: the per-sequence part counters left by a call must not leak into the next."""
+    rounds = [[4096, 129, 2049, 64, 5000], [300, 7000, 65], [131072], [4096] * 9, [1, 2]]
+    max_b = max(len(r) for r in rounds)
+    dims0 = Dims.of(synth.workload("dsv3_b64_l4096", B=max_b, lengths=("list", tuple([64] * max_b))))
+    need = ops.mla_decode_workspace_size(dims0, torch.bfloat16, max_b, 1, 2048)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for i, lens in enumerate(rounds):
+        w = synth.workload("dsv3_b64_l4096", B=len(lens), lengths=("list", tuple(lens)), pages="random")
+        case = Case(w, with_weights=False)
+        dev = case.to_device()
+        assert dev["table"].shape[1] <= 2048
+        o_lat, lse = ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), dev["table"],
+                                             dev["seqlens"], workspace=ws)
+        torch.cuda.synchronize()
+        assert ops.mla_check_status() == 0
+        ref_o, ref_l = _oracle_absorbed(case, case.q_abs64)
+        for b in range(w.B):
+            _assert_close(o_lat[b].float().cpu().numpy(), ref_o[b], "bf16", f"round {i} o_lat seq {b}")
+            _assert_lse(lse[b].cpu().numpy(), ref_l[b], "bf16", f"round {i} lse seq {b}")
+
+
 def test_decode_absorbed_fp32_smallem_shapes():
     w = synth.workload("smallem_fp32", B=3, lengths=("list", (512, 65, 1)))
     case = Case(w, with_weights=False)
