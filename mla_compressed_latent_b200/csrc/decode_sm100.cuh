@@ -67,7 +67,7 @@ constexpr int kQCols = kRow / 2;                       // 288 TMEM columns hold 
 constexpr int kSCol0 = kQCols;                         // S buffers at 288, 352, 416
 constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;                   // lazy rescale threshold (log2 units)
-constexpr bool kExpHalf2 = true;                       // softmax exponentials two per SFU op (f16x2)
+constexpr bool kExpHalf2 = false;                      // softmax exponentials two per SFU op (f16x2)
 constexpr int kThreads = 384;                          // 4 control warps + 8 row warps
 constexpr int kGroup = 256;                            // threads of the row warps (4-11)
 constexpr uint64_t kTimeoutNs = 2000000000ull;

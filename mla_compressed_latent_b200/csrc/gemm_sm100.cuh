@@ -23,7 +23,7 @@ namespace gemm {
 
 constexpr int kBM = 128;         // output features per CTA (MMA M)
 constexpr int kBK = 64;          // K per stage: one 128-byte swizzle row of bf16
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 8;           // a CTA streaming a long K keeps up to 8 chunks (192 KB) in flight
 constexpr int kThreads = 256;    // warp 0 TMA producer, 1 MMA issuer, 2 TMEM owner, 4-7 epilogue
 constexpr int kABytes = kBK * 128 * 2;   // two boxes of 64 k-rows x 64 features
 constexpr int kBarBytes = 1024;          // barriers, TMEM address slot, RoPE inverse frequencies
@@ -54,6 +54,15 @@ struct Params {
 __host__ __device__ constexpr int stage_bytes(int tn) { return kABytes + tn * 128; }
 __host__ __device__ constexpr int smem_bytes(int tn, int stages) { return 1024 + kBarBytes + stages * stage_bytes(tn); }
 
+// Optional phase stamps (profiling builds with -DMLA_DECODE_PROFILE; absent otherwise).
+#ifdef MLA_DECODE_PROFILE
+__device__ unsigned long long g_gemm_time[1024][6];
+#define GEMM_TIME(k) do { const int cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+    if (cta_ < 1024) g_gemm_time[cta_][k] = ptx::globaltimer(); } while (0)
+#else
+#define GEMM_TIME(k) do {} while (0)
+#endif
+
 __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = 0;
@@ -74,6 +83,7 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) GEMM_TIME(0);
   const int m_tiles = (p.M + kBM - 1) / kBM;
   const int h = blockIdx.x / m_tiles, mt = blockIdx.x % m_tiles;
   const int tok0 = blockIdx.y * p.tn;
@@ -100,6 +110,7 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
   __syncthreads();
   allow_dependents();
   ptx::tc_fence_after();
+  if (threadIdx.x == 0) GEMM_TIME(1);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + (slot - raw));
 
   if (warp == 0 && lane == 0) {
@@ -146,20 +157,36 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
       if (row < half) inv_freq[row] = rope_inv_freq(row, p.d_r, p.rope_base);
       ptx::named_bar_sync(1, 128);
       const int my_tok = (p.tn - mt + m_tiles - 1) / m_tiles;
-      for (int i = row; i < my_tok * half; i += 128) {
-        const int tok = tok0 + (i / half) * m_tiles + mt, q = i % half;
-        if (tok >= p.n_tok) continue;
-        const int pos = p.seqlens[tok / p.s_q] - p.s_q + tok % p.s_q;
-        float cs, sn;
-        rope_cos_sin_at(pos, inv_freq[q], &cs, &sn);
-        const __nv_bfloat162 r2 = *reinterpret_cast<const __nv_bfloat162*>(p.rope_in + ((int64_t)tok * p.H + h) * p.d_r + 2 * q);
-        const float x0 = __low2float(r2), x1 = __high2float(r2);
-        __nv_bfloat16* o = p.y + (int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + p.M;
-        *reinterpret_cast<__nv_bfloat162*>(o + 2 * q) = __floats2bfloat162_rn(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+      // four pairs per round, their loads issued together
+      for (int i0 = row; i0 < my_tok * half; i0 += 4 * 128) {
+        __nv_bfloat162 r2[4];
+        int tok[4], q[4], pos[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + 128 * u;
+          tok[u] = tok0 + (i / half) * m_tiles + mt;
+          q[u] = i % half;
+          const bool live = i < my_tok * half && tok[u] < p.n_tok;
+          if (!live) tok[u] = -1;
+          r2[u] = live ? *reinterpret_cast<const __nv_bfloat162*>(p.rope_in + ((int64_t)tok[u] * p.H + h) * p.d_r + 2 * q[u])
+                       : __floats2bfloat162_rn(0.f, 0.f);
+          pos[u] = live ? p.seqlens[tok[u] / p.s_q] - p.s_q + tok[u] % p.s_q : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (tok[u] < 0) continue;
+          float cs, sn;
+          rope_cos_sin_at(pos[u], inv_freq[q[u]], &cs, &sn);
+          const float x0 = __low2float(r2[u]), x1 = __high2float(r2[u]);
+          __nv_bfloat16* o = p.y + (int64_t)tok[u] * p.y_tok_stride + (int64_t)h * p.y_head_stride + p.M;
+          *reinterpret_cast<__nv_bfloat162*>(o + 2 * q[u]) = __floats2bfloat162_rn(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+        }
       }
     }
+    if (threadIdx.x == 128) GEMM_TIME(2);
     const bool ok = __all_sync(0xffffffffu, wait(done, 0));
     ptx::tc_fence_after();
+    if (threadIdx.x == 128) GEMM_TIME(3);
     if (ok) {
       for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
         uint32_t r[32];
@@ -180,12 +207,14 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
       }
     }
   }
+  if (threadIdx.x == 128) GEMM_TIME(4);
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 2) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, tmem_cols);
   }
+  if (threadIdx.x == 0) GEMM_TIME(5);
 }
 
 // ---- host ----------------------------------------------------------------------------------------
@@ -222,7 +251,8 @@ inline int run(const Problem& pr, Params p, cudaStream_t st) {
   p.tn = tokens_per_cta(pr.n_tok);
   const int chunks = pr.K / kBK;
   p.chunks_per_split = (chunks + pr.splits - 1) / pr.splits;
-  p.stages = std::min(kMaxStages, p.chunks_per_split);
+  constexpr int kSmemMax = 232448;   // 227 KB per CTA
+  p.stages = std::min({kMaxStages, p.chunks_per_split, (kSmemMax - 2048) / stage_bytes(p.tn)});
   CUtensorMap tm_w, tm_x;
   if (!tmap::make_bf16_sw128(&tm_w, pr.w, pr.M, (int64_t)pr.H * pr.K, pr.M, kBK)) return MLA_ERR_INVALID_ARG;
   if (!tmap::make_bf16_sw128(&tm_x, pr.x, (int64_t)pr.H * pr.K, pr.n_tok, (int64_t)pr.H * pr.K, p.tn))
@@ -231,8 +261,7 @@ inline int run(const Problem& pr, Params p, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-    if (cudaFuncSetAttribute(head_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_bytes(128, kMaxStages)) != cudaSuccess)
+    if (cudaFuncSetAttribute(head_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess)
       return MLA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_done[dev] = true;
   }
