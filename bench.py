@@ -60,6 +60,25 @@ def load_peaks():
 # ------------------------------------------------------------------------------------------------
 # algorithmic counts of the decode kernel (bytes that must move, FLOPs that must be done)
 # ------------------------------------------------------------------------------------------------
+# DRAM traffic of one decode_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum) from an
+# ncu capture at dsv3_b64_l4096; reported only while the kernel's sources are the ones it was taken
+# on (their hash), otherwise the roofline's traffic is null.
+DECODE_TRAFFIC = {"workload": "dsv3_b64_l4096", "bytes": 311_597_568 + 5_854_464, "sources_sha256_16": "39ef6e30ec242638"}
+DECODE_SOURCES = ("decode_sm100.cuh", "ptx_sm100.cuh", "common.cuh")
+
+
+def decode_traffic(workload):
+    import hashlib
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "mla_compressed_latent_b200", "csrc")
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    if workload == DECODE_TRAFFIC["workload"] and h.hexdigest()[:16] == DECODE_TRAFFIC["sources_sha256_16"]:
+        return DECODE_TRAFFIC["bytes"]
+    return None
+
+
 def decode_counts(w, lens):
     total = int(sum(int(L) for L in lens))
     e = 2 if w.dtype == "bf16" else 4
@@ -402,7 +421,7 @@ def main():
         "decode_us": dec_ms * 1e3,
         "step_breakdown_us": breakdown,
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_kind,
+                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": decode_traffic(w.name), "peak_source": peak_kind,
                      "kernel": "mla_decode_absorbed (decode + split merge)",
                      "tensor_tflops": achieved_tf, "tensor_frac": achieved_tf / peaks["bf16_tflops"],
                      "bound_frac": max(bytes_ / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) / (dec_ms / 1e3)},
