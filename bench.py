@@ -272,6 +272,90 @@ def build_inputs(w, device):
     return dev
 
 
+def run_grouped(args, w, dims, device, world, rank, local):
+    """The GQLA grouped decode (g key/value groups, shared RoPE key) on its own: each step is one
+    mla_decode_gqla_grouped call over the whole batch (RoPE of the query included)."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import synth
+    from mla_compressed_latent_b200 import ops
+    from mla_compressed_latent_b200.ops import GqaCache
+    lens = synth.seq_lengths(w)
+    table, num_pages = synth.block_table(w, lens)
+    n = num_pages * 64
+    K = torch.empty(n, w.g, w.D, dtype=torch.bfloat16, device=device)
+    V = torch.empty(n, w.g, w.d_v, dtype=torch.bfloat16, device=device)
+    R = torch.empty(n, w.d_r, dtype=torch.bfloat16, device=device)
+    for start, k, v, r in synth.gqla_cache_chunks(w, n):
+        K[start:start + len(k)] = torch.from_numpy(k).to(device=device, dtype=torch.bfloat16)
+        V[start:start + len(k)] = torch.from_numpy(v).to(device=device, dtype=torch.bfloat16)
+        R[start:start + len(k)] = torch.from_numpy(r).to(device=device, dtype=torch.bfloat16)
+    step_in = synth.decode_step_inputs(w)
+    qn = torch.from_numpy(step_in["q_nope"]).to(device=device, dtype=torch.bfloat16)
+    qr = torch.from_numpy(step_in["q_rope_raw"]).to(device=device, dtype=torch.bfloat16)
+    gcache = GqaCache(K, V, R, num_pages)
+    seqlens = torch.from_numpy(lens).to(device)
+    tbl = torch.from_numpy(table).to(device)
+    out = torch.empty(w.B, w.s_q, w.H, w.d_v, dtype=torch.bfloat16, device=device)
+    lse = torch.empty(w.B, w.s_q, w.H, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ops.mla_decode_gqla_grouped(dims, qn, qr, gcache, tbl, seqlens, out=out, lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = ops.mla_launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    launches = ops.mla_launch_count() - n0
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    total = int(lens.sum())
+    n_tok = w.B * w.s_q
+    # per cached position: K and V of every group plus the shared RoPE key; per token: the query
+    # parts, the head outputs and the lse
+    bytes_ = total * (w.g * (w.D + w.d_v) + w.d_r) * 2 + n_tok * w.H * (w.D + w.d_r + w.d_v) * 2 + n_tok * w.H * 4
+    flops = total * w.H * 2 * ((w.D + w.d_r) + w.d_v)
+    peaks, peak_kind = load_peaks()
+    sec = ms / 1e3 / args.steps
+    gbs = bytes_ / sec / 1e9
+    line = {
+        "metric": METRIC, "value": world * total / sec, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "seq_len": w.lengths[1] if w.lengths[0] == "fixed" else list(w.lengths),
+                   "H": w.H, "g": w.g, "D": w.D, "d_r": w.d_r, "d_v": w.d_v, "s_q": w.s_q,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2: {total * (w.g * (w.D + w.d_v) + w.d_r) * 2 / 1e6:.0f} MB cache read per step"},
+        "tokens_per_s": world * n_tok / sec,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_kind,
+                     "kernel": "mla_decode_gqla_grouped (decode + split merge)",
+                     "tensor_tflops": flops / sec / 1e12},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
@@ -293,6 +377,8 @@ def main():
 
     w = synth.workload(args.workload)
     dims = Dims.of(w)
+    if w.g:
+        return run_grouped(args, w, dims, device, world, rank, local)
     dev = build_inputs(w, device)
     cache = LatentCache(dev["pool"][:, :w.d_c], dev["pool"][:, w.d_c:], dev["num_pages"])
     n_tok = w.B * w.s_q

@@ -56,7 +56,7 @@ constexpr int kKChunks = kRow / 64;                    // 9 chunks per tile on t
 constexpr int kVChunks = kDC / 64;                     // 8 chunks per tile on the output CTA
 constexpr int kGroupChunks = 3;                       // score CTA: a ring of 3-chunk groups (24 KB),
 constexpr int kGroupsPerTile = kKChunks / kGroupChunks;// 3 per tile, each released as soon as its
-constexpr int kRing = 7;                               // 12 MMAs are done
+constexpr int kRing = 8;                               // 12 MMAs are done
 constexpr int kGroupBytes = kGroupChunks * kChunkBytes;// 24576
 constexpr int kQGroups = 6;                            // a sequence's Q̃ travels the ring first: 18 boxes of
                                                        // 64 heads x 64 columns in 6 groups
@@ -100,8 +100,10 @@ constexpr int kOffEpi = kOffPSlots + kPSlots * kSlotStride;           // 200704
 constexpr int kEpiWarpBytes = 2048;
 constexpr int kRegion1 = kOffEpi + 8 * kEpiWarpBytes;                 // 217088
 constexpr int kRegion = kRegion0 > kRegion1 ? kRegion0 : kRegion1;
-constexpr int kOffStats = kRegion;                     // float [2][128] 1/l per row   (output CTA)
-constexpr int kOffBar = kOffStats + 2 * kH * 4;
+// float [128] 1/l per row (output CTA). One buffer is enough: the score CTA writes a segment's
+// values only after the output CTA released the previous segment's (STATS_EMPTY).
+constexpr int kOffStats = kRegion;
+constexpr int kOffBar = kOffStats + kH * 4;
 // Barriers. Score CTA: K_*, S_*, Q_FULL, P_EMPTY, P_WRITTEN, STG_FREE, STATS_EMPTY. Output CTA:
 // V_*, P_FULL, P_LOCAL, P_EMPTY, STATS_FULL. P_EMPTY[slot] completes in both CTAs when the O MMAs
 // of the slot's tile are done (one multicast commit). Arrivals from the other CTA reach P_EMPTY,
@@ -659,7 +661,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             float* lse_dst = partial ? p.part_lse + ((size_t)pair * 2 + (seg > 0)) * kH : p.lse + (size_t)b * kH;
             lse_dst[r0] = (m0 + log2f(l0)) * 0.69314718055994531f;
             lse_dst[r0 + 8] = (m1 + log2f(l1)) * 0.69314718055994531f;
-            const uint32_t st = stats_remote + ((seg & 1u) * kH) * 4u;
+            const uint32_t st = stats_remote;
             ptx::st_cluster_f32(st + r0 * 4u, 1.f / l0);
             ptx::st_cluster_f32(st + (r0 + 8) * 4u, 1.f / l1);
             ptx::mbar_arrive_remote(bar(STATS_FULL), 1);
@@ -822,7 +824,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
         // every row warp meets here once per segment and agrees whether to go on
         if (ptx::named_bar_or(1, kGroup, !ok)) break;
         ptx::tc_fence_after();
-        const float inv_l = stats[(seg & 1u) * kH + h];
+        const float inv_l = stats[h];
         const bool partial = !(t_lo == 0 && t_hi == tiles_b);
         // 32 columns of the warp's 32 rows at a time: each thread (row) scales its values and puts
         // them in the warp's buffer as one 64-byte row (16-byte chunks XOR-swizzled by row / 2, so
