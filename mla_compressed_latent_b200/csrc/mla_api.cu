@@ -14,6 +14,7 @@
 #include "simt.cuh"
 #include "decode_sm100.cuh"
 #include "gemm_sm100.cuh"
+#include "gqla_sm100.cuh"
 
 namespace {
 
@@ -141,7 +142,7 @@ const char* mla_status_string(int s) {
 uint64_t mla_launch_count(void) { return mla::g_launches.load(std::memory_order_relaxed); }
 
 const char* mla_build_info(void) {
-  return "libmla: sm_100a; kernels: simt (fp32/bf16 all steps), sm100 absorbed decode and per-head projections (tcgen05/TMA)";
+  return "libmla: sm_100a; kernels: simt (fp32/bf16 all steps), sm100 absorbed decode, GQLA grouped decode and per-head projections (tcgen05/TMA)";
 }
 
 int mla_check_status(void* stream) {
@@ -385,7 +386,10 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
 // ------------------------------------------------------------------------------------------------
 size_t mla_gqla_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, int32_t max_pages) {
   if (check_dims(dims) || check_dtype(dtype) || B <= 0 || s_q <= 0 || max_pages <= 0) return 0;
-  return simt_decode_ws(B * s_q, dims->H, dims->d_v, max_pages);
+  size_t ws = simt_decode_ws(B * s_q, dims->H, dims->d_v, max_pages);
+  if (dims->g > 0 && mla::gqla::supported(dims, dtype, s_q))
+    ws = std::max(ws, mla::gqla::workspace_bytes(dims, B, max_pages, num_sms()));
+  return ws;
 }
 
 int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_nope,
@@ -408,6 +412,9 @@ int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, in
   if (!stride_ok(cache->k_stride, dtype, (int64_t)dims->g * dims->D) ||
       !stride_ok(cache->v_stride, dtype, (int64_t)dims->g * dims->d_v) || !stride_ok(cache->rope_stride, dtype, dims->d_r))
     return MLA_ERR_INVALID_ARG;
+  if (mla::gqla::supported(dims, dtype, s_q))
+    return mla::gqla::launch_gqla(dims, B, q_nope, q_rope_raw, cache, block_table, max_pages, seqlens, out, lse,
+                                  workspace, ws_bytes, num_sms(), reinterpret_cast<cudaStream_t>(stream));
   if (hpg % mla::simt::DEC_HEADS || dims->d_v % 32 || dims->d_v > 32 * mla::simt::DEC_MAX_OV) return MLA_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int n_tok = B * s_q;

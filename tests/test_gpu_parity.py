@@ -392,6 +392,39 @@ def test_gqla_grouped_equals_absorbed_on_same_weights():
         assert np.abs(ref_la - ref_l).max() < 5e-3      # the two paths agree up to bf16 storage
 
 
+def test_gqla_ragged_lengths_and_splits():
+    """The grouped path on one position, tile edges (127/128/129 of a 128-position tile), a partial
+    last tile and a long sequence cut into splits (short sequences leave empty splits), every head."""
+    lens = (1, 127, 128, 129, 300, 8192)
+    w = synth.workload("gqla_g8_b32_l8192", B=len(lens), lengths=("list", lens), pages="random")
+    lens_a = np.asarray(lens, np.int32)
+    table, num_pages = synth.block_table(w, lens_a)
+    n = num_pages * 64
+    K = torch.empty(n, w.g, w.D, dtype=torch.bfloat16)
+    V = torch.empty(n, w.g, w.d_v, dtype=torch.bfloat16)
+    R = torch.empty(n, w.d_r, dtype=torch.bfloat16)
+    for start, k, v, r in synth.gqla_cache_chunks(w, n):
+        K[start:start + len(k)] = torch.from_numpy(k)
+        V[start:start + len(k)] = torch.from_numpy(v)
+        R[start:start + len(k)] = torch.from_numpy(r)
+    step = synth.decode_step_inputs(w)
+    qn = torch.from_numpy(step["q_nope"]).to(torch.bfloat16)
+    qr = torch.from_numpy(step["q_rope_raw"]).to(torch.bfloat16)
+    gcache = GqaCache(K.cuda(), V.cuda(), R.cuda(), num_pages)
+    out, lse = ops.mla_decode_gqla_grouped(Dims.of(w), qn.cuda(), qr.cuda(), gcache, torch.from_numpy(table).cuda(),
+                                           torch.from_numpy(lens_a).cuda())
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    Kd, Vd, Rd = K.double().numpy(), V.double().numpy(), R.double().numpy()
+    for b, L in enumerate(lens):
+        p = np.arange(L)
+        idx = table[b, p // 64].astype(np.int64) * 64 + p % 64
+        q_rot = O.rope(qr[b].double().numpy(), np.full((1, w.H), L - 1))
+        ref, ref_l = O.gqla_grouped_decode(qn[b].double().numpy(), q_rot, Kd[idx], Vd[idx], Rd[idx], L, w.sm_scale, w.g)
+        _assert_close(out[b].double().cpu().numpy(), ref, "bf16", f"grouped seq {b} (L={L})")
+        _assert_lse(lse[b].cpu().numpy(), ref_l, "bf16", f"grouped lse seq {b} (L={L})")
+
+
 def test_gqla_full_size_sampled():
     w = synth.workload("gqla_g8_b32_l8192")
     lens = synth.seq_lengths(w)
