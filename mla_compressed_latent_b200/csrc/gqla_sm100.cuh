@@ -30,7 +30,8 @@ constexpr int kTile = 128;               // positions per tile = two pages
 constexpr int kBox = 64 * 128;           // one TMA box: 64 rows x 64 bf16 (8 KB)
 constexpr int kKRBytes = 6 * kBox;       // K (2 column chunks x 2 pages) + RoPE key (2 pages)
 constexpr int kVBytes = 4 * kBox;        // V (2 column chunks x 2 pages)
-constexpr int kStages = 2;
+constexpr int kKRStages = 2;             // [K_g ; k_r] tiles in flight (released by the tile's score MMAs)
+constexpr int kVStages = 3;              // V_g tiles in flight (held one tile longer, until the output MMA)
 constexpr int kQBytes = 3 * kHG * 128;   // [q (2 chunks) ; q_r (1 chunk)] x 16 heads, 128-byte swizzle
 constexpr int kPBytes = 2 * kHG * 128;   // Pᵀ: 16 heads x 128 positions (2 chunks)
 constexpr int kThreads = 256;            // 0 TMA, 1 MMA, 2 TMEM, 3 idle, 4-7 compute
@@ -39,15 +40,15 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // shared memory (from a 1024-aligned base)
 constexpr int kOffKR = 0;
-constexpr int kOffV = kOffKR + kStages * kKRBytes;      // 98304
-constexpr int kOffQ = kOffV + kStages * kVBytes;        // 163840
-constexpr int kOffP = kOffQ + 2 * kQBytes;              // 176128
+constexpr int kOffV = kOffKR + kKRStages * kKRBytes;    // 98304
+constexpr int kOffQ = kOffV + kVStages * kVBytes;       // 196608
+constexpr int kOffP = kOffQ + 2 * kQBytes;              // 208896
 constexpr int kOffRed = kOffP + 2 * kPBytes;            // float [2][4][16] per-warp head maxima; [4][16] sums
 constexpr int kOffInvFreq = kOffRed + 3 * 4 * kHG * 4;  // double [32]
 constexpr int kOffBar = kOffInvFreq + 32 * 8;
 enum Bar : int {
-  KR_FULL = 0, KR_EMPTY = KR_FULL + kStages, V_FULL = KR_EMPTY + kStages, V_EMPTY = V_FULL + kStages,
-  S_FULL = V_EMPTY + kStages, S_EMPTY = S_FULL + 2, P_READY = S_EMPTY + 2, P_FREE = P_READY + 2,
+  KR_FULL = 0, KR_EMPTY = KR_FULL + kKRStages, V_FULL = KR_EMPTY + kKRStages, V_EMPTY = V_FULL + kVStages,
+  S_FULL = V_EMPTY + kVStages, S_EMPTY = S_FULL + 2, P_READY = S_EMPTY + 2, P_FREE = P_READY + 2,
   Q_FULL = P_FREE + 2, Q_EMPTY = Q_FULL + 2, NUM_BARS = Q_EMPTY + 2
 };
 constexpr int kOffTmemSlot = kOffBar + NUM_BARS * 8;
@@ -121,10 +122,8 @@ gqla_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
   const int units = p.B * p.g * p.nsplit;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      ptx::mbar_init(bar(KR_FULL + i), 1); ptx::mbar_init(bar(KR_EMPTY + i), 1);
-      ptx::mbar_init(bar(V_FULL + i), 1); ptx::mbar_init(bar(V_EMPTY + i), 1);
-    }
+    for (int i = 0; i < kKRStages; ++i) { ptx::mbar_init(bar(KR_FULL + i), 1); ptx::mbar_init(bar(KR_EMPTY + i), 1); }
+    for (int i = 0; i < kVStages; ++i) { ptx::mbar_init(bar(V_FULL + i), 1); ptx::mbar_init(bar(V_EMPTY + i), 1); }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bar(S_FULL + i), 1); ptx::mbar_init(bar(S_EMPTY + i), 128);
       ptx::mbar_init(bar(P_READY + i), 128); ptx::mbar_init(bar(P_FREE + i), 1);
@@ -152,7 +151,8 @@ gqla_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         const Unit x = unit_of(p, u);
         const int pages = (x.L + 63) / 64;
         for (int t = x.t0; t < x.t1 && ok; ++t, ++i) {
-          const uint32_t s = i % kStages, ph = ((i / kStages) & 1u) ^ 1u;
+          const uint32_t s = i % kKRStages, ph = ((i / kKRStages) & 1u) ^ 1u;
+          const uint32_t sv = i % kVStages, phv = ((i / kVStages) & 1u) ^ 1u;
           int pg[2];
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
@@ -178,21 +178,21 @@ gqla_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             ptx::tma_load_2d(kr + 2 * kBox + j * kBox, &tm_k, x.gi * kD + 64, pg[j] * 64, bar(KR_FULL + s));
             ptx::tma_load_2d(kr + 4 * kBox + j * kBox, &tm_r, 0, pg[j] * 64, bar(KR_FULL + s));
           }
-          if (!(ok = wait_bar(bar(V_EMPTY + s), ph, abort_flag))) break;
-          const uint32_t vv = base + kOffV + s * kVBytes;
-          ptx::mbar_arrive_expect_tx(bar(V_FULL + s), kVBytes);
+          if (!(ok = wait_bar(bar(V_EMPTY + sv), phv, abort_flag))) break;
+          const uint32_t vv = base + kOffV + sv * kVBytes;
+          ptx::mbar_arrive_expect_tx(bar(V_FULL + sv), kVBytes);
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            ptx::tma_load_2d(vv + j * kBox, &tm_v, x.gi * kDV, pg[j] * 64, bar(V_FULL + s));
-            ptx::tma_load_2d(vv + 2 * kBox + j * kBox, &tm_v, x.gi * kDV + 64, pg[j] * 64, bar(V_FULL + s));
+            ptx::tma_load_2d(vv + j * kBox, &tm_v, x.gi * kDV, pg[j] * 64, bar(V_FULL + sv));
+            ptx::tma_load_2d(vv + 2 * kBox + j * kBox, &tm_v, x.gi * kDV + 64, pg[j] * 64, bar(V_FULL + sv));
           }
         }
       }
       // loads in flight land before the CTA may exit
-      for (uint32_t k = (i > (uint32_t)kStages ? i - kStages : 0); k < i; ++k) {
-        wait_bar(bar(KR_FULL + k % kStages), (k / kStages) & 1u, abort_flag);
-        wait_bar(bar(V_FULL + k % kStages), (k / kStages) & 1u, abort_flag);
-      }
+      for (uint32_t k = (i > (uint32_t)kKRStages ? i - kKRStages : 0); k < i; ++k)
+        wait_bar(bar(KR_FULL + k % kKRStages), (k / kKRStages) & 1u, abort_flag);
+      for (uint32_t k = (i > (uint32_t)kVStages ? i - kVStages : 0); k < i; ++k)
+        wait_bar(bar(V_FULL + k % kVStages), (k / kVStages) & 1u, abort_flag);
     }
   } else if (warp == 1) {
     // ---- MMA issuer (lane 0; the warp zeroes V rows past a sequence's end). Order within a unit: S
@@ -203,9 +203,9 @@ gqla_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     bool ok = true;
     int prev_first = 1, prev_valid = kTile;   // the pending O tile: first of its unit? valid rows
     auto issue_o = [&](uint32_t j) -> bool {
-      const uint32_t s = j % kStages, pb = j % 2;
+      const uint32_t s = j % kVStages, pb = j % 2;
       if (!wait_bar_warp(bar(P_READY + pb), (j / 2) & 1u, abort_flag)) return false;
-      if (!wait_bar_warp(bar(V_FULL + s), (j / kStages) & 1u, abort_flag)) return false;
+      if (!wait_bar_warp(bar(V_FULL + s), (j / kVStages) & 1u, abort_flag)) return false;
       uint8_t* vst = gbase + kOffV + s * kVBytes;
       if (prev_valid < kTile) {   // V rows past the end may hold anything (0 * NaN = NaN): zero them
         const int zr = kTile - prev_valid;
@@ -245,9 +245,9 @@ gqla_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         continue;
       }
       for (int t = x.t0; t < x.t1; ++t, ++i) {
-        const uint32_t s = i % kStages, sb = i % 2;
+        const uint32_t s = i % kKRStages, sb = i % 2;
         if (!(ok = wait_bar_warp(bar(S_EMPTY + sb), ((i / 2) & 1u) ^ 1u, abort_flag))) break;
-        if (!(ok = wait_bar_warp(bar(KR_FULL + s), (i / kStages) & 1u, abort_flag))) break;
+        if (!(ok = wait_bar_warp(bar(KR_FULL + s), (i / kKRStages) & 1u, abort_flag))) break;
         if (lane == 0) {
           ptx::tc_fence_after();
           const uint32_t kr = base + kOffKR + s * kKRBytes, qq = base + kOffQ + qb * kQBytes;
