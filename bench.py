@@ -63,7 +63,7 @@ def load_peaks():
 # DRAM traffic of one decode_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum) from an
 # ncu capture at dsv3_b64_l4096; reported only while the kernel's sources are the ones it was taken
 # on (their hash), otherwise the roofline's traffic is null.
-DECODE_TRAFFIC = {"workload": "dsv3_b64_l4096", "bytes": 311_597_568 + 5_854_464, "sources_sha256_16": "39ef6e30ec242638"}
+DECODE_TRAFFIC = {"workload": "dsv3_b64_l4096", "bytes": 311_548_416 + 4_218_880, "sources_sha256_16": "2e928e5a402f90c0"}
 DECODE_SOURCES = ("decode_sm100.cuh", "ptx_sm100.cuh", "common.cuh")
 
 
