@@ -65,17 +65,20 @@ def load_peaks():
 # on (their hash), otherwise the roofline's traffic is null.
 DECODE_TRAFFIC = {"workload": "dsv3_b64_l4096", "bytes": 311_548_416 + 4_218_880, "sources_sha256_16": "2e928e5a402f90c0"}
 DECODE_SOURCES = ("decode_sm100.cuh", "ptx_sm100.cuh", "common.cuh")
+# the same for one gqla_kernel launch at gqla_g8_b32_l8192
+GQLA_TRAFFIC = {"workload": "gqla_g8_b32_l8192", "bytes": 1_115_177_472 + 11_111_936, "sources_sha256_16": "9275cd6940a94824"}
+GQLA_SOURCES = ("gqla_sm100.cuh", "ptx_sm100.cuh", "common.cuh")
 
 
-def decode_traffic(workload):
+def captured_traffic(workload, record=DECODE_TRAFFIC, sources=DECODE_SOURCES):
     import hashlib
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "mla_compressed_latent_b200", "csrc")
     h = hashlib.sha256()
-    for name in DECODE_SOURCES:
+    for name in sources:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
-    if workload == DECODE_TRAFFIC["workload"] and h.hexdigest()[:16] == DECODE_TRAFFIC["sources_sha256_16"]:
-        return DECODE_TRAFFIC["bytes"]
+    if workload == record["workload"] and h.hexdigest()[:16] == record["sources_sha256_16"]:
+        return record["bytes"]
     return None
 
 
@@ -344,7 +347,8 @@ def run_grouped(args, w, dims, device, world, rank, local):
                    "l2": f"inputs larger than L2: {total * (w.g * (w.D + w.d_v) + w.d_r) * 2 / 1e6:.0f} MB cache read per step"},
         "tokens_per_s": world * n_tok / sec,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_kind,
+                     "frac": gbs / peaks["hbm_gbs"],
+                     "traffic": captured_traffic(w.name, GQLA_TRAFFIC, GQLA_SOURCES), "peak_source": peak_kind,
                      "kernel": "mla_decode_gqla_grouped (decode + split merge)",
                      "tensor_tflops": flops / sec / 1e12},
         "gpu_launches": int(launches),
@@ -507,7 +511,7 @@ def main():
         "decode_us": dec_ms * 1e3,
         "step_breakdown_us": breakdown,
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": decode_traffic(w.name), "peak_source": peak_kind,
+                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": captured_traffic(w.name), "peak_source": peak_kind,
                      "kernel": "mla_decode_absorbed (decode + split merge)",
                      "tensor_tflops": achieved_tf, "tensor_frac": achieved_tf / peaks["bf16_tflops"],
                      "bound_frac": max(bytes_ / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) / (dec_ms / 1e3)},
