@@ -269,6 +269,9 @@ def build_inputs(w, device):
         "q_nope_host": torch.from_numpy(step["q_nope"]).to(tdt).pin_memory(),
         "q_rope_host": torch.from_numpy(step["q_rope_raw"]).to(tdt).pin_memory(),
     }
+    if w.d_q:   # the query chain's weights
+        for k in ("W_DQ", "gamma_q", "W_UQ", "W_QR"):
+            dev[k] = torch.from_numpy(W[k]).to(device=device, dtype=tdt)
     dev["x"] = dev["x_host"].to(device)
     dev["q_nope"] = dev["q_nope_host"].to(device)
     dev["q_rope_raw"] = dev["q_rope_host"].to(device)
@@ -401,29 +404,51 @@ def main():
                          dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
     dec_ev = []
+    # a workload with a query latent starts from hidden states: its queries come from x through the
+    # query chain inside the step
+    from_x = w.d_q > 0
+    if from_x:
+        qn_buf = torch.empty(w.B, w.s_q, w.H, w.D, dtype=tdt, device=device)
+        qr_buf = torch.empty(w.B, w.s_q, w.H, w.d_r, dtype=tdt, device=device)
+        ws_q = torch.empty(max(16, L.load().mla_query_workspace_size(ctypes.byref(dc), w.B, w.s_q, w.C, w.d_q)),
+                           dtype=torch.uint8, device=device)
 
     def step(x, q_nope, q_rope, events=None):
         """One decode step. events: None; "decode" (two events around the decode call, which is all
         the timed region carries, so the other kernels keep overlapping their launches); or "all"
-        (an event between every call, for the per-call breakdown outside the timed region)."""
+        (an event after every call, for the per-call breakdown outside the timed region)."""
         every = events == "all"
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if events else None
+        marks = []
+
+        def mark(name):
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            marks.append((name, e))
+
         if every:
-            ev[0].record(stream)
+            mark("start")
+        if from_x:
+            q_nope, q_rope = ops.mla_project_query(dims, x, dev["W_DQ"], dev["gamma_q"], dev["W_UQ"], dev["W_QR"],
+                                                   q_nope=qn_buf, q_rope_raw=qr_buf, workspace=ws_q)
+            if every:
+                mark("project_q")
         ops.mla_append_cache(dims, x, dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache, workspace=ws_app)
         if every:
-            ev[1].record(stream)
+            mark("append")
         ops.mla_absorb_q(dims, q_nope, q_rope, dev["W_UK"], dev["seqlens"], q_abs=q_abs)
         if events:
-            ev[2].record(stream)
+            mark("absorb_q")
         ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"], o_lat=o_lat, lse=lse, workspace=ws_dec)
         if events:
-            ev[3].record(stream)
+            mark("decode")
         ops.mla_out_proj(dims, o_lat, dev["W_UV"], out=out)
         if every:
-            ev[4].record(stream)
+            mark("out_proj")
         if events:
-            dec_ev.append(ev)
+            dec_ev.append(dict(marks))
+
+    def between(m, a, b):
+        return m[a].elapsed_time(m[b])
 
     for _ in range(args.warmup):
         step(dev["x"], dev["q_nope"], dev["q_rope_raw"])
@@ -459,14 +484,15 @@ def main():
     if clk.rejected():
         ms, launches, clk = timed_region()
         remeasured = True
-    dec_ms = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in dec_ev)
+    dec_ms = statistics.mean(between(m, "absorb_q", "decode") for m in dec_ev)
     # per-call breakdown, outside the timed region (its events stop the calls' launches overlapping)
     dec_ev.clear()
     for _ in range(min(args.steps, 50)):
         step(dev["x"], dev["q_nope"], dev["q_rope_raw"], events="all")
     torch.cuda.synchronize()
-    calls = ("append", "absorb_q", "decode", "out_proj")
-    breakdown = {c: statistics.mean(ev[i].elapsed_time(ev[i + 1]) for ev in dec_ev) * 1e3 for i, c in enumerate(calls)}
+    calls = (("project_q",) if from_x else ()) + ("append", "absorb_q", "decode", "out_proj")
+    order = ("start",) + calls
+    breakdown = {c: statistics.mean(between(m, order[i], c) for m in dec_ev) * 1e3 for i, c in enumerate(calls)}
     assert ops.mla_check_status() == 0
 
     # end to end through the public API: pinned host inputs in, host result out, every step
@@ -479,8 +505,10 @@ def main():
     e0.record(stream)
     for _ in range(e_steps):
         x = dev["x_host"].to(device, non_blocking=True)
-        qn = dev["q_nope_host"].to(device, non_blocking=True)
-        qr = dev["q_rope_host"].to(device, non_blocking=True)
+        qn = qr = None
+        if not from_x:
+            qn = dev["q_nope_host"].to(device, non_blocking=True)
+            qr = dev["q_rope_host"].to(device, non_blocking=True)
         step(x, qn, qr)
         out_host.copy_(out, non_blocking=True)
     e1.record(stream)
@@ -490,7 +518,8 @@ def main():
         t = torch.tensor([e_ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e_ms = float(t.item())
-    h2d = sum(t.numel() * t.element_size() for t in (dev["x_host"], dev["q_nope_host"], dev["q_rope_host"]))
+    h2d = sum(t.numel() * t.element_size()
+              for t in ((dev["x_host"],) if from_x else (dev["x_host"], dev["q_nope_host"], dev["q_rope_host"])))
     d2h = out_host.numel() * out_host.element_size()
 
     bytes_, flops, positions = decode_counts(w, dev["lens"])
@@ -520,6 +549,14 @@ def main():
         "e2e": {"value": world * positions / (e_ms / 1e3 / e_steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e_steps},
     }
+    if from_x:
+        # the query chain is bound by its weights: W_DQ, W_UQ, W_QR read once per step
+        e = 2 if w.dtype == "bf16" else 4
+        q_bytes = (w.C * w.d_q + w.d_q * w.H * (w.D + w.d_r)) * e + n_tok * (w.C + w.H * (w.D + w.d_r)) * e
+        q_us = breakdown["project_q"]
+        line["query_chain"] = {"us": q_us, "bytes": q_bytes, "achieved_gbs": q_bytes / (q_us / 1e6) / 1e9,
+                               "frac": q_bytes / (q_us / 1e6) / 1e9 / peaks["hbm_gbs"],
+                               "note": "timed with an event after every call (no launch overlap)"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         pos, tok, el, seqs = oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": pos / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",

@@ -117,6 +117,27 @@ int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, int32_t B, i
                              const mla_latent_cache_t* cache, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * f2. Query projection chain (« L'attention latente … », « L'obstacle : RoPE » and « Le code »:
+ * the query of a new token also passes through a low-rank latent, normalised like the cache's):
+ *   c_q        = RMSNorm(x[b,t,:] · W_DQ) · gamma_q          (width d_q; eps = dims->rms_eps)
+ *   q_nope     = c_q · W_UQ, split into H heads of D          -> q_nope [B, s_q, H, D]
+ *   q_rope_raw = c_q · W_QR, split into H heads of d_r        -> q_rope_raw [B, s_q, H, d_r]
+ * q_rope_raw is not rotated: mla_absorb_q rotates it at the token's position. c_q is rounded to
+ * dtype once, between the two projections (as the cache's latent rows are).
+ *   x [B, s_q, C]   w_dq [C, d_q]   gamma_q [d_q] or NULL (= 1)   w_uq [d_q, H*D]   w_qr [d_q, H*d_r]
+ *   (all dtype, row-major, 16-byte aligned)
+ * workspace: at least mla_query_workspace_size(...) bytes of device memory (fp32 partial sums of
+ * x·W_DQ, then c_q); its contents need not be initialised. Errors: MLA_ERR_INVALID_ARG for null or
+ * misaligned pointers and non-positive sizes, MLA_ERR_WORKSPACE, MLA_ERR_CUDA; nothing is launched
+ * on an error return.
+ * ------------------------------------------------------------------------------------------- */
+size_t mla_query_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C, int32_t d_q);
+int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                      const void* x, int32_t C, int32_t d_q, const void* w_dq, const void* gamma_q,
+                      const void* w_uq, const void* w_qr, void* q_nope, void* q_rope_raw,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * a2. Query absorption (« Ce que DeepSeek fait de plus »: q·(W_UK c) = (q·W_UK)·c).
  *   q_abs[b,t,h, 0:d_c]       = q_nope[b,t,h,:] · W_UK[h]            (W_UK[h] is [D, d_c])
  *   q_abs[b,t,h, d_c:d_c+d_r] = RoPE(q_rope_raw[b,t,h,:], seqlens[b] - s_q + t)

@@ -7,5 +7,5 @@ fails loudly if the library has not been built.
 from .ops import (  # noqa: F401
     Dims, GqaCache, LatentCache, MlaError, mla_absorb_q, mla_append_cache, mla_build_info,
     mla_check_status, mla_decode_absorbed, mla_launch_count, mla_decode_gqla_grouped, mla_decode_workspace_size,
-    mla_out_proj, mla_status_string,
+    mla_out_proj, mla_project_query, mla_status_string,
 )

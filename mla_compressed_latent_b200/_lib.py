@@ -45,6 +45,9 @@ SIGNATURES = {
                                    PI, PI, c_int32, POINTER(MlaLatentCache), c_void_p, c_size_t, c_void_p]),
     "mla_append_cache_noalloc": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_int32, c_void_p, c_void_p,
                                            PI, PI, c_int32, POINTER(MlaLatentCache), c_void_p]),
+    "mla_query_workspace_size": (c_size_t, [PD, c_int32, c_int32, c_int32, c_int32]),
+    "mla_project_query": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_int32, c_int32, c_void_p, c_void_p,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "mla_absorb_q": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, PI, c_void_p,
                                c_void_p]),
     "mla_decode_workspace_size": (c_size_t, [PD, c_int32, c_int32, c_int32, c_int32]),

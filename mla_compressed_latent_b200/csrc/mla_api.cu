@@ -231,6 +231,92 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
 }
 
 // ------------------------------------------------------------------------------------------------
+// f2: query projection chain
+// ------------------------------------------------------------------------------------------------
+namespace {
+// The tensor-core route takes bf16 with every K a whole number of 64-wide chunks.
+bool query_on_tc(int32_t dtype, int C, int d_q, int H, int D, int d_r) {
+  return dtype == MLA_BF16 && mla::gemm::supported(C, d_q) && mla::gemm::supported(d_q, H * D) &&
+         mla::gemm::supported(d_q, H * d_r);
+}
+// fp32 partial sums of x·W_DQ first (256-byte aligned size), then c_q
+size_t query_part_bytes(int ks, int n_tok, int d_q) { return ((size_t)ks * n_tok * d_q * sizeof(float) + 255) / 256 * 256; }
+}  // namespace
+
+size_t mla_query_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C, int32_t d_q) {
+  if (check_dims(dims) || B <= 0 || s_q <= 0 || C <= 0 || d_q <= 0) return 0;
+  const int n_tok = B * s_q;
+  int ks = append_ksplit(n_tok, C, d_q);
+  if (mla::gemm::supported(C, d_q)) ks = std::max(ks, append_tc_splits(n_tok, C, d_q));
+  return query_part_bytes(ks, n_tok, d_q) + (size_t)n_tok * d_q * sizeof(float);
+}
+
+int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x, int32_t C,
+                      int32_t d_q, const void* w_dq, const void* gamma_q, const void* w_uq, const void* w_qr,
+                      void* q_nope, void* q_rope_raw, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (B <= 0 || s_q <= 0 || C <= 0 || d_q <= 0 || !x || !w_dq || !w_uq || !w_qr || !q_nope || !q_rope_raw)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_dq) || (gamma_q && !aligned16(gamma_q)) || !aligned16(w_uq) ||
+      !aligned16(w_qr) || !aligned16(q_nope) || !aligned16(q_rope_raw))
+    return MLA_ERR_INVALID_ARG;
+  const int n_tok = B * s_q, H = dims->H, D = dims->D, d_r = dims->d_r;
+  const bool tc = query_on_tc(dtype, C, d_q, H, D, d_r);
+  const int ks = tc ? append_tc_splits(n_tok, C, d_q) : append_ksplit(n_tok, C, d_q);
+  const size_t pb = query_part_bytes(ks, n_tok, d_q);
+  const size_t need = pb + (size_t)n_tok * d_q * esize(dtype);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* part = reinterpret_cast<float*>(workspace);
+  void* c_q = reinterpret_cast<char*>(workspace) + pb;
+  const size_t fin_smem = (size_t)d_q * sizeof(float);
+  const int fin_threads = std::min(mla::simt::RMS_THREADS, (d_q + 31) / 32 * 32);
+  if (tc) {
+    using T = __nv_bfloat16;
+    mla::gemm::Params p{};
+    p.mode = 1;
+    p.part = part;
+    if ((rc = mla::gemm::run({w_dq, x, 1, C, d_q, n_tok, ks}, p, st))) return rc;
+    if ((rc = set_smem(mla::simt::rms_rows_kernel<T>, fin_smem))) return rc;
+    mla::launch_pdl(mla::simt::rms_rows_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)part, ks,
+                    n_tok, d_q, (const T*)gamma_q, dims->rms_eps, (T*)c_q);
+    // the two up-projections as single-"head" GEMMs over the whole output width
+    mla::gemm::Params pu{};
+    pu.mode = 0;
+    pu.y = reinterpret_cast<T*>(q_nope);
+    pu.y_tok_stride = (int64_t)H * D;
+    if ((rc = mla::gemm::run({w_uq, c_q, 1, d_q, H * D, n_tok, 1}, pu, st))) return rc;
+    mla::gemm::Params pr{};
+    pr.mode = 0;
+    pr.y = reinterpret_cast<T*>(q_rope_raw);
+    pr.y_tok_stride = (int64_t)H * d_r;
+    if ((rc = mla::gemm::run({w_qr, c_q, 1, d_q, H * d_r, n_tok, 1}, pr, st))) return rc;
+    return launch_status();
+  }
+  const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
+  const int tok_blocks = (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK;
+  auto cols = [](int n) { return (n + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS; };
+  auto chain = [&](auto zero) -> int {
+    using T = decltype(zero);
+    launch(mla::simt::proj_partial_kernel<T>, dim3(cols(d_q), tok_blocks, ks), mla::simt::PROJ_COLS, 0, st,
+           (const T*)x, n_tok, C, (const T*)w_dq, d_q, k_chunk, part, (T*)nullptr);
+    int r = set_smem(mla::simt::rms_rows_kernel<T>, fin_smem);
+    if (r) return r;
+    launch(mla::simt::rms_rows_kernel<T>, n_tok, fin_threads, fin_smem, st, (const float*)part, ks, n_tok, d_q,
+           (const T*)gamma_q, dims->rms_eps, (T*)c_q);
+    // one K slice: the kernel writes the finished dot products straight to its output
+    launch(mla::simt::proj_partial_kernel<T>, dim3(cols(H * D), tok_blocks, 1), mla::simt::PROJ_COLS, 0, st,
+           (const T*)c_q, n_tok, d_q, (const T*)w_uq, H * D, d_q, (float*)nullptr, (T*)q_nope);
+    launch(mla::simt::proj_partial_kernel<T>, dim3(cols(H * d_r), tok_blocks, 1), mla::simt::PROJ_COLS, 0, st,
+           (const T*)c_q, n_tok, d_q, (const T*)w_qr, H * d_r, d_q, (float*)nullptr, (T*)q_rope_raw);
+    return launch_status();
+  };
+  return dtype == MLA_F32 ? chain(0.f) : chain(__nv_bfloat16());
+}
+
+// ------------------------------------------------------------------------------------------------
 // a2
 // ------------------------------------------------------------------------------------------------
 int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_nope,

@@ -56,6 +56,20 @@ proj_partial_kernel(const T* __restrict__ x, int n_tok, int K, const T* __restri
   }
 }
 
+// Sum of the K slices of one output column: slice ks of the column is src[ks * step]; 32 loads
+// are in flight together.
+__device__ __forceinline__ float sum_slices(const float* src, int ksplit, int64_t step) {
+  float s = 0.f;
+  for (int ks = 0; ks < ksplit; ks += 32) {
+    float v[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) v[k] = (ks + k < ksplit) ? src[(ks + k) * step] : 0.f;
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) s += (v[k] + v[k + 1]) + (v[k + 2] + v[k + 3]);
+  }
+  return s;
+}
+
 // =============================================================================================
 // a1 epilogue: sum the K slices, RMSNorm the latent part, rotate the RoPE part, store the row.
 // One block per new token.
@@ -74,20 +88,8 @@ __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit,
   const int tok = blockIdx.x;
   const int b = tok / s_q, t = tok % s_q;
   const int N = d_c + d_r;
-  // the K slices of a column are summed 32 at a time, all 32 loads in flight together
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
-    const float* src = part + (int64_t)tok * N + i;
-    const int64_t step = (int64_t)n_tok * N;
-    float s = 0.f;
-    for (int ks = 0; ks < ksplit; ks += 32) {
-      float v[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) v[k] = (ks + k < ksplit) ? src[(ks + k) * step] : 0.f;
-#pragma unroll
-      for (int k = 0; k < 32; k += 4) s += (v[k] + v[k + 1]) + (v[k + 2] + v[k + 3]);
-    }
-    z[i] = s;
-  }
+  for (int i = threadIdx.x; i < N; i += blockDim.x)
+    z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
   __syncthreads();
   float ss = 0.f;
   for (int i = threadIdx.x; i < d_c; i += blockDim.x) ss = fmaf(z[i], z[i], ss);
@@ -110,6 +112,34 @@ __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit,
     const float a = z[d_c + 2 * i], bb = z[d_c + 2 * i + 1];
     st(rope + row * rope_stride + 2 * i, a * cs - bb * sn);
     st(rope + row * rope_stride + 2 * i + 1, a * sn + bb * cs);
+  }
+}
+
+// =============================================================================================
+// Query chain, middle step: c_q = RMSNorm(sum of the K slices of x·W_DQ) · gamma_q, one row of N
+// values per token, stored in T. One block per token (blockDim a multiple of 32, at most
+// RMS_THREADS: the launch bound keeps the block's registers within the SM's).
+// =============================================================================================
+constexpr int RMS_THREADS = 512;
+
+template <typename T>
+__global__ void __launch_bounds__(RMS_THREADS) rms_rows_kernel(const float* __restrict__ part, int ksplit, int n_tok, int N,
+                                const T* __restrict__ gamma, float eps, T* __restrict__ out) {
+  extern __shared__ float z[];
+  __shared__ float red[32];
+  grid_dependency_wait();   // launched with programmatic dependent launch after the projection
+  allow_dependents();
+  const int tok = blockIdx.x;
+  for (int i = threadIdx.x; i < N; i += blockDim.x)
+    z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
+  __syncthreads();
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) ss = fmaf(z[i], z[i], ss);
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)N + eps);
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    const float gm = gamma ? ld(gamma + i) : 1.f;
+    st(out + (int64_t)tok * N + i, z[i] * inv * gm);
   }
 }
 

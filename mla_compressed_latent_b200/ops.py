@@ -132,6 +132,27 @@ def mla_append_cache(dims: Dims, x, w_dkv_kr, gamma, seqlens, block_table, cache
     _check("mla_append_cache", rc)
 
 
+def mla_project_query(dims: Dims, x, w_dq, gamma_q, w_uq, w_qr, q_nope=None, q_rope_raw=None, workspace=None,
+                      stream=None):
+    """x [B, s_q, C] -> (q_nope [B, s_q, H, D], q_rope_raw [B, s_q, H, d_r]) through
+    c_q = RMSNorm(x·W_DQ)·gamma_q (w_dq [C, d_q], w_uq [d_q, H*D], w_qr [d_q, H*d_r])."""
+    lib = L.load()
+    B, s_q, C = x.shape
+    d_q = w_dq.shape[1]
+    if q_nope is None:
+        q_nope = torch.empty(B, s_q, dims.H, dims.D, dtype=x.dtype, device=x.device)
+    if q_rope_raw is None:
+        q_rope_raw = torch.empty(B, s_q, dims.H, dims.d_r, dtype=x.dtype, device=x.device)
+    d = dims.c()
+    need = lib.mla_query_workspace_size(ctypes.byref(d), B, s_q, C, d_q)
+    workspace, wsb = _workspace(need, x.device, workspace)
+    rc = lib.mla_project_query(ctypes.byref(d), _dt(x), B, s_q, _ptr(x), C, d_q, _ptr(w_dq), _ptr(gamma_q),
+                               _ptr(w_uq), _ptr(w_qr), _ptr(q_nope), _ptr(q_rope_raw),
+                               _ptr(workspace) if workspace is not None else None, wsb, _stream(stream))
+    _check("mla_project_query", rc)
+    return q_nope, q_rope_raw
+
+
 def mla_absorb_q(dims: Dims, q_nope, q_rope_raw, w_uk, seqlens, q_abs=None, stream=None):
     lib = L.load()
     B, s_q, H, D = q_nope.shape

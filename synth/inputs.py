@@ -86,6 +86,10 @@ WORKLOADS = {
         Workload("dsv3_b64_l4096", "bf16", B=64, s_q=1, H=128, D=128, d_r=64, d_c=512, d_v=128,
                  C=7168, lengths=("fixed", 4096),
                  description="DeepSeek-V2/V3-shaped absorbed decode, batch 64 x 4096 positions"),
+        Workload("dsv3_fromx_b64_l4096", "bf16", B=64, s_q=1, H=128, D=128, d_r=64, d_c=512, d_v=128,
+                 C=7168, d_q=1536, lengths=("fixed", 4096),
+                 description="the DeepSeek-shaped step from hidden states: queries through the query chain "
+                             "(d_q = 1536), batch 64 x 4096 positions"),
         Workload("longctx_b8", "bf16", B=8, s_q=1, H=128, D=128, d_r=64, d_c=512, d_v=128,
                  C=7168, lengths=("uniform", 16384, 131072),
                  description="long-context absorbed decode, 8 sequences of 16K-128K positions"),

@@ -278,10 +278,13 @@ def _gpu_step(w, case, dev):
     return out, out_model, lse
 
 
-def test_smallem_layer_fp32_from_hidden_states():
+@pytest.mark.parametrize("queries", ["drawn", "from_x"])
+def test_smallem_layer_fp32_from_hidden_states(queries):
     """The Smallem-scale layer in fp32: every position's row appended from x by the GPU (511 as one
     prefill call, the new token as a decode step), then absorb -> decode -> out_proj, against the
-    expanded definition of the oracle built from the same x."""
+    expanded definition of the oracle built from the same x. With queries "from_x" the new token's
+    query also comes from its x through the query chain (mla_project_query), so the whole step runs
+    from hidden states."""
     w = synth.workload("smallem_fp32")
     L = 512
     case = Case(w)
@@ -293,7 +296,11 @@ def test_smallem_layer_fp32_from_hidden_states():
     prefill_len = torch.tensor([L - 1], dtype=torch.int32, device="cuda")
     ops.mla_append_cache(dims, xt[None, :L - 1], dev["w_dkv_kr"], None, prefill_len, dev["table"], cache)
     ops.mla_append_cache(dims, xt[None, L - 1:], dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache)
-    q_abs = ops.mla_absorb_q(dims, dev["q_nope"], dev["q_rope_raw"], dev["W_UK"], dev["seqlens"])
+    q_nope, q_rope_raw = dev["q_nope"], dev["q_rope_raw"]
+    if queries == "from_x":
+        q_nope, q_rope_raw = ops.mla_project_query(dims, xt[None, L - 1:], dev["W_DQ"], dev["gamma_q"], dev["W_UQ"],
+                                                   dev["W_QR"])
+    q_abs = ops.mla_absorb_q(dims, q_nope, q_rope_raw, dev["W_UK"], dev["seqlens"])
     o_lat, lse = ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"])
     out, out_model = ops.mla_out_proj(dims, o_lat, dev["W_UV"], w_o=dev["W_O"])
     torch.cuda.synchronize()
@@ -303,12 +310,43 @@ def test_smallem_layer_fp32_from_hidden_states():
     _assert_close(got_rows[:, :w.d_c], c, "f32", "latent rows")
     _assert_close(got_rows[:, w.d_c:], kr, "f32", "rope rows")
     pos = np.array([L - 1])
-    q_rot = O.rope(case.q_rope_raw64[0], pos[:, None] * np.ones((1, w.H)))
-    ref, ref_lse = O.expanded_decode(case.q_nope64[0], q_rot, c, kr, case.W64["W_UK"], case.W64["W_UV"], L, w.sm_scale)
+    if queries == "from_x":
+        q_ref, _, q_rot = O.query_parts(x_all[L - 1:].astype(np.float64), case.W64["W_DQ"], case.W64["W_UQ"],
+                                        case.W64["W_QR"], w.H, w.D, w.d_r, pos, case.W64["gamma_q"], w.rms_eps,
+                                        w.rope_base)
+    else:
+        q_ref = case.q_nope64[0]
+        q_rot = O.rope(case.q_rope_raw64[0], pos[:, None] * np.ones((1, w.H)))
+    ref, ref_lse = O.expanded_decode(q_ref, q_rot, c, kr, case.W64["W_UK"], case.W64["W_UV"], L, w.sm_scale)
     _assert_close(out[0].double().cpu().numpy(), ref, "f32", "head outputs")
     _assert_lse(lse[0].cpu().numpy(), ref_lse, "f32", "lse")
     ref_model = ref.reshape(1, -1) @ case.W64["W_O"]
     _assert_close(out_model[0].double().cpu().numpy(), ref_model, "f32", "layer output")
+
+
+@pytest.mark.parametrize("name,over", [
+    ("smallem_fp32", {}),
+    ("smallem_fp32", dict(B=3, s_q=2)),
+    ("dsv3_b64_l4096", dict(d_q=1536, lengths=("fixed", 64))),
+    ("dsv3_b64_l4096", dict(d_q=1536, B=50, s_q=3, lengths=("fixed", 64))),
+])
+def test_project_query(name, over):
+    """f2, the query chain x -> RMSNorm(x·W_DQ)·gamma_q -> (·W_UQ, ·W_QR), against the oracle's
+    query_parts in fp64: the CUDA-core route in fp32, the tensor-core route in bf16 at the DeepSeek
+    widths (C = 7168, d_q = 1536, H·D = 16384), one token per sequence and a ragged 150-token batch."""
+    w = synth.workload(name, **over)
+    case = Case(w)
+    dev = case.to_device()
+    dims = Dims.of(w)
+    q_nope, q_rope_raw = ops.mla_project_query(dims, dev["x"], dev["W_DQ"], dev["gamma_q"], dev["W_UQ"], dev["W_QR"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    n = w.B * w.s_q
+    ref_nope, ref_raw, _ = O.query_parts(case.x64.reshape(n, w.C), case.W64["W_DQ"], case.W64["W_UQ"],
+                                         case.W64["W_QR"], w.H, w.D, w.d_r, np.zeros(n), case.W64["gamma_q"],
+                                         w.rms_eps, w.rope_base)
+    _assert_close(q_nope.double().cpu().numpy().reshape(n, w.H, w.D), ref_nope, w.dtype, "q_nope")
+    _assert_close(q_rope_raw.double().cpu().numpy().reshape(n, w.H, w.d_r), ref_raw, w.dtype, "q_rope_raw")
 
 
 def test_full_step_dsv3_against_oracle():

@@ -91,6 +91,26 @@ def test_append_rejects_missing_workspace(lib):
     assert rc == L.MLA_ERR_WORKSPACE
 
 
+def test_project_query_validates_before_any_launch(lib):
+    d = _dims()
+    good = ctypes.c_void_p(4096)
+    odd = ctypes.c_void_p(4100)
+    need = lib.mla_query_workspace_size(ctypes.byref(d), 64, 1, 7168, 1536)
+    # at least the fp32 partial sums of one K slice and the fp32-sized c_q rows
+    assert need >= 2 * 64 * 1536 * 4
+    assert lib.mla_query_workspace_size(ctypes.byref(d), 64, 1, 7168, 0) == 0
+    args = [good, 7168, 1536, good, None, good, good, good, good]
+    rc = lib.mla_project_query(ctypes.byref(d), 1, 64, 1, *args, None, 0, None)
+    assert rc == L.MLA_ERR_WORKSPACE
+    for i in (0, 3, 5, 6, 7, 8):   # x, w_dq, w_uq, w_qr, q_nope, q_rope_raw
+        for bad in (None, odd):
+            a = list(args)
+            a[i] = bad
+            assert lib.mla_project_query(ctypes.byref(d), 1, 64, 1, *a, good, need, None) == L.MLA_ERR_INVALID_ARG
+    assert lib.mla_project_query(ctypes.byref(d), 1, 0, 1, *args, good, need, None) == L.MLA_ERR_INVALID_ARG
+    assert lib.mla_project_query(ctypes.byref(d), 5, 64, 1, *args, good, need, None) == L.MLA_ERR_INVALID_ARG
+
+
 def test_gqla_rejects_bad_groups(lib):
     d = _dims(g=3)
     good = ctypes.c_void_p(4096)
