@@ -49,6 +49,12 @@ struct Params {
   int d_r, H, s_q;
   const int32_t* seqlens;
   float rope_base;
+  // Optional second problem in the same launch (mode 0, no rotated tail): the CTAs past the first
+  // problem's H * m_tiles take the m-tiles of a second weight [K, M2] on the same tokens and write
+  // y2[tok * y2_tok_stride + m]. M2 = 0: none.
+  int M2;
+  __nv_bfloat16* y2;
+  int64_t y2_tok_stride;
 };
 
 __host__ __device__ constexpr int stage_bytes(int tn) { return kABytes + tn * 128; }
@@ -76,16 +82,23 @@ __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-// grid: x = head * m_tiles + m_tile, y = token block, z = K split
-__global__ void __launch_bounds__(kThreads, 1)
-head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const Params p) {
+// grid: x = head * m_tiles + m_tile (then, with kTwo, the second problem's m-tiles), y = token block,
+// z = K split. The tensor maps stay kernel parameters (TMA reads them from parameter space); the
+// body is instantiated once with a single weight map, and once with a second one.
+template <bool kTwo>
+__device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
+                                               const CUtensorMap& tm_w2, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) GEMM_TIME(0);
   const int m_tiles = (p.M + kBM - 1) / kBM;
-  const int h = blockIdx.x / m_tiles, mt = blockIdx.x % m_tiles;
+  const bool second = kTwo && (int)blockIdx.x >= p.H * m_tiles;   // a CTA of the second problem
+  const int h = second ? 0 : blockIdx.x / m_tiles;
+  const int mt = second ? blockIdx.x - p.H * m_tiles : blockIdx.x % m_tiles;
+  const int M = second ? p.M2 : p.M;
+  const CUtensorMap* tw = second ? &tm_w2 : &tm_w;
   const int tok0 = blockIdx.y * p.tn;
   const int split = blockIdx.z;
   const int kc0 = split * p.chunks_per_split;
@@ -101,7 +114,7 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     for (int s = 0; s < S; ++s) { ptx::mbar_init(full0 + 8u * s, 1); ptx::mbar_init(empty0 + 8u * s, 1); }
     ptx::mbar_init(done, 1);
     ptx::fence_mbar_init();
-    ptx::prefetch_tmap(&tm_w);
+    ptx::prefetch_tmap(tw);
     ptx::prefetch_tmap(&tm_x);
   }
   if (warp == 2) { ptx::tmem_alloc(slot, tmem_cols); ptx::tmem_relinquish(); }
@@ -121,8 +134,8 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
       const uint32_t st = ring + s * sbytes;
       const int k = h * p.K + (kc0 + i) * kBK;
       ptx::mbar_arrive_expect_tx(full0 + 8u * s, sbytes);
-      ptx::tma_load_2d(st, &tm_w, mt * kBM, k, full0 + 8u * s);
-      ptx::tma_load_2d(st + kABytes / 2, &tm_w, mt * kBM + 64, k, full0 + 8u * s);
+      ptx::tma_load_2d(st, tw, mt * kBM, k, full0 + 8u * s);
+      ptx::tma_load_2d(st + kABytes / 2, tw, mt * kBM + 64, k, full0 + 8u * s);
       ptx::tma_load_2d(st + kABytes, &tm_x, k, tok0, full0 + 8u * s);
     }
   } else if (warp == 1 && lane == 0) {
@@ -148,7 +161,7 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     const int row = threadIdx.x - 128;
     const int m = mt * kBM + row;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    if (p.rope_in != nullptr) {
+    if (p.rope_in != nullptr && !second) {
       // the rotated tail does not depend on the GEMM: done while the main loop runs, the token
       // block's tokens dealt out over the head's m-tiles (token j of the block goes to m-tile j % m_tiles);
       // the pairs' inverse frequencies are computed once, into shared memory
@@ -192,14 +205,16 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
         uint32_t r[32];
         ptx::tmem_ld32(tmem + lane_off + (uint32_t)c, r);
         ptx::tmem_wait_ld();
-        if (m >= p.M) continue;
+        if (m >= M) continue;
         const int kn = min(32, p.n_tok - tok0 - c);
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
           if (k >= kn) break;
           const int tok = tok0 + c + k;
           const float v = nk > 0 ? __uint_as_float(r[k]) : 0.f;
-          if (p.mode == 0)
+          if (second)
+            p.y2[(int64_t)tok * p.y2_tok_stride + m] = __float2bfloat16_rn(v);
+          else if (p.mode == 0)
             p.y[(int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + m] = __float2bfloat16_rn(v);
           else
             p.part[((int64_t)split * p.n_tok + tok) * p.M + m] = v;
@@ -217,6 +232,17 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
   if (threadIdx.x == 0) GEMM_TIME(5);
 }
 
+__global__ void __launch_bounds__(kThreads, 1)
+head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const Params p) {
+  head_gemm_body<false>(tm_w, tm_x, tm_w, p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+head_gemm2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                  const __grid_constant__ CUtensorMap tm_w2, const Params p) {
+  head_gemm_body<true>(tm_w, tm_x, tm_w2, p);
+}
+
 // ---- host ----------------------------------------------------------------------------------------
 // Shapes the kernel takes: K a multiple of 64 (whole chunks), M a multiple of 8 (16-byte weight rows).
 inline bool supported(int K, int M) { return K > 0 && K % kBK == 0 && M > 0 && M % 8 == 0; }
@@ -225,11 +251,12 @@ inline bool supported_rope(int d_r) { return d_r > 0 && d_r <= 128; }
 
 inline int tokens_per_cta(int n_tok) { return n_tok <= 32 ? 32 : (n_tok <= 64 ? 64 : 128); }
 
-// Split of K for mode 1: about one CTA per SM, every split non-empty. Returns the number of splits.
+// Split of K for mode 1: at most one CTA per SM (a CTA streaming a long K fills an SM's shared
+// memory, so one more would start a second wave), every split non-empty. Returns the number of splits.
 inline int plan_splits(int M, int K, int n_tok, int num_sms, int max_splits) {
   const int chunks = K / kBK;
   const int base = ((M + kBM - 1) / kBM) * ((n_tok + tokens_per_cta(n_tok) - 1) / tokens_per_cta(n_tok));
-  int ks = std::max(1, std::min({(num_sms + base - 1) / base, chunks, max_splits}));
+  int ks = std::max(1, std::min({num_sms / base, chunks, max_splits}));
   const int per = (chunks + ks - 1) / ks;
   return (chunks + per - 1) / per;
 }
@@ -239,12 +266,19 @@ struct Problem {
   const void* x;             // [n_tok, H * K] row-major bf16
   int H, K, M, n_tok;
   int splits;                // 1 for mode 0
+  const void* w2 = nullptr;  // optional second weight [K, M2] (H = 1, mode 0; output p.y2)
+  int M2 = 0;
+  int num_sms = 0;           // SMs of the device (0: unknown)
 };
 
 // Launches on `st`; returns MLA_OK, or an error status with nothing launched.
 inline int run(const Problem& pr, Params p, cudaStream_t st) {
   if (!supported(pr.K, pr.M) || pr.n_tok <= 0 || pr.H <= 0 || pr.splits <= 0) return MLA_ERR_UNSUPPORTED;
+  const bool two = pr.w2 != nullptr;
+  if (two && (pr.H != 1 || pr.splits != 1 || p.mode != 0 || p.rope_in != nullptr || !p.y2 || !supported(pr.K, pr.M2)))
+    return MLA_ERR_UNSUPPORTED;
   p.M = pr.M;
+  p.M2 = two ? pr.M2 : 0;
   p.K = pr.K;
   p.n_tok = pr.n_tok;
   p.H = pr.H;
@@ -253,20 +287,31 @@ inline int run(const Problem& pr, Params p, cudaStream_t st) {
   p.chunks_per_split = (chunks + pr.splits - 1) / pr.splits;
   constexpr int kSmemMax = 232448;   // 227 KB per CTA
   p.stages = std::min({kMaxStages, p.chunks_per_split, (kSmemMax - 2048) / stage_bytes(p.tn)});
-  CUtensorMap tm_w, tm_x;
+  const int m_ctas = pr.H * ((pr.M + kBM - 1) / kBM) + (two ? (pr.M2 + kBM - 1) / kBM : 0);
+  const int ctas = m_ctas * ((pr.n_tok + p.tn - 1) / p.tn) * pr.splits;
+  // more CTAs than SMs: a ring that lets two CTAs share an SM keeps the whole grid in one wave
+  if (pr.num_sms > 0 && ctas > pr.num_sms)
+    p.stages = std::max(1, std::min(p.stages, (kSmemMax / 2 - 2048) / stage_bytes(p.tn)));
+  CUtensorMap tm_w, tm_x, tm_w2;
   if (!tmap::make_bf16_sw128(&tm_w, pr.w, pr.M, (int64_t)pr.H * pr.K, pr.M, kBK)) return MLA_ERR_INVALID_ARG;
+  if (two && !tmap::make_bf16_sw128(&tm_w2, pr.w2, pr.M2, pr.K, pr.M2, kBK)) return MLA_ERR_INVALID_ARG;
   if (!tmap::make_bf16_sw128(&tm_x, pr.x, (int64_t)pr.H * pr.K, pr.n_tok, (int64_t)pr.H * pr.K, p.tn))
     return MLA_ERR_INVALID_ARG;
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-    if (cudaFuncSetAttribute(head_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess)
+    if (cudaFuncSetAttribute(head_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess ||
+        cudaFuncSetAttribute(head_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess)
       return MLA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_done[dev] = true;
   }
-  const dim3 grid(pr.H * ((pr.M + kBM - 1) / kBM), (pr.n_tok + p.tn - 1) / p.tn, pr.splits);
-  mla::launch_pdl(head_gemm_kernel, grid, dim3(kThreads), (size_t)smem_bytes(p.tn, p.stages), st, tm_w, tm_x, p);
+  const dim3 grid(m_ctas, (pr.n_tok + p.tn - 1) / p.tn, pr.splits);
+  const size_t smem = (size_t)smem_bytes(p.tn, p.stages);
+  if (two)
+    mla::launch_pdl(head_gemm2_kernel, grid, dim3(kThreads), smem, st, tm_w, tm_x, tm_w2, p);
+  else
+    mla::launch_pdl(head_gemm_kernel, grid, dim3(kThreads), smem, st, tm_w, tm_x, p);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

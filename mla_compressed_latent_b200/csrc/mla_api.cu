@@ -76,6 +76,12 @@ int append_ksplit(int n_tok, int K, int N) {
   return ks;
 }
 
+// A tensor-core projection problem with the device's SM count filled in (it sizes the ring).
+mla::gemm::Problem with_sms(mla::gemm::Problem pr) {
+  pr.num_sms = num_sms();
+  return pr;
+}
+
 // The tensor-core projection takes bf16 with whole 64-wide K chunks and 16-byte weight rows.
 bool append_on_tc(int32_t dtype, int C, int N) { return dtype == MLA_BF16 && mla::gemm::supported(C, N); }
 int append_tc_splits(int n_tok, int C, int N) { return mla::gemm::plan_splits(N, C, n_tok, num_sms(), 64); }
@@ -194,7 +200,7 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     mla::gemm::Params p{};
     p.mode = 1;
     p.part = reinterpret_cast<float*>(workspace);
-    if ((rc = mla::gemm::run({w_dkv_kr, x, 1, C, N, n_tok, ks}, p, st))) return rc;
+    if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, ks}), p, st))) return rc;
     const size_t fin_smem = (size_t)N * sizeof(float);
     if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
     const int fin_threads = std::min(1024, (N + 31) / 32 * 32);   // one thread per output column
@@ -278,21 +284,22 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
     mla::gemm::Params p{};
     p.mode = 1;
     p.part = part;
-    if ((rc = mla::gemm::run({w_dq, x, 1, C, d_q, n_tok, ks}, p, st))) return rc;
+    if ((rc = mla::gemm::run(with_sms({w_dq, x, 1, C, d_q, n_tok, ks}), p, st))) return rc;
     if ((rc = set_smem(mla::simt::rms_rows_kernel<T>, fin_smem))) return rc;
     mla::launch_pdl(mla::simt::rms_rows_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)part, ks,
                     n_tok, d_q, (const T*)gamma_q, dims->rms_eps, (T*)c_q);
-    // the two up-projections as single-"head" GEMMs over the whole output width
+    // both up-projections in one launch, each a single-"head" GEMM over its whole output width
     mla::gemm::Params pu{};
     pu.mode = 0;
     pu.y = reinterpret_cast<T*>(q_nope);
     pu.y_tok_stride = (int64_t)H * D;
-    if ((rc = mla::gemm::run({w_uq, c_q, 1, d_q, H * D, n_tok, 1}, pu, st))) return rc;
-    mla::gemm::Params pr{};
-    pr.mode = 0;
-    pr.y = reinterpret_cast<T*>(q_rope_raw);
-    pr.y_tok_stride = (int64_t)H * d_r;
-    if ((rc = mla::gemm::run({w_qr, c_q, 1, d_q, H * d_r, n_tok, 1}, pr, st))) return rc;
+    pu.y2 = reinterpret_cast<T*>(q_rope_raw);
+    pu.y2_tok_stride = (int64_t)H * d_r;
+    mla::gemm::Problem up{w_uq, c_q, 1, d_q, H * D, n_tok, 1};
+    up.w2 = w_qr;
+    up.M2 = H * d_r;
+    up.num_sms = num_sms();
+    if ((rc = mla::gemm::run(up, pu, st))) return rc;
     return launch_status();
   }
   const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
@@ -341,7 +348,7 @@ int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
     p.s_q = s_q;
     p.seqlens = seqlens;
     p.rope_base = dims->rope_base;
-    return mla::gemm::run({w_uk, q_nope, H, D, d_c, n_tok, 1}, p, st);
+    return mla::gemm::run(with_sms({w_uk, q_nope, H, D, d_c, n_tok, 1}), p, st);
   }
   dim3 grid(H, (n_tok + mla::simt::HG_TOK - 1) / mla::simt::HG_TOK);
   const size_t smem = (size_t)mla::simt::HG_TOK * D * sizeof(float);
@@ -439,7 +446,7 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
     p.y = reinterpret_cast<__nv_bfloat16*>(out);
     p.y_tok_stride = (int64_t)H * d_v;
     p.y_head_stride = d_v;
-    if ((rc = mla::gemm::run({w_uv, o_lat, H, d_c, d_v, n_tok, 1}, p, st))) return rc;
+    if ((rc = mla::gemm::run(with_sms({w_uv, o_lat, H, d_c, d_v, n_tok, 1}), p, st))) return rc;
     if (w_o) {
       using T = __nv_bfloat16;
       launch(mla::simt::proj_partial_kernel<T>, ogrid, mla::simt::PROJ_COLS, 0, st, (const T*)out, n_tok, K,
