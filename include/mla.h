@@ -39,7 +39,7 @@ extern "C" {
 enum mla_status {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer or stride */
-  MLA_ERR_UNSUPPORTED = 2,   /* valid arguments this build has no kernel for (dtype, shape) */
+  MLA_ERR_UNSUPPORTED = 2,   /* valid arguments the library has no kernel for (dtype, shape) */
   MLA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the matching *_workspace_size */
   MLA_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch error, bad device) */
   MLA_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel gave up */

@@ -10,7 +10,7 @@ import synth
 
 TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 
-# the benchmark spec tolerances
+# parity bars: max|Δ| / max|ref| of the outputs, and |Δ lse| (fp32: relative to max(1, max|lse|))
 TOL = {"f32": dict(out=1e-5, lse=1e-5), "bf16": dict(out=2e-2, lse=1e-3)}
 
 

@@ -108,8 +108,8 @@ def test_decode_workspace_reused_across_calls():
         assert ops.mla_check_status() == 0
         ref_o, ref_l = _oracle_absorbed(case, case.q_abs64)
         for b in range(w.B):
-            _assert_close(o_lat[b].float().cpu().numpy(), ref_o[b], "bf16", f"round {i} o_lat seq {b}")
-            _assert_lse(lse[b].cpu().numpy(), ref_l[b], "bf16", f"round {i} lse seq {b}")
+            _assert_close(o_lat[b].float().cpu().numpy(), ref_o[b], "bf16", f"call {i} o_lat seq {b}")
+            _assert_lse(lse[b].cpu().numpy(), ref_l[b], "bf16", f"call {i} lse seq {b}")
 
 
 def test_decode_absorbed_fp32_smallem_shapes():
