@@ -330,6 +330,66 @@ def test_whole_layer_from_hidden_states_matches_sdpa():
     np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-13)
 
 
+def _identity_query_chain(x, gamma_q=None, eps=0.0, positions=None):
+    """query_parts with W_DQ, W_UQ and W_QR all identities (C = d_q = H·D = H·d_r): its outputs are
+    then x itself, normalised per token and split into heads, which the checks below can see
+    without restating the formula."""
+    H, D = 3, 4
+    n, C = x.shape
+    assert C == H * D
+    eye = np.eye(C)
+    pos = np.zeros(n) if positions is None else positions
+    return O.query_parts(x, eye, eye, eye, H, D, D, pos, gamma_q, eps)
+
+
+def test_query_parts_split_heads_in_order_and_normalise_each_token():
+    """Query chain (« L'obstacle : RoPE », « Le code »): with identity projections, every head's
+    part is a positive multiple of its own slice of x (head h = columns h·D .. h·D + D - 1, no
+    mixing), the factor is shared by all heads of a token, and each token's query has mean square
+    exactly 1 (RMSNorm with eps = 0, over that token's d_q values)."""
+    x = _rng(40).standard_normal((5, 12)) * np.array([[0.1], [1.0], [3.0], [7.0], [0.5]])
+    q_nope, q_raw, q_rot = _identity_query_chain(x)
+    for part in (q_nope, q_raw):
+        flat = part.reshape(5, 12)
+        ratio = flat / x
+        np.testing.assert_allclose(ratio, ratio[:, :1] * np.ones((1, 12)), rtol=1e-13)
+        assert (ratio > 0).all()
+        np.testing.assert_allclose((flat ** 2).mean(axis=1), 1.0, rtol=1e-13)
+    np.testing.assert_allclose(q_rot, q_raw, rtol=0, atol=1e-15)   # RoPE at position 0 is the identity
+
+
+def test_query_parts_scale_invariance_gain_and_rotation():
+    """RMSNorm removes a token's scale; the gain γ_q multiplies c_q and so every output; the RoPE
+    part is a rotation of q_rope_raw (pair norms kept) at the token's position."""
+    x = _rng(41).standard_normal((3, 12))
+    a = _identity_query_chain(x)
+    b = _identity_query_chain(x * np.array([[5.0], [0.25], [40.0]]))
+    for u, v in zip(a, b):
+        np.testing.assert_allclose(u, v, rtol=1e-12, atol=1e-14)
+    g = _identity_query_chain(x, gamma_q=np.full(12, 2.0))
+    np.testing.assert_allclose(g[0], 2 * a[0], rtol=1e-13)
+    np.testing.assert_allclose(g[1], 2 * a[1], rtol=1e-13)
+    _, q_raw, q_rot = _identity_query_chain(x, positions=np.array([3, 17, 100]))
+    pair = lambda v: np.hypot(v[..., 0::2], v[..., 1::2])
+    np.testing.assert_allclose(pair(q_rot), pair(q_raw), rtol=1e-13)
+    assert np.abs(q_rot - q_raw).max() > 1e-3
+
+
+def test_query_parts_with_random_weights_match_torch_rms_norm():
+    """Random projections: c_q through torch's own rms_norm (its normalised_shape fixes the axis),
+    then the two up-projections; the oracle's heads are column blocks of those products."""
+    r = _rng(42)
+    n, C, d_q, H, D, d_r = 4, 20, 12, 3, 5, 2
+    x = r.standard_normal((n, C))
+    W_DQ, W_UQ, W_QR = r.standard_normal((C, d_q)), r.standard_normal((d_q, H * D)), r.standard_normal((d_q, H * d_r))
+    gamma = r.uniform(0.5, 1.5, d_q)
+    q_nope, q_raw, _ = O.query_parts(x, W_DQ, W_UQ, W_QR, H, D, d_r, np.zeros(n), gamma, 1e-6)
+    c_q = torch.nn.functional.rms_norm(torch.from_numpy(x @ W_DQ), (d_q,), torch.from_numpy(gamma), eps=1e-6).numpy()
+    for h in range(H):
+        np.testing.assert_allclose(q_nope[:, h], c_q @ W_UQ[:, h * D:(h + 1) * D], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(q_raw[:, h], c_q @ W_QR[:, h * d_r:(h + 1) * d_r], rtol=1e-12, atol=1e-13)
+
+
 # ------------------------------------------------------------------------------------------
 # planted mistakes: plausible slips in the oracle must fail the pins above
 # ------------------------------------------------------------------------------------------
@@ -411,6 +471,39 @@ def test_planted_merge_without_max_shift_weighting_is_caught(monkeypatch):
         test_merge_of_disjoint_parts_equals_whole()
 
 
+def test_planted_transposed_head_split_is_caught(monkeypatch):
+    def bad(x, W_DQ, W_UQ, W_QR, H, D, d_r, positions, gamma_q=None, eps=1e-6, base=10000.0):
+        q_nope, q_raw, q_rot = _QUERY(x, W_DQ, W_UQ, W_QR, H, D, d_r, positions, gamma_q, eps, base)
+        n = q_nope.shape[0]
+        # heads taken as the inner index of the H·D columns instead of the outer one
+        q_nope = q_nope.reshape(n, H * D).reshape(n, D, H).transpose(0, 2, 1)
+        return q_nope, q_raw, q_rot
+    _planted(monkeypatch, "query_parts", bad)
+    with pytest.raises(AssertionError):
+        test_query_parts_split_heads_in_order_and_normalise_each_token()
+
+
+def test_planted_dropped_query_normalisation_is_caught(monkeypatch):
+    def bad(x, W_DQ, W_UQ, W_QR, H, D, d_r, positions, gamma_q=None, eps=1e-6, base=10000.0):
+        # the query latent c_q left unnormalised
+        return _unnormalised_query(x, W_DQ, W_UQ, W_QR, H, D, d_r, positions, gamma_q, base)
+    _planted(monkeypatch, "query_parts", bad)
+    with pytest.raises(AssertionError):
+        test_query_parts_scale_invariance_gain_and_rotation()
+
+
+def _unnormalised_query(x, W_DQ, W_UQ, W_QR, H, D, d_r, positions, gamma_q, base):
+    """The query chain with its RMSNorm left out (a planted slip)."""
+    c_q = np.asarray(x, float) @ np.asarray(W_DQ, float)
+    if gamma_q is not None:
+        c_q = c_q * gamma_q
+    n = c_q.shape[0]
+    q_nope = (c_q @ W_UQ).reshape(n, H, D)
+    q_raw = (c_q @ W_QR).reshape(n, H, d_r)
+    return q_nope, q_raw, O.rope(q_raw, np.asarray(positions, float)[:, None] * np.ones((1, H)), base)
+
+
+_QUERY = O.query_parts
 _ABSORBED = O.absorbed_decode
 _ABSORB = O.absorb_query
 _EXPANDED = O.expanded_decode
