@@ -48,6 +48,18 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
+def max_over_ranks(x, world, device=None):
+    """The largest x over all ranks, returned on every rank (a time is the slowest rank's; a flag
+    raised on any rank is raised on all). Every rank must call it at the same point."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -326,11 +338,7 @@ def run_grouped(args, w, dims, device, world, rank, local):
         t1.record(stream)
         torch.cuda.synchronize()
     launches = ops.mla_launch_count() - n0
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, device)
     total = int(lens.sum())
     n_tok = w.B * w.s_q
     # per cached position: K and V of every group plus the shared RoPE key; per token: the query
@@ -471,17 +479,15 @@ def main():
             t1.record(stream)
             torch.cuda.synchronize()
         launches = ops.mla_launch_count() - n0
-        ms = t0.elapsed_time(t1)
+        ms = max_over_ranks(t0.elapsed_time(t1), world, device)
         if world > 1:
-            t = torch.tensor([ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
             dist.barrier()
         return ms, launches, clk
 
     ms, launches, clk = timed_region()
     remeasured = False
-    if clk.rejected():
+    # measured again on every rank if any rank's clocks were rejected (the ranks' collectives stay in step)
+    if max_over_ranks(1.0 if clk.rejected() else 0.0, world, device) > 0:
         ms, launches, clk = timed_region()
         remeasured = True
     dec_ms = statistics.mean(between(m, "absorb_q", "decode") for m in dec_ev)
@@ -513,11 +519,7 @@ def main():
         out_host.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     h2d = sum(t.numel() * t.element_size()
               for t in ((dev["x_host"],) if from_x else (dev["x_host"], dev["q_nope_host"], dev["q_rope_host"])))
     d2h = out_host.numel() * out_host.element_size()
