@@ -128,8 +128,9 @@ int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, int32_t B, i
  *   (all dtype, row-major, 16-byte aligned)
  * workspace: at least mla_query_workspace_size(...) bytes of device memory (fp32 partial sums of
  * x·W_DQ, then c_q); its contents need not be initialised. Errors: MLA_ERR_INVALID_ARG for null or
- * misaligned pointers and non-positive sizes, MLA_ERR_WORKSPACE, MLA_ERR_CUDA; nothing is launched
- * on an error return.
+ * misaligned pointers and non-positive sizes, MLA_ERR_WORKSPACE: returned before anything is
+ * enqueued. MLA_ERR_CUDA (a failed launch) may come after earlier kernels of the chain were
+ * enqueued; the outputs are then undefined.
  * ------------------------------------------------------------------------------------------- */
 size_t mla_query_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C, int32_t d_q);
 int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,

@@ -279,13 +279,16 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
   void* c_q = reinterpret_cast<char*>(workspace) + pb;
   const size_t fin_smem = (size_t)d_q * sizeof(float);
   const int fin_threads = std::min(mla::simt::RMS_THREADS, (d_q + 31) / 32 * 32);
+  // attributes first: a failure here leaves nothing enqueued
+  if ((rc = dtype == MLA_F32 ? set_smem(mla::simt::rms_rows_kernel<float>, fin_smem)
+                             : set_smem(mla::simt::rms_rows_kernel<__nv_bfloat16>, fin_smem)))
+    return rc;
   if (tc) {
     using T = __nv_bfloat16;
     mla::gemm::Params p{};
     p.mode = 1;
     p.part = part;
     if ((rc = mla::gemm::run(with_sms({w_dq, x, 1, C, d_q, n_tok, ks}), p, st))) return rc;
-    if ((rc = set_smem(mla::simt::rms_rows_kernel<T>, fin_smem))) return rc;
     mla::launch_pdl(mla::simt::rms_rows_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)part, ks,
                     n_tok, d_q, (const T*)gamma_q, dims->rms_eps, (T*)c_q);
     // both up-projections in one launch, each a single-"head" GEMM over its whole output width
@@ -309,8 +312,6 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
     using T = decltype(zero);
     launch(mla::simt::proj_partial_kernel<T>, dim3(cols(d_q), tok_blocks, ks), mla::simt::PROJ_COLS, 0, st,
            (const T*)x, n_tok, C, (const T*)w_dq, d_q, k_chunk, part, (T*)nullptr);
-    int r = set_smem(mla::simt::rms_rows_kernel<T>, fin_smem);
-    if (r) return r;
     launch(mla::simt::rms_rows_kernel<T>, n_tok, fin_threads, fin_smem, st, (const float*)part, ks, n_tok, d_q,
            (const T*)gamma_q, dims->rms_eps, (T*)c_q);
     // one K slice: the kernel writes the finished dot products straight to its output
