@@ -22,9 +22,13 @@
  *  - Paged cache: position p of sequence b lives in page block_table[b*max_pages + p/page_size],
  *    slot p % page_size; page_size is 64. Row r = page*64 + slot of a pool starts at
  *    base + r*stride elements.
- *  - Return value: MLA_OK, or an error code with nothing launched. Errors found on the device
- *    (a page id outside the pool, a wait that timed out) are recorded in a per-device status
- *    word that mla_check_status() reads; the offending access is skipped, never performed.
+ *  - Return value: MLA_OK or an error code. Argument errors (MLA_ERR_INVALID_ARG,
+ *    MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE) are found on the host before anything is enqueued.
+ *    MLA_ERR_CUDA reports a failed CUDA call (a launch, a kernel attribute); in a call that
+ *    enqueues several kernels it may follow the earlier ones, and the call's outputs are then
+ *    undefined. Errors found on the device (a page id outside the pool, a wait that timed out)
+ *    are recorded in a per-device status word that mla_check_status() reads; the offending
+ *    access is skipped, never performed.
  */
 #ifndef MLA_H_
 #define MLA_H_
@@ -128,9 +132,8 @@ int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, int32_t B, i
  *   (all dtype, row-major, 16-byte aligned)
  * workspace: at least mla_query_workspace_size(...) bytes of device memory (fp32 partial sums of
  * x·W_DQ, then c_q); its contents need not be initialised. Errors: MLA_ERR_INVALID_ARG for null or
- * misaligned pointers and non-positive sizes, MLA_ERR_WORKSPACE: returned before anything is
- * enqueued. MLA_ERR_CUDA (a failed launch) may come after earlier kernels of the chain were
- * enqueued; the outputs are then undefined.
+ * misaligned pointers and non-positive sizes, MLA_ERR_WORKSPACE, MLA_ERR_CUDA (see the conventions
+ * above: the chain enqueues three or four kernels).
  * ------------------------------------------------------------------------------------------- */
 size_t mla_query_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C, int32_t d_q);
 int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
