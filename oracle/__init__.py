@@ -5,4 +5,4 @@ reference arm of the bench may import, call or run anything in this package. The
 (the C-ABI library and its Python binding) never touches it, and this package imports nothing
 from the product path: the two share no code, only the seeded inputs of ``synth``.
 """
-from . import mla_oracle, cache_sizes, roofline  # noqa: F401
+from . import mla_oracle, cache_sizes, roofline, fp8_cache  # noqa: F401
