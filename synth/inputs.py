@@ -30,7 +30,7 @@ import numpy as np
 __all__ = [
     "Workload", "WORKLOADS", "workload", "seq_lengths", "block_table", "weights",
     "decode_step_inputs", "cache_row_chunks", "context_hidden_states", "gqla_cache_chunks",
-    "SEED_WEIGHTS", "SEED_DECODE", "SEED_CACHE", "SEED_LENGTHS", "SEED_PAGES",
+    "SEED_WEIGHTS", "SEED_DECODE", "SEED_CACHE", "SEED_LENGTHS", "SEED_PAGES", "CACHE_CHUNK_ROWS",
 ]
 
 SEED_WEIGHTS = 0
