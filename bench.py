@@ -178,40 +178,72 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_sample(w, seconds, max_seqs=None):
-    """Run the fp64 oracle's decode step (absorb, absorbed decode, W_UV projection) sequence by
-    sequence until `seconds` pass; return (positions, tokens, elapsed, sequences)."""
+_ORACLE_SETUP = {}
+_ORACLE_ROWS = {}
+
+
+def _oracle_setup(w):
+    """The oracle's weights (fp64) and this step's inputs, drawn once per workload."""
+    if w not in _ORACLE_SETUP:
+        import numpy as np
+        import synth
+        W = synth.weights(w)
+        _ORACLE_SETUP[w] = (W["W_UK"].astype(np.float64), W["W_UV"].astype(np.float64),
+                            synth.decode_step_inputs(w))
+    return _ORACLE_SETUP[w]
+
+
+def _oracle_rows(w, n):
+    """(b, c, k_r) in fp64 for the first n sequences, in order; the rows of a one- or two-sequence
+    sample are kept for the next call (the reference arm times the same sequence every step)."""
     import numpy as np
     import synth
-    from oracle import mla_oracle as O
-    lens = synth.seq_lengths(w)
-    W = synth.weights(w)
-    step = synth.decode_step_inputs(w)
-    W_UK = W["W_UK"].astype(np.float64)
-    W_UV = W["W_UV"].astype(np.float64)
-    chunks = synth.cache_row_chunks(w, int(lens[: (max_seqs or w.B)].sum()))
-    buf = []
-    pos_done = tok_done = seqs = 0
-    off = 0
-    t0 = time.perf_counter()
-    for b in range(w.B if max_seqs is None else min(w.B, max_seqs)):
-        L = int(lens[b])
-        while sum(len(c) for c, _ in buf) < off + L:
+    if (w, n) in _ORACLE_ROWS:
+        yield from _ORACLE_ROWS[(w, n)]
+        return
+    lens = synth.seq_lengths(w)[:n]
+    chunks = synth.cache_row_chunks(w, int(lens.sum()))
+    pend_c = np.zeros((0, w.d_c), np.float32)
+    pend_k = np.zeros((0, w.d_r), np.float32)
+    keep = [] if n <= 2 else None
+    for b, L in enumerate(lens):
+        L = int(L)
+        while len(pend_c) < L:
             _, c, kr = next(chunks)
-            buf.append((c, kr))
-        c = np.concatenate([x for x, _ in buf])[off:off + L].astype(np.float64)
-        kr = np.concatenate([y for _, y in buf])[off:off + L].astype(np.float64)
-        off += L
+            pend_c = np.concatenate([pend_c, c])
+            pend_k = np.concatenate([pend_k, kr])
+        item = (b, pend_c[:L].astype(np.float64), pend_k[:L].astype(np.float64))
+        pend_c, pend_k = pend_c[L:], pend_k[L:]
+        if keep is not None:
+            keep.append(item)
+            if len(keep) == n:
+                _ORACLE_ROWS[(w, n)] = keep
+        yield item
+
+
+def oracle_sample(w, seconds, max_seqs=None):
+    """Run the fp64 oracle's decode step (absorb, absorbed decode, W_UV projection) sequence by
+    sequence until `seconds` of oracle time pass; drawing the inputs is not timed. Returns
+    (positions, tokens, oracle seconds, sequences)."""
+    from oracle import mla_oracle as O
+    W_UK, W_UV, step = _oracle_setup(w)
+    n = w.B if max_seqs is None else min(w.B, max_seqs)
+    pos_done = tok_done = seqs = 0
+    el = 0.0
+    for b, c, kr in _oracle_rows(w, n):
+        L = len(c)
+        t0 = time.perf_counter()
         pos = O.token_positions(L, w.s_q)
         q_abs = O.absorb_query(step["q_nope"][b], step["q_rope_raw"][b], W_UK, pos, w.rope_base)
         o_lat, _ = O.absorbed_decode(q_abs, c, kr, L, w.sm_scale)
         O.out_projection(o_lat, W_UV)
+        el += time.perf_counter() - t0
         pos_done += L
         tok_done += w.s_q
         seqs += 1
-        if time.perf_counter() - t0 >= seconds:
+        if el >= seconds:
             break
-    return pos_done, tok_done, time.perf_counter() - t0, seqs
+    return pos_done, tok_done, el, seqs
 
 
 def run_reference(args, rank, world):
