@@ -193,7 +193,8 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
   const bool tc = append_on_tc(dtype, C, N);
   const int ks = tc ? append_tc_splits(n_tok, C, N) : append_ksplit(n_tok, C, N);
   const size_t need = (size_t)ks * n_tok * N * sizeof(float);
-  if (!workspace || ws_bytes < need || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < need) return MLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (tc) {
     using T = __nv_bfloat16;
@@ -273,7 +274,8 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
   const int ks = tc ? append_tc_splits(n_tok, C, d_q) : append_ksplit(n_tok, C, d_q);
   const size_t pb = query_part_bytes(ks, n_tok, d_q);
   const size_t need = pb + (size_t)n_tok * d_q * esize(dtype);
-  if (!workspace || ws_bytes < need || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < need) return MLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* part = reinterpret_cast<float*>(workspace);
   void* c_q = reinterpret_cast<char*>(workspace) + pb;
