@@ -189,6 +189,8 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
  *   out[b,t,h,:] = sum_j softmax(s)_j * V[j, g(h), :]          lse[b,t,h] = log sum_j exp(s_j)
  *   q_nope [B, s_q, H, D]  q_rope_raw [B, s_q, H, d_r]  out [B, s_q, H, d_v] (dtype)  lse fp32
  * workspace: at least mla_gqla_workspace_size(...) bytes.
+ * Requires every seqlens[b] >= s_q, as a3 does. The bf16 tensor-core kernel does not check it on
+ * the device: a shorter sequence leaves its outputs undefined, without a status.
  * ------------------------------------------------------------------------------------------- */
 size_t mla_gqla_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                                int32_t max_pages);
