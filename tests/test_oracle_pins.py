@@ -284,6 +284,65 @@ def test_append_one_at_a_time_equals_bulk():
         np.testing.assert_allclose(kr1[0], kr_all[j], rtol=1e-13, atol=1e-13)
 
 
+def _latent_rows_case():
+    r = _rng(43)
+    n, C, d_c, d_r = 6, 24, 10, 8
+    x = r.standard_normal((n, C)) * r.uniform(0.2, 5.0, (n, 1))
+    W_DKV, W_KR = r.standard_normal((C, d_c)), r.standard_normal((C, d_r))
+    gamma = r.uniform(0.5, 1.5, d_c)
+    positions = np.array([0, 1, 5, 77, 1000, 131071])
+    return x, W_DKV, W_KR, gamma, positions
+
+
+def test_latent_rows_match_torch_rms_norm_and_complex_rotation():
+    """Cache rows (« L'idée : garder un résumé », « L'obstacle : RoPE »): the latent is torch's own
+    rms_norm of x·W_DKV (its normalised_shape fixes the axis), times the gain; the RoPE key is
+    x·W_KR with each adjacent pair (2i, 2i+1) read as a complex number and multiplied by
+    exp(i·pos·10000^(-2i/d_r)) at the row's own position. Position 0 leaves the key unrotated."""
+    x, W_DKV, W_KR, gamma, positions = _latent_rows_case()
+    c, k_r = O.latent_rows(x, W_DKV, W_KR, positions, gamma, 1e-6, 10000.0)
+    d_c, d_r = W_DKV.shape[1], W_KR.shape[1]
+    c_ref = torch.nn.functional.rms_norm(torch.from_numpy(x @ W_DKV), (d_c,), torch.from_numpy(gamma), eps=1e-6).numpy()
+    np.testing.assert_allclose(c, c_ref, rtol=1e-12, atol=1e-13)
+    z = x @ W_KR
+    pairs = z[:, 0::2] + 1j * z[:, 1::2]
+    turn = 10000.0 ** (-2.0 * np.arange(d_r // 2) / d_r)
+    rotated = pairs * np.exp(1j * positions[:, None].astype(float) * turn[None, :])
+    k_ref = np.empty_like(z)
+    k_ref[:, 0::2], k_ref[:, 1::2] = rotated.real, rotated.imag
+    np.testing.assert_allclose(k_r, k_ref, rtol=1e-9, atol=1e-9)
+    np.testing.assert_array_equal(k_r[0], z[0])
+    c1, _ = O.latent_rows(x, W_DKV, W_KR, positions, None, 0.0)
+    np.testing.assert_allclose((c1 ** 2).mean(axis=1), 1.0, rtol=1e-13)
+
+
+def test_planted_latent_row_slips_are_caught(monkeypatch):
+    """Three plausible slips in the cache-row oracle each fail the pin above: the key rotated one
+    position late, the latent and the RoPE part normalised together, and the two column blocks of
+    the concatenated projection [W_DKV | W_KR] taken in the wrong order."""
+    good = O.latent_rows
+
+    def late(x, W_DKV, W_KR, positions, gamma=None, eps=1e-6, base=10000.0):
+        return good(x, W_DKV, W_KR, np.asarray(positions) + 1, gamma, eps, base)
+
+    def joint(x, W_DKV, W_KR, positions, gamma=None, eps=1e-6, base=10000.0):
+        d_c = np.asarray(W_DKV).shape[1]
+        zn = O.rms_norm(np.asarray(x, float) @ np.concatenate([W_DKV, W_KR], 1), None, eps)
+        c = zn[:, :d_c] * (1.0 if gamma is None else np.asarray(gamma))
+        return c, O.rope(zn[:, d_c:], positions, base)
+
+    def swapped(x, W_DKV, W_KR, positions, gamma=None, eps=1e-6, base=10000.0):
+        d_c = np.asarray(W_DKV).shape[1]
+        z = np.asarray(x, float) @ np.concatenate([W_KR, W_DKV], 1)
+        return O.rms_norm(z[:, :d_c], gamma, eps), O.rope(z[:, d_c:], positions, base)
+
+    for bad in (late, joint, swapped):
+        monkeypatch.setattr(O, "latent_rows", bad)
+        with pytest.raises(AssertionError):
+            test_latent_rows_match_torch_rms_norm_and_complex_rotation()
+    monkeypatch.setattr(O, "latent_rows", good)
+
+
 def test_multi_token_step_equals_sequential_single_token_steps():
     # causal among the new tokens: token t of an s_q step is a 1-token step on seqlen - s_q + t + 1
     s_q, n = 4, 30
