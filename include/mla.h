@@ -16,6 +16,8 @@
  *    16-byte aligned and every row stride a multiple of 16 bytes.
  *  - dtype is MLA_F32 or MLA_BF16; it is the storage type of the cache, weights, queries and
  *    outputs of that call. Accumulation, softmax and normalisation are fp32 in every kernel.
+ *  - B sequences with s_q new tokens each: B * s_q must not exceed INT32_MAX (else
+ *    MLA_ERR_INVALID_ARG).
  *  - seqlens[b] counts the cached positions of sequence b INCLUDING this step's s_q new tokens;
  *    new token t (0 <= t < s_q) sits at position seqlens[b] - s_q + t and attends positions
  *    0 .. seqlens[b] - s_q + t (causal among the new tokens).
@@ -52,7 +54,8 @@ enum mla_status {
 
 enum mla_dtype { MLA_F32 = 0, MLA_BF16 = 1 };
 
-/* Shapes of one layer. sm_scale multiplies every score: 1/sqrt(D + d_r) (« L'obstacle : RoPE »). */
+/* Shapes of one layer. sm_scale multiplies every score; 0 selects 1/sqrt(D + d_r), the scale of
+ * « L'obstacle : RoPE » (a negative or NaN value is an invalid argument). */
 typedef struct mla_dims {
   int32_t H;          /* query heads */
   int32_t D;          /* no-RoPE width of a query/key head (qk_nope) */
@@ -61,7 +64,7 @@ typedef struct mla_dims {
   int32_t d_v;        /* value head width */
   int32_t g;          /* GQLA groups, H % g == 0 (0 when the grouped path is not used) */
   int32_t page_size;  /* positions per cache page; must be 64 */
-  float sm_scale;     /* score scale */
+  float sm_scale;     /* score scale; 0 = 1/sqrt(D + d_r) */
   float rms_eps;      /* RMSNorm epsilon: c = z / sqrt(mean(z^2) + rms_eps) * gamma */
   float rope_base;    /* RoPE: pair (2i, 2i+1) turns by pos * rope_base^(-2i/d_r) */
 } mla_dims_t;
@@ -110,10 +113,13 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
  * mla_append_cache, minus the workspace: the split-K partial sums go to a 4 MiB buffer that is
  * part of the library's device image (every GPU that loads the library holds it until exit).
  * Nothing is allocated or freed. Limit: B * s_q * (d_c + d_r) <= 1,048,576, else
- * MLA_ERR_WORKSPACE is returned and nothing is launched. The first call on each device looks up
- * the buffer's device address (with that device current) and caches it; make that first call
- * before any stream capture. All calls share the buffer: calls that overlap on the GPU (streams
- * with no ordering between them) race on it. Nothing in it needs to start at zero.
+ * MLA_ERR_WORKSPACE is returned and nothing is launched. In bf16 with C a multiple of 64 the
+ * projection runs on the tensor cores, as in mla_append_cache. The first call on each device looks
+ * up the buffer's device address (with that device current) and caches it; make that first call
+ * before any stream capture. A reset of the device (cudaDeviceReset) makes the cached address
+ * stale: after one, this call must not be used again in the same process. All calls share the
+ * buffer: calls that overlap on the GPU (streams with no ordering between them) race on it.
+ * Nothing in it needs to start at zero.
  * ------------------------------------------------------------------------------------------- */
 int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                              const void* x, int32_t C, const void* w_dkv_kr, const void* gamma,
@@ -189,8 +195,8 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
  *   out[b,t,h,:] = sum_j softmax(s)_j * V[j, g(h), :]          lse[b,t,h] = log sum_j exp(s_j)
  *   q_nope [B, s_q, H, D]  q_rope_raw [B, s_q, H, d_r]  out [B, s_q, H, d_v] (dtype)  lse fp32
  * workspace: at least mla_gqla_workspace_size(...) bytes.
- * Requires every seqlens[b] >= s_q, as a3 does. The bf16 tensor-core kernel does not check it on
- * the device: a shorter sequence leaves its outputs undefined, without a status.
+ * Requires every seqlens[b] >= s_q, as a3 does: a sequence shorter than that is reported on the
+ * device (MLA_ERR_DEVICE_CHECK) and its outputs are undefined.
  * ------------------------------------------------------------------------------------------- */
 size_t mla_gqla_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                                int32_t max_pages);

@@ -137,6 +137,9 @@ gqla_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
   }
   if (warp == 2) { ptx::tmem_alloc(base + kOffTmemSlot, kTmemCols); ptx::tmem_relinquish(); }
   grid_dependency_wait();
+  // a sequence must hold at least its new token: an empty one is reported (its outputs stay unwritten)
+  for (int b = blockIdx.x * kThreads + threadIdx.x; b < p.B; b += gridDim.x * kThreads)
+    if (p.seqlens[b] < 1) report(MLA_ERR_DEVICE_CHECK);
   ptx::tc_fence_before();
   __syncthreads();
   allow_dependents();

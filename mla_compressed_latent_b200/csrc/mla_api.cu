@@ -47,9 +47,22 @@ int check_dims(const mla_dims_t* d) {
   if (d->H <= 0 || d->D <= 0 || d->d_r <= 0 || (d->d_r & 1) || d->d_c <= 0 || d->d_v <= 0)
     return MLA_ERR_INVALID_ARG;
   if (d->page_size != 64) return MLA_ERR_INVALID_ARG;
-  if (!(d->sm_scale > 0.f) || !(d->rms_eps >= 0.f) || !(d->rope_base > 0.f)) return MLA_ERR_INVALID_ARG;
+  if (!(d->sm_scale >= 0.f) || !(d->rms_eps >= 0.f) || !(d->rope_base > 0.f)) return MLA_ERR_INVALID_ARG;
   return MLA_OK;
 }
+
+// The score scale a call uses: dims->sm_scale, or 1/sqrt(D + d_r) when it is 0.
+float score_scale(const mla_dims_t* d) {
+  return d->sm_scale > 0.f ? d->sm_scale : (float)(1.0 / sqrt((double)d->D + (double)d->d_r));
+}
+mla_dims_t with_scale(const mla_dims_t* d) {
+  mla_dims_t r = *d;
+  r.sm_scale = score_scale(d);
+  return r;
+}
+
+// Token counts are formed as B * s_q in 32 bits; a product past INT32_MAX is an invalid argument.
+bool tokens_ok(int32_t B, int32_t s_q) { return B > 0 && s_q > 0 && (int64_t)B * s_q <= INT32_MAX; }
 
 int check_dtype(int32_t dtype) { return (dtype == MLA_F32 || dtype == MLA_BF16) ? MLA_OK : MLA_ERR_INVALID_ARG; }
 
@@ -167,7 +180,7 @@ int mla_check_status(void* stream) {
 // a1
 // ------------------------------------------------------------------------------------------------
 size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C) {
-  if (check_dims(dims) || B <= 0 || s_q <= 0 || C <= 0) return 0;
+  if (check_dims(dims) || !tokens_ok(B, s_q) || C <= 0) return 0;
   const int n_tok = B * s_q, N = dims->d_c + dims->d_r;
   int ks = append_ksplit(n_tok, C, N);
   if (mla::gemm::supported(C, N)) ks = std::max(ks, append_tc_splits(n_tok, C, N));
@@ -181,7 +194,7 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
-  if (B <= 0 || s_q <= 0 || C <= 0 || max_pages <= 0 || !x || !w_dkv_kr || !seqlens || !block_table || !cache)
+  if (!tokens_ok(B, s_q) || C <= 0 || max_pages <= 0 || !x || !w_dkv_kr || !seqlens || !block_table || !cache)
     return MLA_ERR_INVALID_ARG;
   if (!cache->latent || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_dkv_kr) || (gamma && !aligned16(gamma)) || !aligned16(cache->latent) ||
@@ -196,14 +209,17 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
   if (!workspace || ws_bytes < need) return MLA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MLA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t fin_smem = (size_t)N * sizeof(float);
+  // attributes first: a failure here leaves nothing enqueued
+  if ((rc = dtype == MLA_F32 ? set_smem(mla::simt::append_finish_kernel<float>, fin_smem)
+                             : set_smem(mla::simt::append_finish_kernel<__nv_bfloat16>, fin_smem)))
+    return rc;
   if (tc) {
     using T = __nv_bfloat16;
     mla::gemm::Params p{};
     p.mode = 1;
     p.part = reinterpret_cast<float*>(workspace);
     if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, ks}), p, st))) return rc;
-    const size_t fin_smem = (size_t)N * sizeof(float);
-    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
     const int fin_threads = std::min(1024, (N + 31) / 32 * 32);   // one thread per output column
     mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)p.part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
@@ -214,12 +230,10 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
   dim3 grid((N + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS,
             (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK, ks);
   float* part = reinterpret_cast<float*>(workspace);
-  const size_t fin_smem = (size_t)N * sizeof(float);
   if (dtype == MLA_F32) {
     using T = float;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, 
         (const T*)x, n_tok, C, (const T*)w_dkv_kr, N, k_chunk, part, nullptr);
-    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
     launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, 
         part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
         block_table, max_pages, (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride,
@@ -228,7 +242,6 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     using T = __nv_bfloat16;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, 
         (const T*)x, n_tok, C, (const T*)w_dkv_kr, N, k_chunk, part, nullptr);
-    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
     launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, 
         part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
         block_table, max_pages, (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride,
@@ -251,7 +264,7 @@ size_t query_part_bytes(int ks, int n_tok, int d_q) { return ((size_t)ks * n_tok
 }  // namespace
 
 size_t mla_query_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C, int32_t d_q) {
-  if (check_dims(dims) || B <= 0 || s_q <= 0 || C <= 0 || d_q <= 0) return 0;
+  if (check_dims(dims) || !tokens_ok(B, s_q) || C <= 0 || d_q <= 0) return 0;
   const int n_tok = B * s_q;
   int ks = append_ksplit(n_tok, C, d_q);
   if (mla::gemm::supported(C, d_q)) ks = std::max(ks, append_tc_splits(n_tok, C, d_q));
@@ -264,7 +277,7 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
-  if (B <= 0 || s_q <= 0 || C <= 0 || d_q <= 0 || !x || !w_dq || !w_uq || !w_qr || !q_nope || !q_rope_raw)
+  if (!tokens_ok(B, s_q) || C <= 0 || d_q <= 0 || !x || !w_dq || !w_uq || !w_qr || !q_nope || !q_rope_raw)
     return MLA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_dq) || (gamma_q && !aligned16(gamma_q)) || !aligned16(w_uq) ||
       !aligned16(w_qr) || !aligned16(q_nope) || !aligned16(q_rope_raw))
@@ -334,7 +347,7 @@ int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
-  if (B <= 0 || s_q <= 0 || !q_nope || !q_rope_raw || !w_uk || !seqlens || !q_abs) return MLA_ERR_INVALID_ARG;
+  if (!tokens_ok(B, s_q) || !q_nope || !q_rope_raw || !w_uk || !seqlens || !q_abs) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_nope) || !aligned16(q_rope_raw) || !aligned16(w_uk) || !aligned16(q_abs) || !aligned16(seqlens))
     return MLA_ERR_INVALID_ARG;
   const int n_tok = B * s_q;
@@ -375,7 +388,7 @@ int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
 // a3 + a4
 // ------------------------------------------------------------------------------------------------
 size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, int32_t max_pages) {
-  if (check_dims(dims) || check_dtype(dtype) || B <= 0 || s_q <= 0 || max_pages <= 0) return 0;
+  if (check_dims(dims) || check_dtype(dtype) || !tokens_ok(B, s_q) || max_pages <= 0) return 0;
   size_t ws = simt_decode_ws(B * s_q, dims->H, dims->d_c, max_pages);
   ws = std::max(ws, mla::sm100::decode_workspace_bytes(dims, dtype, B, s_q, num_sms()));
   return ws;
@@ -388,7 +401,7 @@ int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
-  if (B <= 0 || s_q <= 0 || max_pages <= 0 || !q_abs || !cache || !block_table || !seqlens || !o_lat || !lse)
+  if (!tokens_ok(B, s_q) || max_pages <= 0 || !q_abs || !cache || !block_table || !seqlens || !o_lat || !lse)
     return MLA_ERR_INVALID_ARG;
   if (!cache->latent || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_abs) || !aligned16(cache->latent) || !aligned16(cache->rope) || !aligned16(block_table) ||
@@ -400,7 +413,8 @@ int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_
   const int n_tok = B * s_q;
 
   if (mla::sm100::decode_supported(dims, dtype, B, s_q)) {
-    return mla::sm100::launch_decode(dims, B, s_q, q_abs, cache, block_table, max_pages, seqlens, o_lat, lse,
+    const mla_dims_t dd = with_scale(dims);
+    return mla::sm100::launch_decode(&dd, B, s_q, q_abs, cache, block_table, max_pages, seqlens, o_lat, lse,
                                      workspace, ws_bytes, num_sms(), st);
   }
 
@@ -416,7 +430,7 @@ int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_
   A.Dk = dims->d_c; A.Dv = dims->d_c; A.d_r = dims->d_r; A.H = dims->H; A.heads_per_group = dims->H;
   A.kv_shared = 1;
   A.block_table = block_table; A.max_pages = max_pages; A.num_pages = cache->num_pages;
-  A.seqlens = seqlens; A.s_q = s_q; A.sm_scale = dims->sm_scale; A.rope_base = dims->rope_base;
+  A.seqlens = seqlens; A.s_q = s_q; A.sm_scale = score_scale(dims); A.rope_base = dims->rope_base;
   A.out = o_lat; A.out_head_stride = dims->d_c; A.lse = lse;
   SimtSplit sp = simt_split(n_tok, dims->H, max_pages);
   A.nsplit = sp.nsplit; A.chunk = sp.chunk;
@@ -432,7 +446,7 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
-  if (B <= 0 || s_q <= 0 || !o_lat || !w_uv || !out) return MLA_ERR_INVALID_ARG;
+  if (!tokens_ok(B, s_q) || !o_lat || !w_uv || !out) return MLA_ERR_INVALID_ARG;
   if (w_o && (C <= 0 || !out_model)) return MLA_ERR_INVALID_ARG;
   if (!aligned16(o_lat) || !aligned16(w_uv) || !aligned16(out) || (w_o && (!aligned16(w_o) || !aligned16(out_model))))
     return MLA_ERR_INVALID_ARG;
@@ -481,7 +495,7 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
 // a6
 // ------------------------------------------------------------------------------------------------
 size_t mla_gqla_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, int32_t max_pages) {
-  if (check_dims(dims) || check_dtype(dtype) || B <= 0 || s_q <= 0 || max_pages <= 0) return 0;
+  if (check_dims(dims) || check_dtype(dtype) || !tokens_ok(B, s_q) || max_pages <= 0) return 0;
   size_t ws = simt_decode_ws(B * s_q, dims->H, dims->d_v, max_pages);
   if (dims->g > 0 && mla::gqla::supported(dims, dtype, s_q))
     ws = std::max(ws, mla::gqla::workspace_bytes(dims, B, max_pages, num_sms()));
@@ -496,7 +510,7 @@ int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, in
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
   if (dims->g <= 0 || dims->H % dims->g) return MLA_ERR_INVALID_ARG;
-  if (B <= 0 || s_q <= 0 || max_pages <= 0 || !q_nope || !q_rope_raw || !cache || !block_table || !seqlens ||
+  if (!tokens_ok(B, s_q) || max_pages <= 0 || !q_nope || !q_rope_raw || !cache || !block_table || !seqlens ||
       !out || !lse)
     return MLA_ERR_INVALID_ARG;
   if (!cache->k || !cache->v || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
@@ -508,9 +522,11 @@ int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, in
   if (!stride_ok(cache->k_stride, dtype, (int64_t)dims->g * dims->D) ||
       !stride_ok(cache->v_stride, dtype, (int64_t)dims->g * dims->d_v) || !stride_ok(cache->rope_stride, dtype, dims->d_r))
     return MLA_ERR_INVALID_ARG;
-  if (mla::gqla::supported(dims, dtype, s_q))
-    return mla::gqla::launch_gqla(dims, B, q_nope, q_rope_raw, cache, block_table, max_pages, seqlens, out, lse,
+  if (mla::gqla::supported(dims, dtype, s_q)) {
+    const mla_dims_t dd = with_scale(dims);
+    return mla::gqla::launch_gqla(&dd, B, q_nope, q_rope_raw, cache, block_table, max_pages, seqlens, out, lse,
                                   workspace, ws_bytes, num_sms(), reinterpret_cast<cudaStream_t>(stream));
+  }
   if (hpg % mla::simt::DEC_HEADS || dims->d_v % 32 || dims->d_v > 32 * mla::simt::DEC_MAX_OV) return MLA_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int n_tok = B * s_q;
@@ -524,7 +540,7 @@ int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, in
   A.Dk = dims->D; A.Dv = dims->d_v; A.d_r = dims->d_r; A.H = dims->H; A.heads_per_group = hpg;
   A.kv_shared = 0;
   A.block_table = block_table; A.max_pages = max_pages; A.num_pages = cache->num_pages;
-  A.seqlens = seqlens; A.s_q = s_q; A.sm_scale = dims->sm_scale; A.rope_base = dims->rope_base;
+  A.seqlens = seqlens; A.s_q = s_q; A.sm_scale = score_scale(dims); A.rope_base = dims->rope_base;
   A.out = out; A.out_head_stride = dims->d_v; A.lse = lse;
   SimtSplit sp = simt_split(n_tok, dims->H, max_pages);
   A.nsplit = sp.nsplit; A.chunk = sp.chunk;
@@ -582,7 +598,7 @@ extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, i
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
-  if (B <= 0 || s_q <= 0 || C <= 0 || max_pages <= 0 || !x || !w_dkv_kr || !seqlens || !block_table || !cache)
+  if (!tokens_ok(B, s_q) || C <= 0 || max_pages <= 0 || !x || !w_dkv_kr || !seqlens || !block_table || !cache)
     return MLA_ERR_INVALID_ARG;
   if (!cache->latent || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_dkv_kr) || (gamma && !aligned16(gamma)) || !aligned16(cache->latent) ||
@@ -594,19 +610,38 @@ extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, i
   // as many K slices as the built-in buffer holds, at most the number the workspace path uses
   const size_t per_slice = (size_t)n_tok * N;
   if (per_slice > kAppendScratchFloats) return MLA_ERR_WORKSPACE;   // B*s_q*(d_c+d_r) > 1,048,576
-  const int ks = std::min(append_ksplit(n_tok, C, N), (int)(kAppendScratchFloats / per_slice));
+  const int cap = (int)(kAppendScratchFloats / per_slice);
+  const bool tc = append_on_tc(dtype, C, N);
+  const int ks = std::min(tc ? append_tc_splits(n_tok, C, N) : append_ksplit(n_tok, C, N), cap);
+  const size_t fin_smem = (size_t)N * sizeof(float);
+  // attributes first: a failure here leaves nothing enqueued
+  if ((rc = dtype == MLA_F32 ? set_smem(mla::simt::append_finish_kernel<float>, fin_smem)
+                             : set_smem(mla::simt::append_finish_kernel<__nv_bfloat16>, fin_smem)))
+    return rc;
   float* part = nullptr;
   if ((rc = append_scratch_address(&part))) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (tc) {
+    // the tensor-core projection writes one fp32 slice per K split (an empty split writes zeros)
+    using T = __nv_bfloat16;
+    mla::gemm::Params p{};
+    p.mode = 1;
+    p.part = part;
+    if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, ks}), p, st))) return rc;
+    const int fin_threads = std::min(1024, (N + 31) / 32 * 32);
+    mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st,
+                    (const float*)part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps,
+                    dims->rope_base, seqlens, block_table, max_pages, (T*)cache->latent, cache->latent_stride,
+                    (T*)cache->rope, cache->rope_stride, cache->num_pages);
+    return launch_status();
+  }
   const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
   dim3 grid((N + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS,
             (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK, ks);
-  const size_t fin_smem = (size_t)N * sizeof(float);
   if (dtype == MLA_F32) {
     using T = float;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, (const T*)x, n_tok, C,
            (const T*)w_dkv_kr, N, k_chunk, part, (T*)nullptr);
-    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
     launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
            (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);
@@ -614,7 +649,6 @@ extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, i
     using T = __nv_bfloat16;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, (const T*)x, n_tok, C,
            (const T*)w_dkv_kr, N, k_chunk, part, (T*)nullptr);
-    if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
     launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
            (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);

@@ -7,7 +7,6 @@ the computation runs in the library's CUDA kernels; a failing call raises MlaErr
 from __future__ import annotations
 
 import ctypes
-import math
 from dataclasses import dataclass
 
 import torch
@@ -36,8 +35,8 @@ class Dims:
     rope_base: float = 10000.0
 
     def c(self) -> L.MlaDims:
-        scale = self.sm_scale or 1.0 / math.sqrt(self.D + self.d_r)
-        return L.MlaDims(self.H, self.D, self.d_r, self.d_c, self.d_v, self.g, self.page_size, scale,
+        # sm_scale 0 lets the library use its default, 1/sqrt(D + d_r)
+        return L.MlaDims(self.H, self.D, self.d_r, self.d_c, self.d_v, self.g, self.page_size, self.sm_scale,
                          self.rms_eps, self.rope_base)
 
     @staticmethod

@@ -59,7 +59,7 @@ def _dims(**kw):
 def test_invalid_dims_rejected_before_any_launch(lib):
     p = ctypes.c_void_p(16)
     cache = L.MlaLatentCache(16, 576, 16 + 1024, 576, 10)
-    for bad in [_dims(H=0), _dims(d_r=3), _dims(page_size=32), _dims(sm_scale=0.0), _dims(d_c=-1)]:
+    for bad in [_dims(H=0), _dims(d_r=3), _dims(page_size=32), _dims(sm_scale=-1.0), _dims(d_c=-1)]:
         rc = lib.mla_decode_absorbed(ctypes.byref(bad), 1, 1, 1, p, ctypes.byref(cache), p, 1, p, p, p, None, 0, None)
         assert rc == L.MLA_ERR_INVALID_ARG
 

@@ -119,8 +119,28 @@ def test_one_bad_argument_is_rejected(lib, name, i, bad, want):
 def test_bad_dtype_and_dims_are_rejected(lib, name):
     tmpl = CALLS[name][0]
     assert _call(lib, name, tmpl, dtype=7) == L.MLA_ERR_INVALID_ARG
-    for bad in (_dims(H=0), _dims(d_c=-1), _dims(page_size=32), _dims(sm_scale=0.0)):
+    for bad in (_dims(H=0), _dims(d_c=-1), _dims(page_size=32), _dims(sm_scale=-1.0), _dims(sm_scale=float("nan"))):
         assert _call(lib, name, tmpl, dims=bad) == L.MLA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", list(CALLS))
+def test_token_count_past_int32_is_rejected(lib, name):
+    """B * s_q is formed in 32 bits: a product past INT32_MAX is an invalid argument, found before
+    any size is computed from it."""
+    tmpl = list(CALLS[name][0])
+    tmpl[0], tmpl[1] = 1 << 16, 1 << 16
+    assert _call(lib, name, tmpl) == L.MLA_ERR_INVALID_ARG
+    tmpl[0], tmpl[1] = 46341, 46341
+    assert _call(lib, name, tmpl) == L.MLA_ERR_INVALID_ARG
+
+
+def test_zero_score_scale_selects_the_default(lib):
+    """sm_scale = 0 is valid (the library then uses 1/sqrt(D + d_r)); the size queries answer for it."""
+    d = _dims(sm_scale=0.0)
+    assert lib.mla_decode_workspace_size(ctypes.byref(d), 1, 64, 1, 64) > 0
+    assert lib.mla_append_workspace_size(ctypes.byref(d), 64, 1, 7168) > 0
+    big = _dims(sm_scale=0.0)
+    assert lib.mla_append_workspace_size(ctypes.byref(big), 1 << 16, 1 << 16, 7168) == 0
 
 
 @pytest.mark.parametrize("field,value", [("latent", 0), ("rope", 0), ("latent", ODD), ("latent_stride", 577),

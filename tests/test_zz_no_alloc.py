@@ -4,7 +4,8 @@ Such callers (a framework whose memory pool owns the device, a plugin that only 
 tensors of the call, a serving process that must not call cudaMalloc) get the same result as
 mla_append_cache without passing a workspace: the partial sums live in a fixed buffer inside the
 library. These checks call it through the C ABI and compare it with the workspace entry point on
-two calls in a row (the shared buffer keeps the first call's contents when the second one runs).
+two calls in a row (the shared buffer keeps the first call's contents when the second one runs), and
+the rows each call writes with the fp64 oracle's cache rows.
 This file is collected last so that a failure here never hides the other tests.
 """
 import ctypes
@@ -14,6 +15,7 @@ import pytest
 import torch
 
 import synth
+from oracle import mla_oracle as O
 from mla_compressed_latent_b200 import _lib as L
 from mla_compressed_latent_b200 import ops
 from mla_compressed_latent_b200.ops import Dims, LatentCache
@@ -66,6 +68,13 @@ def test_noalloc_append_matches_workspace_append_on_two_calls(name, B):
         pos = (lens - 7 * call - 1).astype(np.int64)
         rows = table[np.arange(B), pos // 64].astype(np.int64) * 64 + pos % 64
         assert np.all(np.abs(got[rows]).max(axis=1) > 0)
+        # and they are the oracle's cache rows of these tokens at these positions
+        w64 = wcat.double().cpu().numpy()   # the weights as stored (the call reads them in its dtype)
+        c, kr = O.latent_rows(x[:, 0].double().cpu().numpy(), w64[:, :w.d_c], w64[:, w.d_c:], pos, None,
+                              w.rms_eps, w.rope_base)
+        want = np.concatenate([c, kr], 1)
+        err = np.abs(got[rows] - want).max() / np.abs(want).max()
+        assert err <= TOL[w.dtype], f"call {call}: rows vs oracle max|Δ|/max|ref| = {err:.3e}"
 
 
 def test_noalloc_append_rejects_batches_beyond_its_buffer():
