@@ -31,24 +31,6 @@
 namespace mla {
 namespace sm100 {
 
-// Optional per-role cycle counters (build with -DMLA_DECODE_PROFILE; absent otherwise).
-#ifdef MLA_DECODE_PROFILE
-__device__ long long g_prof[148][2][12][16];
-#define PROF_DECL() long long prof_[14] = {0}; const long long prof_t0_ = clock64()
-#define PROF_MARK(v) const long long v = clock64()
-#define PROF_ADD(i, from) (prof_[i] += clock64() - (from))
-#define PROF_SAVE(its) do { if (pair < 148) { for (int k_ = 0; k_ < 14; ++k_) g_prof[pair][rank][warp][k_] = prof_[k_]; \
-    g_prof[pair][rank][warp][14] = clock64() - prof_t0_; g_prof[pair][rank][warp][15] = (its); } } while (0)
-__device__ unsigned long long g_ptime[148][2][16];
-#define PROF_TIME(k) do { if (pair < 148) g_ptime[pair][rank][k] = ptx::globaltimer(); } while (0)
-#else
-#define PROF_TIME(k) do {} while (0)
-#define PROF_DECL() do {} while (0)
-#define PROF_MARK(v) do {} while (0)
-#define PROF_ADD(i, from) do {} while (0)
-#define PROF_SAVE(its) do {} while (0)
-#endif
-
 constexpr int kH = 128, kDC = 512, kDR = 64, kRow = kDC + kDR;
 constexpr int kTile = 64;                              // positions per tile = one cache page
 constexpr int kChunkBytes = 64 * 128;                  // one TMA box: 64 rows x 64 bf16
@@ -67,7 +49,6 @@ constexpr int kQCols = kRow / 2;                       // 288 TMEM columns hold 
 constexpr int kSCol0 = kQCols;                         // S buffers at 288, 352, 416
 constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;                   // lazy rescale threshold (log2 units)
-constexpr bool kExpHalf2 = false;                      // softmax exponentials two per SFU op (f16x2)
 constexpr int kThreads = 384;                          // 4 control warps + 8 row warps
 constexpr int kGroup = 256;                            // threads of the row warps (4-11)
 constexpr uint64_t kTimeoutNs = 2000000000ull;
@@ -127,15 +108,16 @@ constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 64, false);   // S = QÌƒ Â
 constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, 256, true);   // O += P Â· C   (MN-major B)
 
 struct Params {
-  const __nv_bfloat16* q_abs;  // [B, 128, 576]
+  const __nv_bfloat16* q_abs;  // [B, s_q, 128, 576]
   const int32_t* block_table;
   int max_pages;
   int num_pages;
   const int32_t* seqlens;
   int B;
+  int s_q;                     // new tokens per sequence (the pairs form groups of s_q, one token each)
   int max_tiles;               // max_pages: a sequence never reads past its table row
-  __nv_bfloat16* o_lat;        // [B, 128, 512]
-  float* lse;                  // [B, 128]
+  __nv_bfloat16* o_lat;        // [B, s_q, 128, 512]
+  float* lse;                  // [B, s_q, 128]
   float* part_o;               // [2 * pairs, 128, 512]
   float* part_lse;             // [2 * pairs, 128]
   float sm_scale_log2;         // sm_scale * log2(e)
@@ -185,23 +167,10 @@ __device__ __forceinline__ void softmax_rows(const uint32_t (&sr)[32], int valid
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int c = 8 * j + 2 * t4;
-    float e00, e01, e10, e11;
-    if constexpr (kExpHalf2) {
-      // two exponentials per SFU operation: arguments (at most 2^kRescaleLog2) rounded to f16
-      // (relative error of the result at most about 2^-8, the order of P's own bf16 rounding),
-      // a masked column's argument is -inf, whose exponential is 0
-      const float x00 = (!kMask || c < valid) ? fmaf(__uint_as_float(sr[4 * j]), scale2, -m0) : -INFINITY;
-      const float x01 = (!kMask || c + 1 < valid) ? fmaf(__uint_as_float(sr[4 * j + 1]), scale2, -m0) : -INFINITY;
-      const float x10 = (!kMask || c < valid) ? fmaf(__uint_as_float(sr[4 * j + 2]), scale2, -m1) : -INFINITY;
-      const float x11 = (!kMask || c + 1 < valid) ? fmaf(__uint_as_float(sr[4 * j + 3]), scale2, -m1) : -INFINITY;
-      ptx::ex2_half2(x00, x01, e00, e01);
-      ptx::ex2_half2(x10, x11, e10, e11);
-    } else {
-      e00 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j]), scale2, -m0)) : 0.f;
-      e01 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 1]), scale2, -m0)) : 0.f;
-      e10 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 2]), scale2, -m1)) : 0.f;
-      e11 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 3]), scale2, -m1)) : 0.f;
-    }
+    const float e00 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j]), scale2, -m0)) : 0.f;
+    const float e01 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 1]), scale2, -m0)) : 0.f;
+    const float e10 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 2]), scale2, -m1)) : 0.f;
+    const float e11 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 3]), scale2, -m1)) : 0.f;
     if (j & 1) {
       ls1 += e00 + e01;
       ls3 += e10 + e11;
@@ -258,12 +227,14 @@ struct SegIter {
   }
 };
 
-// The work split. Default: the tiles of all sequences laid end to end and cut into one contiguous
-// range per pair (balanced to a tile), pair p taking [p*T/P, (p+1)*T/P). A sequence cut between pairs
-// costs its pairs a segment switch, fp32 partials and the merge; so when there are no more sequences
-// than pairs and the longest is within kSplitSlack tiles of the balanced share, each pair takes one
-// whole sequence instead (pair p takes sequence p; nothing is cut). Both the decode and the merge
-// kernel decide it the same way from seqlens.
+// The work split. The pairs form G = P / s_q groups of s_q pairs; pair p is token p % s_q of group
+// p / s_q, and the s_q pairs of a group walk the same tiles together (each page is read from DRAM
+// once and from L2 by the group's other pairs). Default: the tiles of all sequences laid end to end
+// and cut into one contiguous range per group (balanced to a tile), group g taking [g*T/G, (g+1)*T/G).
+// A sequence cut between groups costs its pairs a segment switch, fp32 partials and the merge; so
+// when there are no more sequences than groups and the longest is within kSplitSlack tiles of the
+// balanced share, each group takes one whole sequence instead (group g takes sequence g; nothing is
+// cut). Both the decode and the merge kernel decide it the same way from seqlens.
 constexpr int kSplitSlack = 12;
 __device__ __forceinline__ bool whole_sequences(int B, int npairs, long long T, int max_tb) {
   return B <= npairs && (long long)max_tb <= (T + npairs - 1) / npairs + kSplitSlack;
@@ -271,7 +242,7 @@ __device__ __forceinline__ bool whole_sequences(int B, int npairs, long long T, 
 
 // One warp: total tiles T, this pair's range, and the sequence holding its first tile. Lane l scans
 // sequences [l*per, (l+1)*per).
-__device__ void plan_range(const int32_t* seqlens, int B, int max_tiles, int pair, int npairs, long long* out) {
+__device__ void plan_range(const int32_t* seqlens, int B, int s_q, int max_tiles, int pair, int npairs, long long* out) {
   const int lane = threadIdx.x & 31;
   const int per = (B + 31) / 32;
   const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
@@ -279,7 +250,7 @@ __device__ void plan_range(const int32_t* seqlens, int B, int max_tiles, int pai
   int max_tb = 0;
   for (int b = b0; b < b1; ++b) {
     const int L = seqlens[b];
-    if (L < 1 || (L + kTile - 1) / kTile > max_tiles) report(MLA_ERR_DEVICE_CHECK);
+    if (L < s_q || (L + kTile - 1) / kTile > max_tiles) report(MLA_ERR_DEVICE_CHECK);
     const int tb = tiles_of(L, max_tiles);
     local += tb;
     max_tb = max(max_tb, tb);
@@ -294,19 +265,24 @@ __device__ void plan_range(const int32_t* seqlens, int B, int max_tiles, int pai
   const long long T = __shfl_sync(0xffffffffu, incl, 31);
   const long long excl = incl - local;
   if (lane == 0) out[4] = T;
-  if (whole_sequences(B, npairs, T, max_tb)) {
-    // pair p: sequence p whole
-    if (pair >= B) {
+  const int G = npairs / s_q, grp = pair / s_q;
+  if (grp >= G) {   // left over when s_q does not divide the pairs: no work
+    if (lane == 0) { out[0] = 0; out[1] = 0; out[2] = 0; out[3] = B; }
+    return;
+  }
+  if (whole_sequences(B, G, T, max_tb)) {
+    // group g: sequence g whole
+    if (grp >= B) {
       if (lane == 0) { out[0] = 0; out[1] = 0; out[2] = 0; out[3] = B; }
-    } else if (pair >= b0 && pair < b1) {
+    } else if (grp >= b0 && grp < b1) {
       long long off = excl;
-      for (int b = b0; b < pair; ++b) off += tiles_of(seqlens[b], max_tiles);
-      out[0] = off; out[1] = off + tiles_of(seqlens[pair], max_tiles); out[2] = off; out[3] = pair;
+      for (int b = b0; b < grp; ++b) off += tiles_of(seqlens[b], max_tiles);
+      out[0] = off; out[1] = off + tiles_of(seqlens[grp], max_tiles); out[2] = off; out[3] = grp;
     }
     return;
   }
-  const long long start = (long long)pair * T / npairs;
-  const long long end = (long long)(pair + 1) * T / npairs;
+  const long long start = (long long)grp * T / G;
+  const long long end = (long long)(grp + 1) * T / G;
   if (start < end && start >= excl && start < incl) {
     long long off = excl;
     for (int b = b0; b < b1; ++b) {
@@ -384,7 +360,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
   auto bar = [&](int i) -> uint32_t { return base + kOffBar + 8u * (uint32_t)i; };
   const uint32_t abort_addr = base + kOffAbort;
   long long* work = reinterpret_cast<long long*>(gbase + kOffWork);
-  if (threadIdx.x == 0) PROF_TIME(0);
 
   if (threadIdx.x == 0) {
     // arrival counts: TMA producers and tcgen05.commit arrive once; thread groups one by one
@@ -414,14 +389,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
   }
   // nothing above touched global memory; from here on the previous kernel's results are needed
   grid_dependency_wait();
-  if (warp == 3) plan_range(p.seqlens, p.B, p.max_tiles, pair, npairs, work);
+  if (warp == 3) plan_range(p.seqlens, p.B, p.s_q, p.max_tiles, pair, npairs, work);
   ptx::tc_fence_before();
   __syncthreads();
   // (no early allow_dependents(): the merge that follows would park its blocks on these SMs)
   ptx::cluster_sync();      // the peer's barriers are initialised before any remote arrive
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffTmemSlot);
-  if (threadIdx.x == 0) PROF_TIME(1);
   SegIter segs{work[0], work[1], work[2], (int)work[3]};
   int b, t_lo, t_hi, tiles_b;
   // row-warp geometry (warps 4-11)
@@ -429,6 +403,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
   const int r0 = 32 * qd + 16 * sub + (lane >> 2);                       // and r0 + 8
   const uint32_t s_lane = (uint32_t)(32 * qd + 16 * sub) << 16;          // TMEM lane field of the warp
   const float scale2 = p.sm_scale_log2;
+  // this pair's new token: row block v = b * s_q + tok of the queries and outputs; it sees the
+  // first seqlens[b] - s_q + 1 + tok positions of its sequence
+  const int tok = pair % p.s_q;
+  auto vrow = [&](int bb) -> long long { return (long long)bb * p.s_q + tok; };
+  auto vlen = [&](int bb) -> int { return p.seqlens[bb] - (p.s_q - 1 - tok); };
 
   if (rank == 0) {
     // ============================== score CTA ==============================
@@ -445,7 +424,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             ptx::mbar_arrive_expect_tx(bar(K_FULL + s), kGroupBytes);
             for (int j = 0; j < kGroupChunks; ++j) {
               const int qc = qg * kGroupChunks + j;
-              ptx::tma_load_2d(base + kOffK + s * kGroupBytes + j * kChunkBytes, &tm_q, 64 * (qc >> 1), b * kH + 64 * (qc & 1), bar(K_FULL + s));
+              ptx::tma_load_2d(base + kOffK + s * kGroupBytes + j * kChunkBytes, &tm_q, 64 * (qc >> 1), (int)vrow(b) * kH + 64 * (qc & 1), bar(K_FULL + s));
             }
           }
           for (int t = t_lo; t < t_hi && ok; ++t, ++it) {
@@ -464,7 +443,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             }
           }
         }
-        PROF_TIME(2);
         // loads still in flight must land before the CTA may exit
         const uint32_t ng = gi;
         for (uint32_t k = (ng > (uint32_t)kRing ? ng - kRing : 0); k < ng; ++k)
@@ -475,26 +453,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
         const uint32_t slot_remote0 = ptx::map_to_cta(base + kOffPSlots, 1);
         uint32_t it = 0;
         bool ok = true;
-        PROF_DECL();
         while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
           for (int t = t_lo; t < t_hi; ++t, ++it) {
             const uint32_t stg = it % kStaging, slot = it % kPSlots;
-            PROF_MARK(c0);
             if (!(ok = wait_bar(bar(P_WRITTEN + stg), (it / kStaging) & 1u, abort_addr, false))) break;
-            PROF_ADD(0, c0);
-            PROF_MARK(c1);
             // the slot is free once the output CTA's MMAs of tile it - kPSlots are done
             if (!(ok = wait_bar(bar(P_EMPTY + slot), ((it / kPSlots) & 1u) ^ 1u, abort_addr, true))) break;
-            PROF_ADD(1, c1);
-            PROF_MARK(c2);
             const uint32_t full = ptx::map_to_cta(bar(P_FULL + slot), 1);
             const uint32_t src = base + kOffStaging + stg * kStgStride, dst = slot_remote0 + slot * kSlotStride;
             ptx::mbar_arrive_expect_tx_remote(bar(P_FULL + slot), 1, kCopyBytes);
             ptx::bulk_copy_to_cta(dst, src, kCopyBytes, full);
-            PROF_ADD(2, c2);
           }
         }
-        PROF_SAVE(it);
         // before leaving: every copy has landed and every slot came back
         for (uint32_t k = (it > (uint32_t)kPSlots ? it - kPSlots : 0); k < it; ++k)
           wait_bar(bar(P_EMPTY + k % kPSlots), (k / kPSlots) & 1u, abort_addr, true, false);
@@ -507,30 +477,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
         const uint64_t k_desc = ptx::smem_desc_sw128(base + kOffK, 16, 1024);
         uint32_t it = 0, seg = 0, gq = 0;
         bool ok = true;
-        PROF_DECL();
         while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
-          PROF_MARK(q0);
           if (!(ok = wait_bar(bar(Q_FULL), seg & 1u, abort_addr, false))) break;
-          PROF_ADD(4, q0);
           if (parity == 0)   // every row-warp thread has copied its part of the query out of the ring
             for (int qg = 0; qg < kQGroups; ++qg) ptx::mbar_arrive(bar(K_EMPTY + (gq + qg) % kRing));
           ++seg;
           gq += kQGroups;
           for (int t = t_lo; t < t_hi && ok; ++t, ++it, gq += kGroupsPerTile) {
             if ((it & 1u) != parity) continue;
-            PROF_MARK(c0);
             const uint32_t sb = it % kSBufs;
             const uint32_t g0 = gq;
             if (!(ok = wait_bar(bar(S_EMPTY + sb), ((it / kSBufs) & 1u) ^ 1u, abort_addr, false))) break;
             const uint32_t d = tmem + kSCol0 + 64u * sb;
-            PROF_ADD(0, c0);
 #pragma unroll
             for (int q = 0; q < kGroupsPerTile; ++q) {
               const uint32_t gi = g0 + q, s = gi % kRing;
-              PROF_MARK(c1);
               if (!(ok = wait_bar(bar(K_FULL + s), (gi / kRing) & 1u, abort_addr, false))) break;
-              PROF_ADD(1, c1);
-              PROF_MARK(c2);
               ptx::tc_fence_after();
               const uint64_t gd = k_desc + (uint64_t)(s * (kGroupBytes >> 4));
 #pragma unroll
@@ -542,13 +504,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
                 for (int k = 0; k < 4; ++k) ptx::mma_ts(d, a + 8u * k, bd + 2 * k, kIdescS, (q | j | k) ? 1u : 0u);
               }
               ptx::mma_commit(bar(K_EMPTY + s));
-              PROF_ADD(2, c2);
             }
             if (!ok) break;
             ptx::mma_commit(bar(S_FULL + sb));
           }
         }
-        PROF_SAVE(it);
       }
     } else if (warp >= 4) {
       // ---- row warps: the softmax of their 16 rows
@@ -558,11 +518,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
       const uint32_t stats_remote = ptx::map_to_cta(base + kOffStats, 1);
       uint32_t it = 0, seg = 0, gq = 0;
       bool ok = true;
-      PROF_DECL();
       while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
-        const int L = p.seqlens[b];
-        if (threadIdx.x == 128) PROF_TIME(12);
-        PROF_MARK(q0);
+        const int L = vlen(b);
         // QÌƒ of this sequence into TMEM columns [0, 288), from the 6 ring groups that carry it (the
         // previous segment's S MMAs are done: their last result was read below). Half g fills
         // column blocks [5g, 5 + 4g) of 64 values (32 TMEM columns).
@@ -591,8 +548,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           ptx::tc_fence_before();
           ptx::mbar_arrive(bar(Q_FULL));
         }
-        PROF_ADD(7, q0);
-        if (threadIdx.x == 128) PROF_TIME(13);
         int nb = -1;
         {
           SegIter peek = segs;
@@ -604,38 +559,29 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
         for (int t = t_lo; t < t_hi; ++t, ++it) {
           const uint32_t s = it % kSBufs, stg = it % kStaging;
           if (nb >= 0 && t == max(t_lo, t_hi - 3)) {   // the next segment's query row into L2
-            const char* nq = reinterpret_cast<const char*>(p.q_abs + ((size_t)nb * kH + h) * kRow);
+            const char* nq = reinterpret_cast<const char*>(p.q_abs + ((size_t)vrow(nb) * kH + h) * kRow);
             for (int k = g ? 5 : 0; k < (g ? 9 : 5); ++k) ptx::prefetch_l2(nq + 128 * k);
           }
           // probe this tile's staging buffer now; the answer is used after the arithmetic
           const bool stg_free = ptx::mbar_test_wait_cluster(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u);
-          PROF_MARK(c0);
           if (!wait_bar_warp(bar(S_FULL + s), (it / kSBufs) & 1u, abort_addr, false)) { ok = false; break; }
-          PROF_ADD(0, c0);
-          PROF_MARK(c1);
           uint32_t sr[32];
           ptx::tc_fence_after();
           ptx::tmem_ld_16x256b_x8(tmem + s_lane + kSCol0 + 64u * s, sr);
           ptx::tmem_wait_ld();
           ptx::tc_fence_before();
           ptx::mbar_arrive(bar(S_EMPTY + s));
-          PROF_ADD(1, c1);
-          PROF_MARK(c3);
           uint32_t pk0[8], pk1[8];
           float al0 = 1.f, al1 = 1.f;
           const int valid = L - t * kTile;
           if (valid >= kTile) softmax_rows<false>(sr, kTile, t4, scale2, m0, m1, l0, l1, al0, al1, pk0, pk1);
           else softmax_rows<true>(sr, valid, t4, scale2, m0, m1, l0, l1, al0, al1, pk0, pk1);
-          PROF_ADD(3, c3);
-          PROF_MARK(c4);
           // this tile's staging buffer must have been copied out (tile it - kStaging)
           if (!__all_sync(0xffffffffu, stg_free) &&
               !wait_bar_warp(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u, abort_addr, true)) {
             ok = false;
             break;
           }
-          PROF_ADD(4, c4);
-          PROF_MARK(c5);
           const uint32_t st0 = base + kOffStaging + stg * kStgStride;
           store_p_rows(st0, 32 * qd + 16 * sub, lane, pk0, pk1);
           if (t4 == 0) {
@@ -646,7 +592,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           // visible to the bulk copy (async proxy), then handed to the copier
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(bar(P_WRITTEN + stg));
-          PROF_ADD(5, c5);
         }
         if (!ok) break;
         {
@@ -658,19 +603,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           if (!wait_bar_warp(bar(STATS_EMPTY), (seg & 1u) ^ 1u, abort_addr, true)) { ok = false; break; }
           if (t4 == 0) {
             const bool partial = !(t_lo == 0 && t_hi == tiles_b);
-            float* lse_dst = partial ? p.part_lse + ((size_t)pair * 2 + (seg > 0)) * kH : p.lse + (size_t)b * kH;
+            float* lse_dst = partial ? p.part_lse + ((size_t)pair * 2 + (seg > 0)) * kH : p.lse + (size_t)vrow(b) * kH;
+            // a segment with no visible position (a token's masked last tile alone) has l = 0:
+            // lse -inf and a zero part, which the merge weighs by 0
             lse_dst[r0] = (m0 + log2f(l0)) * 0.69314718055994531f;
             lse_dst[r0 + 8] = (m1 + log2f(l1)) * 0.69314718055994531f;
             const uint32_t st = stats_remote;
-            ptx::st_cluster_f32(st + r0 * 4u, 1.f / l0);
-            ptx::st_cluster_f32(st + (r0 + 8) * 4u, 1.f / l1);
+            ptx::st_cluster_f32(st + r0 * 4u, l0 > 0.f ? 1.f / l0 : 0.f);
+            ptx::st_cluster_f32(st + (r0 + 8) * 4u, l1 > 0.f ? 1.f / l1 : 0.f);
             ptx::mbar_arrive_remote(bar(STATS_FULL), 1);
           }
         }
         ++seg;
       }
-      PROF_SAVE(it);
-      if (threadIdx.x == 128) PROF_TIME(3);
       // before leaving: the output CTA's last release of the stats must have landed here
       if (t4 == 0 && seg > 0) wait_bar(bar(STATS_EMPTY), (seg - 1) & 1u, abort_addr, true, false);
     }
@@ -713,24 +658,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
       const uint64_t p_desc0 = ptx::smem_desc_sw128(base + kOffPSlots, 16, 1024);
       uint32_t it = 0;
       bool ok = true;
-      PROF_DECL();
       while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
-        const int L = p.seqlens[b];
+        const int L = vlen(b);
         for (int t = t_lo; t < t_hi; ++t, ++it) {
           const uint32_t slot = it % kPSlots, s = it % kVStages;
-          PROF_MARK(c0);
           if (!(ok = wait_bar_warp(bar(P_LOCAL + slot), (it / kPSlots) & 1u, abort_addr, false))) break;
-          PROF_ADD(0, c0);
-          PROF_MARK(c2);
           if (!(ok = wait_bar_warp(bar(V_FULL + s), (it / kVStages) & 1u, abort_addr, false))) break;
-          PROF_ADD(1, c2);
-          PROF_MARK(c3);
-          // the last page of a sequence: skip whole 16-row steps past its end and zero the rows of
-          // the last step that lie past it (a pool row there may hold anything, and 0 * NaN = NaN)
+          // a tile past the token's last visible position (the last page of a sequence, or with
+          // several new tokens the one before it): skip whole 16-row steps past the end and zero the
+          // rows of the last step that lie past it (a pool row there may hold anything, and
+          // 0 * NaN = NaN). At least one step runs, so that a segment's first tile always sets O.
           int nk = kTile / 16;
-          if (t == tiles_b - 1) {
-            const int valid = L - t * kTile;
-            nk = (valid + 15) / 16;
+          if (L - t * kTile < kTile) {
+            const int valid = max(0, L - t * kTile);
+            nk = max(1, (valid + 15) / 16);
             const int zr = nk * 16 - valid;
             if (zr > 0) {
               uint8_t* vst = gbase + kOffV + s * kVStageBytes;
@@ -759,11 +700,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             ptx::mma_commit_mc(bar(P_EMPTY + slot), (uint16_t)0x3);
           }
           __syncwarp();
-          PROF_ADD(2, c3);
         }
       }
-      if (lane == 0) PROF_SAVE(it);
-      if (lane == 0) PROF_TIME(4);
     } else if (warp >= 4) {
       // ---- row warps: rescale of the warp's own 16 rows of O before a tile whose P was computed
       // against a larger maximum, and the segment epilogue
@@ -774,19 +712,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
       float* stats = reinterpret_cast<float*>(gbase + kOffStats);
       uint32_t it = 0, seg = 0;
       bool ok = true;
-      PROF_DECL();
       while (segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
         for (int t = t_lo; t < t_hi; ++t, ++it) {
           if (!ok) continue;   // after a failure: skip to the segment end, where all row warps meet
           const uint32_t slot = it % kPSlots;
-          PROF_MARK(c0);
           if (!wait_bar_warp(bar(P_FULL + slot), (it / kPSlots) & 1u, abort_addr, true)) { ok = false; continue; }
-          PROF_ADD(0, c0);
-          PROF_MARK(c1);
           const float* alpha_s = reinterpret_cast<const float*>(gbase + kOffPSlots + slot * kSlotStride + kAlphaOff);
           const float al0 = alpha_s[r0], al1 = alpha_s[r0 + 8];
-          PROF_ADD(1, c1);
-          PROF_MARK(c2);
           // O rows of this warp computed against an older maximum: scale them once the MMAs of the
           // previous tile are done (16x256b: rows r0, r0 + 8, 8 columns per 256-bit chunk). The slot's
           // phase before that one (tile it - 1 - kPSlots) completed before tile it - 1's P_FULL, so the
@@ -811,16 +743,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             }
             ptx::tmem_wait_st();
           }
-          PROF_ADD(2, c2);
           ptx::tc_fence_before();
           ptx::mbar_arrive(bar(P_LOCAL + slot));
         }
         // segment end: O / l out, 1/l from the score CTA
-        if (threadIdx.x == 128) PROF_TIME(8);
         if (ok && !wait_bar_warp(bar(P_EMPTY + (it - 1) % kPSlots), ((it - 1) / kPSlots) & 1u, abort_addr, false)) ok = false;
-        if (threadIdx.x == 128) PROF_TIME(9);
         if (ok && !wait_bar_warp(bar(STATS_FULL), seg & 1u, abort_addr, true)) ok = false;
-        if (threadIdx.x == 128) PROF_TIME(10);
         // every row warp meets here once per segment and agrees whether to go on
         if (ptx::named_bar_or(1, kGroup, !ok)) break;
         ptx::tc_fence_after();
@@ -865,7 +793,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
               flush(reinterpret_cast<char*>(dst + 16 * half), kDC * sizeof(float));
             }
           } else {
-            __nv_bfloat16* dst = p.o_lat + (size_t)b * kH * kDC + col0 + c;
+            __nv_bfloat16* dst = p.o_lat + (size_t)vrow(b) * kH * kDC + col0 + c;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int j = 8 * k;
@@ -878,32 +806,27 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
             flush(reinterpret_cast<char*>(dst), kDC * sizeof(__nv_bfloat16));
           }
         }
-        if (threadIdx.x == 128) PROF_TIME(11);
         // O may be overwritten by the next segment's first MMA once every row warp arrived on its
         // P_LOCAL (after this point, in program order); the score CTA may write the next 1/l values
         ptx::tc_fence_before();
         ptx::mbar_arrive_remote(bar(STATS_EMPTY), 0);
         ++seg;
       }
-      PROF_SAVE(it);
-      if (threadIdx.x == 128) PROF_TIME(5);
     }
   }
 
   // teardown: TMEM back, then leave together so no remote access can target an exited CTA
   ptx::tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) PROF_TIME(6);
   if (warp == 2) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
   ptx::cluster_sync();
-  if (threadIdx.x == 0) PROF_TIME(7);
 }
 
 // ---- merge of split sequences ------------------------------------------------------------------------
-// pair p covers global tiles [p*T/P, (p+1)*T/P); the pair holding tile x is floor(((x+1)*P - 1) / T).
+// group g covers global tiles [g*T/G, (g+1)*T/G); the group holding tile x is floor(((x+1)*G - 1) / T).
 __device__ __forceinline__ int pair_of(long long x, long long T, int P) { return (int)(((x + 1) * P - 1) / T); }
 
 // One warp per (sequence, head), 4 heads per block of 128 threads (about 1.4 waves at 48 registers).
@@ -911,9 +834,12 @@ __device__ __forceinline__ int pair_of(long long x, long long T, int P) { return
 // partial loads before combining them.
 constexpr int kMergeHeads = 4;
 __global__ void __launch_bounds__(32 * kMergeHeads)
-merge_kernel(const int32_t* __restrict__ seqlens, int B, int max_tiles, int npairs, const float* __restrict__ part_o,
+merge_kernel(const int32_t* __restrict__ seqlens, int B, int s_q, int max_tiles, int npairs, const float* __restrict__ part_o,
              const float* __restrict__ part_lse, __nv_bfloat16* __restrict__ o_lat, float* __restrict__ lse) {
-  const int b = blockIdx.x;
+  // block x: new token v = b * s_q + tok of sequence b; its parts come from pair (group, tok) of the
+  // groups that covered the sequence's tiles
+  const int v = blockIdx.x, b = v / s_q, tok = v % s_q;
+  const int G = npairs / s_q;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   grid_dependency_wait();
   allow_dependents();
@@ -935,15 +861,15 @@ merge_kernel(const int32_t* __restrict__ seqlens, int B, int max_tiles, int npai
     max_tb = max(max_tb, __shfl_xor_sync(0xffffffffu, max_tb, o));
   }
   const long long T = local, off = before, tb = tiles_of(__ldg(seqlens + b), max_tiles);
-  if (tb == 0 || T == 0 || whole_sequences(B, npairs, T, max_tb)) return;   // nothing was cut
-  const int p0 = pair_of(off, T, npairs), p1 = pair_of(off + tb - 1, T, npairs);
-  if (p0 == p1) return;                       // written whole by one pair
+  if (tb == 0 || T == 0 || G == 0 || whole_sequences(B, G, T, max_tb)) return;   // nothing was cut
+  const int p0 = pair_of(off, T, G), p1 = pair_of(off + tb - 1, T, G);   // groups
+  if (p0 == p1) return;                       // written whole by one group
   const int h = blockIdx.y * kMergeHeads + warp;
-  // a pair with an empty range wrote nothing; the others' parts in order, lane q holds part p0 + q's lse
+  // a group with an empty range wrote nothing; the others' parts in order, lane q holds group p0 + q's lse
   auto slot = [&](int q) -> int {
-    const long long start_q = (long long)q * T / npairs;
-    if ((long long)(q + 1) * T / npairs <= start_q) return -1;
-    return q * 2 + (start_q < off ? 1 : 0);
+    const long long start_q = (long long)q * T / G;
+    if ((long long)(q + 1) * T / G <= start_q) return -1;
+    return (q * s_q + tok) * 2 + (start_q < off ? 1 : 0);
   };
   float mx = -INFINITY;
   for (int q0 = p0; q0 <= p1; q0 += 32) {
@@ -978,17 +904,20 @@ merge_kernel(const int32_t* __restrict__ seqlens, int B, int max_tiles, int npai
     }
   }
   const float inv = 1.f / tot;
-  uint2* dst = reinterpret_cast<uint2*>(o_lat + ((size_t)b * kH + h) * kDC) + lane;
+  uint2* dst = reinterpret_cast<uint2*>(o_lat + ((size_t)v * kH + h) * kDC) + lane;
 #pragma unroll
   for (int k = 0; k < 4; ++k)
     dst[32 * k] = make_uint2(ptx::pack_bf16x2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
                              ptx::pack_bf16x2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
-  if (lane == 0) lse[(size_t)b * kH + h] = mx + logf(tot);
+  if (lane == 0) lse[(size_t)v * kH + h] = mx + logf(tot);
 }
 
 // ---- host side -----------------------------------------------------------------------------------------
+// s_q new tokens per sequence take s_q pairs each (one token per pair): at most kMaxTokens.
+constexpr int kMaxTokens = 8;
 inline bool decode_supported(const mla_dims_t* d, int32_t dtype, int32_t B, int32_t s_q) {
-  return dtype == MLA_BF16 && d->H == kH && d->d_c == kDC && d->d_r == kDR && s_q == 1 && B >= 1;
+  return dtype == MLA_BF16 && d->H == kH && d->d_c == kDC && d->d_r == kDR && s_q >= 1 && s_q <= kMaxTokens &&
+         B >= 1;
 }
 
 inline int max_pairs(int num_sms) { return num_sms / 2; }
@@ -1025,8 +954,7 @@ inline int active_pairs(int num_sms) {
 inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void* q_abs, const mla_latent_cache_t* cache,
                          const int32_t* block_table, int32_t max_pages, const int32_t* seqlens, void* o_lat, float* lse,
                          void* workspace, size_t ws_bytes, int num_sms, cudaStream_t st) {
-  (void)s_q;
-  if (!workspace || ws_bytes < decode_workspace_bytes(d, MLA_BF16, B, 1, num_sms)) return MLA_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < decode_workspace_bytes(d, MLA_BF16, B, s_q, num_sms)) return MLA_ERR_WORKSPACE;
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1039,9 +967,10 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   const int64_t rows = (int64_t)cache->num_pages * kTile;
   if (!make_tmap(&tm_lat, cache->latent, kDC, rows, cache->latent_stride)) return MLA_ERR_INVALID_ARG;
   if (!make_tmap(&tm_rope, cache->rope, kDR, rows, cache->rope_stride)) return MLA_ERR_INVALID_ARG;
-  CUtensorMap tm_q;   // q_abs as [B*128 heads, 576]: boxes of 64 heads x 64 columns
-  if (!make_tmap(&tm_q, q_abs, kRow, (int64_t)B * kH, kRow)) return MLA_ERR_INVALID_ARG;
+  CUtensorMap tm_q;   // q_abs as [B*s_q*128 heads, 576]: boxes of 64 heads x 64 columns
+  if (!make_tmap(&tm_q, q_abs, kRow, (int64_t)B * s_q * kH, kRow)) return MLA_ERR_INVALID_ARG;
   const int P = active_pairs(num_sms);
+  if (P < s_q) return MLA_ERR_UNSUPPORTED;   // every token of a sequence needs a pair of its own
   Params prm;
   prm.q_abs = reinterpret_cast<const __nv_bfloat16*>(q_abs);
   prm.block_table = block_table;
@@ -1049,6 +978,7 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   prm.num_pages = cache->num_pages;
   prm.seqlens = seqlens;
   prm.B = B;
+  prm.s_q = s_q;
   prm.max_tiles = max_pages;
   prm.o_lat = reinterpret_cast<__nv_bfloat16*>(o_lat);
   prm.lse = lse;
@@ -1056,7 +986,7 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   prm.part_lse = prm.part_o + (size_t)2 * max_pairs(num_sms) * kH * kDC;
   prm.sm_scale_log2 = d->sm_scale * 1.4426950408889634f;
   launch_pdl(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
-  launch_pdl(merge_kernel, dim3(B, kH / kMergeHeads), dim3(32 * kMergeHeads), 0, st, seqlens, (int)B, (int)max_pages, P, (const float*)prm.part_o,
+  launch_pdl(merge_kernel, dim3(B * s_q, kH / kMergeHeads), dim3(32 * kMergeHeads), 0, st, seqlens, (int)B, (int)s_q, (int)max_pages, P, (const float*)prm.part_o,
          (const float*)prm.part_lse, prm.o_lat, lse);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

@@ -60,15 +60,6 @@ struct Params {
 __host__ __device__ constexpr int stage_bytes(int tn) { return kABytes + tn * 128; }
 __host__ __device__ constexpr int smem_bytes(int tn, int stages) { return 1024 + kBarBytes + stages * stage_bytes(tn); }
 
-// Optional phase stamps (profiling builds with -DMLA_DECODE_PROFILE; absent otherwise).
-#ifdef MLA_DECODE_PROFILE
-__device__ unsigned long long g_gemm_time[1024][6];
-#define GEMM_TIME(k) do { const int cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
-    if (cta_ < 1024) g_gemm_time[cta_][k] = ptx::globaltimer(); } while (0)
-#else
-#define GEMM_TIME(k) do {} while (0)
-#endif
-
 __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = 0;
@@ -92,7 +83,6 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) GEMM_TIME(0);
   const int m_tiles = (p.M + kBM - 1) / kBM;
   const bool second = kTwo && (int)blockIdx.x >= p.H * m_tiles;   // a CTA of the second problem
   const int h = second ? 0 : blockIdx.x / m_tiles;
@@ -123,7 +113,6 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
   __syncthreads();
   allow_dependents();
   ptx::tc_fence_after();
-  if (threadIdx.x == 0) GEMM_TIME(1);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + (slot - raw));
 
   if (warp == 0 && lane == 0) {
@@ -196,10 +185,8 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
         }
       }
     }
-    if (threadIdx.x == 128) GEMM_TIME(2);
     const bool ok = __all_sync(0xffffffffu, wait(done, 0));
     ptx::tc_fence_after();
-    if (threadIdx.x == 128) GEMM_TIME(3);
     if (ok) {
       for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
         uint32_t r[32];
@@ -222,14 +209,12 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
       }
     }
   }
-  if (threadIdx.x == 128) GEMM_TIME(4);
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 2) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, tmem_cols);
   }
-  if (threadIdx.x == 0) GEMM_TIME(5);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)

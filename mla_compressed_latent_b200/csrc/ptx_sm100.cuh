@@ -145,13 +145,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// 2^a, 2^b by one f16x2 SFU operation (arguments rounded to f16); results widened back to f32.
-__device__ __forceinline__ void ex2_half2(float a, float b, float& ea, float& eb) {
-  uint32_t h;
-  asm("{\n\t.reg .b32 x;\n\tcvt.rn.f16x2.f32 x, %2, %1;\n\tex2.approx.f16x2 %0, x;\n\t}" : "=r"(h) : "f"(a), "f"(b));
-  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-      : "=f"(ea), "=f"(eb) : "r"(h));
-}
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }

@@ -69,6 +69,16 @@ SMALL_DECODE = [
     ([131072], 1, "random"),
     (list(np.random.default_rng(11).integers(1, 2000, 200)), 1, "random"),
     ([64 * 70] * 3 + [64 * 5 + 1], 1, "contiguous"),
+    # several new tokens (one worker pair per token, the pairs of a sequence walking its tiles
+    # together): a token whose visible positions end on a page boundary sees its sequence's last
+    # page fully masked; with s_q = 4 the mask reaches into the page before; odd s_q leaves pairs
+    # idle; one long sequence cut between every group; many short ones per group
+    ([65, 129, 64 * 5 + 1, 2], 2, "random"),
+    ([65, 66, 4, 64 * 3 + 2, 64 * 3 + 3], 4, "random"),
+    ([100, 5000, 3, 64 * 40 + 1], 3, "contiguous"),
+    ([8, 70, 64 * 20 + 3], 8, "random"),
+    ([131072], 2, "random"),
+    (list(np.random.default_rng(12).integers(4, 3000, 150)), 4, "random"),
 ]
 
 
@@ -144,9 +154,10 @@ def test_decode_absorbed_full_size(name):
         _assert_lse(gl, ref_l[b], "bf16", f"lse seq {b}")
 
 
-def test_decode_mtp_random_pages_full_size_sampled():
+@pytest.mark.parametrize("name", ["mtp_sq2_b128", "mtp_sq4_b128"])
+def test_decode_mtp_random_pages_full_size_sampled(name):
     """Multi-token step, random page table, full batch; oracle on a seeded sample of sequences."""
-    w = synth.workload("mtp_sq2_b128")
+    w = synth.workload(name)
     case = Case(w, with_weights=False)
     dev = case.to_device()
     o_lat, lse = ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"])
