@@ -30,6 +30,8 @@ sys.path.insert(0, ROOT)
 METRIC = "MLA decode cache-positions/s and tokens/s; % of B200 roofline (HBM or TC)"
 UNIT = "positions/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal B200 figures (context for the measured fractions): HBM3e ~8 TB/s, dense bf16 2.25 PFLOP/s
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
 def parse():
@@ -41,6 +43,7 @@ def parse():
     p.add_argument("--workload", default="dsv3_b64_l4096")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="bound on the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-secondary", action="store_true", help="skip the other configurations' decode timings")
     return p.parse_args()
 
 
@@ -297,14 +300,24 @@ def build_inputs(w, device):
         p = np.arange(L)
         idx[off:off + L] = table[b, p // 64].astype(np.int64) * 64 + p % 64
         off += L
-    for start, c, kr in synth.cache_row_chunks(w, total):
-        n = len(c)
-        rows = torch.from_numpy(np.concatenate([c, kr], axis=1)).to(device=device, dtype=tdt)
-        pool[torch.from_numpy(idx[start:start + n]).to(device)] = rows
     W = synth.weights(w)
     step = synth.decode_step_inputs(w)
+    from_hidden = w.dtype == "bf16" and w.lengths[0] == "fixed" and w.lengths[1] % 64 == 0
+    if from_hidden:
+        # the configured recipe: every cached row is c = RMSNorm(x·W_DKV), k_r = RoPE(x·W_KR) of hidden
+        # states x ~ N(0, 1), written by the library's own cache append, 64 positions of every
+        # sequence per call (x drawn on the GPU by torch's CUDA generator)
+        fill_cache_from_hidden_states(w, pool, num_pages, table, lens, W, device)
+    else:
+        for start, c, kr in synth.cache_row_chunks(w, total):
+            n = len(c)
+            rows = torch.from_numpy(np.concatenate([c, kr], axis=1)).to(device=device, dtype=tdt)
+            pool[torch.from_numpy(idx[start:start + n]).to(device)] = rows
     dev = {
         "pool": pool, "num_pages": num_pages, "lens": lens,
+        "cache_recipe": ("rows written by mla_append_cache from hidden states x ~ N(0,1): c = RMSNorm(x W_DKV), "
+                         "k_r = RoPE(x W_KR)") if from_hidden else
+                        "latent rows uniform on the sphere of radius sqrt(d_c), RoPE keys N(0,1)",
         "seqlens": torch.from_numpy(lens).to(device), "table": torch.from_numpy(table).to(device),
         "w_dkv_kr": torch.from_numpy(np.concatenate([W["W_DKV"], W["W_KR"]], 1)).to(device=device, dtype=tdt),
         "W_UK": torch.from_numpy(W["W_UK"]).to(device=device, dtype=tdt),
@@ -320,6 +333,225 @@ def build_inputs(w, device):
     dev["q_nope"] = dev["q_nope_host"].to(device)
     dev["q_rope_raw"] = dev["q_rope_host"].to(device)
     return dev
+
+
+# configurations whose decode call the default run also times on its own: long-context split-KV,
+# the GQLA grouped path, multi-token steps with 2 and 4 new tokens
+SECONDARY = ("longctx_b8", "gqla_g8_b32_l8192", "mtp_sq2_b128", "mtp_sq4_b128")
+
+
+def run_e2e(args, w, dev, step, out, stream, device, world, from_x, e_steps):
+    """End-to-end steps through the public API with host buffers: returns ({ms, h2d, d2h}, graph_ok)."""
+    import torch
+    import torch.distributed as dist
+    x_host, qn_host, qr_host = dev["x_host"], dev["q_nope_host"], dev["q_rope_host"]
+    ins = [(torch.empty_like(x_host, device=device), torch.empty_like(qn_host, device=device),
+            torch.empty_like(qr_host, device=device)) for _ in range(2)]
+    outs = [torch.empty_like(out) for _ in range(2)]
+    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    for k in range(2):
+        ins[k][0].copy_(x_host)
+        ins[k][1].copy_(qn_host)
+        ins[k][2].copy_(qr_host)
+
+    def body(k):
+        xi, qn, qr = ins[k]
+        step(xi, None if from_x else qn, None if from_x else qr, out_t=outs[k])
+
+    graphs, graph_ok = [], True
+    try:
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for k in range(2):
+                body(k)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        for k in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                body(k)
+            graphs.append(g)
+        torch.cuda.synchronize()
+    except Exception:  # noqa: BLE001  (capture unavailable: the same calls, launched directly)
+        graphs, graph_ok = [], False
+        torch.cuda.synchronize()
+
+    def device_step(k):
+        if graph_ok:
+            graphs[k].replay()
+        else:
+            body(k)
+
+    h2d_s, d2h_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("in_ready", "done", "out_free")}
+    for k in range(2):   # every event recorded once, so the first waits return at once
+        for n in ev:
+            ev[n][k].record(stream)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e_steps):
+        k = i % 2
+        h2d_s.wait_event(ev["done"][k])            # step i-2 has finished reading these inputs
+        with torch.cuda.stream(h2d_s):
+            ins[k][0].copy_(x_host, non_blocking=True)
+            if not from_x:
+                ins[k][1].copy_(qn_host, non_blocking=True)
+                ins[k][2].copy_(qr_host, non_blocking=True)
+        ev["in_ready"][k].record(h2d_s)
+        stream.wait_event(ev["in_ready"][k])
+        stream.wait_event(ev["out_free"][k])       # step i-2's result has left this buffer
+        device_step(k)
+        ev["done"][k].record(stream)
+        d2h_s.wait_event(ev["done"][k])
+        with torch.cuda.stream(d2h_s):
+            out_host[k].copy_(outs[k], non_blocking=True)
+        ev["out_free"][k].record(d2h_s)
+    for k in range(2):
+        stream.wait_event(ev["out_free"][k])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    h2d = x_host.numel() * x_host.element_size()
+    if not from_x:
+        h2d += qn_host.numel() * qn_host.element_size() + qr_host.numel() * qr_host.element_size()
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    del graphs
+    return {"ms": ms, "h2d": h2d, "d2h": d2h}, graph_ok
+
+
+def gpu_latent_pool(w, num_pages, device, seed=2):
+    """A paged latent pool drawn on the GPU with the recipe of synth.cache_row_chunks: latent rows
+    uniform on the sphere of radius sqrt(d_c), RoPE keys N(0, 1) (drawn by torch's CUDA generator,
+    in chunks, so that large pools need no host work)."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    rows = num_pages * 64
+    pool = torch.empty(rows, w.d_c + w.d_r, dtype=torch.bfloat16, device=device)
+    step = 1 << 20
+    for r0 in range(0, rows, step):
+        n = min(step, rows - r0)
+        g = torch.randn(n, w.d_c, generator=gen, device=device)
+        pool[r0:r0 + n, :w.d_c] = g * (math.sqrt(w.d_c) / g.norm(dim=1, keepdim=True))
+        pool[r0:r0 + n, w.d_c:] = torch.randn(n, w.d_r, generator=gen, device=device)
+    return pool
+
+
+def time_decode_alone(name, device, steps, warmup, peaks):
+    """The decode call of one workload on its own (absorbed, or grouped for a GQLA workload), timed
+    with CUDA events around each call on the launching stream; returns its line fragment."""
+    import numpy as np
+    import torch
+    import synth
+    from mla_compressed_latent_b200 import ops
+    from mla_compressed_latent_b200.ops import Dims, LatentCache, GqaCache
+    w = synth.workload(name)
+    dims = Dims.of(w)
+    lens = synth.seq_lengths(w)
+    table, num_pages = synth.block_table(w, lens)
+    tbl = torch.from_numpy(table).to(device)
+    seqlens = torch.from_numpy(lens).to(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1)
+    stream = torch.cuda.current_stream()
+    total = int(lens.sum())
+    n_tok = w.B * w.s_q
+    if w.g:
+        rows = num_pages * 64
+        K = torch.randn(rows, w.g, w.D, generator=gen, device=device).to(torch.bfloat16)
+        V = torch.randn(rows, w.g, w.d_v, generator=gen, device=device).to(torch.bfloat16)
+        R = torch.randn(rows, w.d_r, generator=gen, device=device).to(torch.bfloat16)
+        qn = torch.randn(w.B, w.s_q, w.H, w.D, generator=gen, device=device).to(torch.bfloat16)
+        qr = torch.randn(w.B, w.s_q, w.H, w.d_r, generator=gen, device=device).to(torch.bfloat16)
+        cache = GqaCache(K, V, R, num_pages)
+        out = torch.empty(w.B, w.s_q, w.H, w.d_v, dtype=torch.bfloat16, device=device)
+        lse = torch.empty(w.B, w.s_q, w.H, dtype=torch.float32, device=device)
+        import ctypes
+        from mla_compressed_latent_b200 import _lib as L
+        dc = dims.c()
+        ws = torch.empty(max(16, int(L.load().mla_gqla_workspace_size(ctypes.byref(dc), L.MLA_BF16, w.B, w.s_q,
+                                                                      table.shape[1]))),
+                         dtype=torch.uint8, device=device)
+
+        def call():
+            ops.mla_decode_gqla_grouped(dims, qn, qr, cache, tbl, seqlens, out=out, lse=lse, workspace=ws)
+        bytes_ = total * (w.g * (w.D + w.d_v) + w.d_r) * 2 + n_tok * w.H * (w.D + w.d_r + w.d_v) * 2 + n_tok * w.H * 4
+        flops = total * w.H * 2 * ((w.D + w.d_r) + w.d_v)
+        kernel = "mla_decode_gqla_grouped (decode + split merge)"
+    else:
+        pool = gpu_latent_pool(w, num_pages, device)
+        cache = LatentCache(pool[:, :w.d_c], pool[:, w.d_c:], num_pages)
+        q_abs = torch.randn(w.B, w.s_q, w.H, w.d_c + w.d_r, generator=gen, device=device)
+        q_abs[..., :w.d_c] *= math.sqrt(w.D / w.d_c)
+        q_abs = q_abs.to(torch.bfloat16)
+        o_lat = torch.empty(w.B, w.s_q, w.H, w.d_c, dtype=torch.bfloat16, device=device)
+        lse = torch.empty(w.B, w.s_q, w.H, dtype=torch.float32, device=device)
+        ws = torch.empty(max(16, ops.mla_decode_workspace_size(dims, torch.bfloat16, w.B, w.s_q, table.shape[1])),
+                         dtype=torch.uint8, device=device)
+
+        def call():
+            ops.mla_decode_absorbed(dims, q_abs, cache, tbl, seqlens, o_lat=o_lat, lse=lse, workspace=ws)
+        bytes_, flops, _ = decode_counts(w, lens)
+        kernel = "mla_decode_absorbed (decode + split merge)"
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    rc = ops.mla_check_status()
+    if rc != 0:
+        raise RuntimeError(f"{name}: device status {ops.mla_status_string(rc)}")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    sec = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+    gbs, tfs = bytes_ / sec / 1e9, flops / sec / 1e12
+    t_hbm, t_tc = bytes_ / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)
+    if t_tc > t_hbm:
+        roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tfs / peaks["bf16_tflops"],
+                "frac_sustained": tfs / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "frac_nominal": tfs / NOMINAL_PEAKS["bf16_tflops"], "hbm_gbs": gbs}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"], "frac_nominal": gbs / NOMINAL_PEAKS["hbm_gbs"], "tensor_tflops": tfs}
+    roof.update({"traffic": None, "kernel": kernel, "bytes_per_launch": bytes_, "flops_per_launch": flops})
+    del cache
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return {"decode_us": sec * 1e6, "positions_per_s": total / sec, "tokens_per_s": n_tok / sec,
+            "config": {"B": w.B, "s_q": w.s_q, "lengths": list(w.lengths), "pages": w.pages, "g": w.g,
+                       "positions": total},
+            "roofline": roof, "steps": steps, "inputs": "drawn on the GPU (torch CUDA generator), synth recipe"}
+
+
+def fill_cache_from_hidden_states(w, pool, num_pages, table, lens, W, device, seed=2):
+    """Fill every sequence's cached rows through mla_append_cache from x ~ N(0, 1) (all sequences
+    the same length, a multiple of 64): call k appends positions 64k .. 64k+63 of every sequence."""
+    import numpy as np
+    import torch
+    from mla_compressed_latent_b200 import ops
+    from mla_compressed_latent_b200.ops import Dims, LatentCache
+    dims = Dims.of(w)
+    cache = LatentCache(pool[:, :w.d_c], pool[:, w.d_c:], num_pages)
+    wcat = torch.from_numpy(np.concatenate([W["W_DKV"], W["W_KR"]], 1)).to(device=device, dtype=torch.bfloat16)
+    tbl = torch.from_numpy(table).to(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    L = int(lens[0])
+    for k in range(L // 64):
+        x = torch.randn(w.B, 64, w.C, generator=gen, device=device).to(torch.bfloat16)
+        sl = torch.full((w.B,), 64 * (k + 1), dtype=torch.int32, device=device)
+        ops.mla_append_cache(dims, x, wcat, None, sl, tbl, cache)
+    torch.cuda.synchronize()
+    rc = ops.mla_check_status()
+    if rc != 0:
+        raise RuntimeError(f"cache fill: device status {ops.mla_status_string(rc)}")
 
 
 def run_grouped(args, w, dims, device, world, rank, local):
@@ -453,7 +685,7 @@ def main():
         ws_q = torch.empty(max(16, L.load().mla_query_workspace_size(ctypes.byref(dc), w.B, w.s_q, w.C, w.d_q)),
                            dtype=torch.uint8, device=device)
 
-    def step(x, q_nope, q_rope, events=None):
+    def step(x, q_nope, q_rope, events=None, out_t=None):
         """One decode step. events: None; "decode" (two events around the decode call, which is all
         the timed region carries, so the other kernels keep overlapping their launches); or "all"
         (an event after every call, for the per-call breakdown outside the timed region)."""
@@ -481,7 +713,7 @@ def main():
         ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"], o_lat=o_lat, lse=lse, workspace=ws_dec)
         if events:
             mark("decode")
-        ops.mla_out_proj(dims, o_lat, dev["W_UV"], out=out)
+        ops.mla_out_proj(dims, o_lat, dev["W_UV"], out=out if out_t is None else out_t)
         if every:
             mark("out_proj")
         if events:
@@ -533,29 +765,12 @@ def main():
     breakdown = {c: statistics.mean(between(m, order[i], c) for m in dec_ev) * 1e3 for i, c in enumerate(calls)}
     assert ops.mla_check_status() == 0
 
-    # end to end through the public API: pinned host inputs in, host result out, every step
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # end to end through the public API: pinned host inputs in, host result out, every step. The
+    # device part of a step is one CUDA graph replay (its library calls captured once per buffer
+    # set); step i's inputs are copied in on one stream and step i-1's result copied out on another
+    # while step i runs on the compute stream (double-buffered device inputs and outputs).
     e_steps = max(3, min(args.steps, 200))
-    e0.record(stream)
-    for _ in range(e_steps):
-        x = dev["x_host"].to(device, non_blocking=True)
-        qn = qr = None
-        if not from_x:
-            qn = dev["q_nope_host"].to(device, non_blocking=True)
-            qr = dev["q_rope_host"].to(device, non_blocking=True)
-        step(x, qn, qr)
-        out_host.copy_(out, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-    h2d = sum(t.numel() * t.element_size()
-              for t in ((dev["x_host"],) if from_x else (dev["x_host"], dev["q_nope_host"], dev["q_rope_host"])))
-    d2h = out_host.numel() * out_host.element_size()
-
+    e2e, graph_ok = run_e2e(args, w, dev, step, out, stream, device, world, from_x, e_steps)
     bytes_, flops, positions = decode_counts(w, dev["lens"])
     peaks, peak_kind = load_peaks()
     step_s = ms / 1e3 / args.steps
@@ -569,19 +784,23 @@ def main():
         "config": {"workload": w.name, "B": w.B, "seq_len": w.lengths[1] if w.lengths[0] == "fixed" else list(w.lengths),
                    "H": w.H, "D": w.D, "d_c": w.d_c, "d_r": w.d_r, "d_v": w.d_v, "s_q": w.s_q,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"inputs larger than L2: {positions * (w.d_c + w.d_r) * (2 if w.dtype == 'bf16' else 4) / 1e6:.0f} MB cache read per step"},
+                   "l2": f"inputs larger than L2: {positions * (w.d_c + w.d_r) * (2 if w.dtype == 'bf16' else 4) / 1e6:.0f} MB cache read per step",
+                   "cache": dev["cache_recipe"]},
         "tokens_per_s": world * n_tok / step_s,
         "decode_us": dec_ms * 1e3,
         "step_breakdown_us": breakdown,
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": captured_traffic(w.name), "peak_source": peak_kind,
+                     "frac": achieved_gbs / peaks["hbm_gbs"], "frac_nominal": achieved_gbs / NOMINAL_PEAKS["hbm_gbs"],
+                     "peak_nominal": NOMINAL_PEAKS["hbm_gbs"], "traffic": captured_traffic(w.name), "peak_source": peak_kind,
                      "kernel": "mla_decode_absorbed (decode + split merge)",
                      "tensor_tflops": achieved_tf, "tensor_frac": achieved_tf / peaks["bf16_tflops"],
                      "bound_frac": max(bytes_ / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) / (dec_ms / 1e3)},
         "gpu_launches": int(launches),
         "clocks": {**clk.summary(), "remeasured": remeasured},
-        "e2e": {"value": world * positions / (e_ms / 1e3 / e_steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e_steps},
+        "e2e": {"value": world * positions / (e2e["ms"] / 1e3 / e_steps), "unit": UNIT,
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "steps": e_steps,
+                "ms_per_step": e2e["ms"] / e_steps, "cuda_graph": graph_ok,
+                "overlap": "inputs copied in and outputs copied out on their own streams, double-buffered"},
     }
     if from_x:
         # the query chain is bound by its weights: W_DQ, W_UQ, W_QR read once per step
@@ -591,6 +810,12 @@ def main():
         line["query_chain"] = {"us": q_us, "bytes": q_bytes, "achieved_gbs": q_bytes / (q_us / 1e6) / 1e9,
                                "frac": q_bytes / (q_us / 1e6) / 1e9 / peaks["hbm_gbs"],
                                "note": "timed with an event after every call (no launch overlap)"}
+    if world == 1 and not args.no_secondary:
+        # the other configurations' decode calls, each timed on its own (a few seconds in all)
+        line["secondary"] = {}
+        for name in SECONDARY:
+            if name != w.name:
+                line["secondary"][name] = time_decode_alone(name, device, max(5, min(args.steps, 20)), 3, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         pos, tok, el, seqs = oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": pos / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",

@@ -181,7 +181,8 @@ int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_
  * a5. Output projection (« Ce que DeepSeek fait de plus »: the weighted latent sum is projected
  * once by W_UV; « Le code »: the layer's final projection).
  *   out[b,t,h,:] = o_lat[b,t,h,:] · W_UV[h]                   (W_UV[h] is [d_c, d_v])
- *   if w_o != NULL: out_model[b,t,:] = concat_h(out[b,t,h,:]) · W_O   (W_O is [H*d_v, C])
+ *   if w_o != NULL: out_model[b,t,:] = concat_h(out[b,t,h,:]) · W_O   (W_O is [H*d_v, C]; in bf16 with
+ *   H*d_v a multiple of 64 and C of 8 this second product runs on the tensor cores too)
  *   o_lat [B, s_q, H, d_c]  w_uv [H, d_c, d_v]  out [B, s_q, H, d_v]  out_model [B, s_q, C] (dtype)
  * ------------------------------------------------------------------------------------------- */
 int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
@@ -204,6 +205,40 @@ int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, in
                             const void* q_nope, const void* q_rope_raw, const mla_gqa_cache_t* cache,
                             const int32_t* block_table, int32_t max_pages, const int32_t* seqlens,
                             void* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * f3. Append to the expanded GQA cache of the grouped path (« Résumé technique : GQLA … »,
+ * « Chemin GQA »: the latent is expanded into g key/value groups once, when the cache is written).
+ * For each new token (b, t) at position seqlens[b] - s_q + t:
+ *   c   = RMSNorm(x[b,t,:] · W_DKV) · gamma            (rounded to dtype, as a latent cache row is)
+ *   k_r = RoPE(x[b,t,:] · W_KR, position)             -> cache->rope row
+ *   K[g] = W_UK[g] · c   (W_UK [g, D, d_c])           -> cache->k row [g, D]
+ *   V[g] = c · W_UV[g]   (W_UV [g, d_c, d_v])         -> cache->v row [g, d_v]
+ *   x [B, s_q, C]   w_dkv_kr [C, d_c + d_r]   gamma [d_c] or NULL   (all dtype)
+ * Only MLA_BF16 with C and d_c multiples of 64 and D, d_v multiples of 8 (else MLA_ERR_UNSUPPORTED).
+ * workspace: at least mla_gqa_append_workspace_size(...) bytes (fp32 partial sums, then c, K and V of
+ * the new tokens); contents need not be initialised. The call enqueues five kernels.
+ * ------------------------------------------------------------------------------------------- */
+size_t mla_gqa_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C);
+int mla_append_gqa_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x, int32_t C,
+                         const void* w_dkv_kr, const void* gamma, const void* w_uk_g, const void* w_uv_g,
+                         const int32_t* seqlens, const int32_t* block_table, int32_t max_pages,
+                         const mla_gqa_cache_t* cache, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * f3. The value up-projection absorbed into the output projection (« Résumé technique : GQLA … »,
+ * « Chemin MQA-Absorbé »: the up-projections are absorbed into the query and output projections).
+ * mla_preabsorb_out_weights builds, once per layer, W_UVO[h] = W_UV[h] · W_O[h*d_v : (h+1)*d_v, :]:
+ *   w_uv [H, d_c, d_v]   w_o [H*d_v, C]   ->   w_uvo [H, d_c, C]   (all dtype; H GEMMs enqueued)
+ * mla_out_proj_preabsorbed then computes the layer output straight from the weighted latents:
+ *   out_model[b,t,:] = concat_h(o_lat[b,t,h,:]) · W_UVO     (o_lat [B, s_q, H, d_c], w_uvo as above)
+ * which equals mla_out_proj with w_o up to rounding. Note the weight is H*d_c x C: it pays off only
+ * when d_c * H * C is small against the two projections it replaces.
+ * ------------------------------------------------------------------------------------------- */
+int mla_preabsorb_out_weights(const mla_dims_t* dims, int32_t dtype, const void* w_uv, const void* w_o, int32_t C,
+                              void* w_uvo, void* stream);
+int mla_out_proj_preabsorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* o_lat,
+                             const void* w_uvo, int32_t C, void* out_model, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Status.

@@ -59,6 +59,12 @@ SIGNATURES = {
     "mla_decode_gqla_grouped": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_void_p,
                                           POINTER(MlaGqaCache), PI, c_int32, PI, c_void_p, c_void_p, c_void_p,
                                           c_size_t, c_void_p]),
+    "mla_gqa_append_workspace_size": (c_size_t, [PD, c_int32, c_int32, c_int32]),
+    "mla_append_gqa_cache": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_int32, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, PI, PI, c_int32, POINTER(MlaGqaCache), c_void_p, c_size_t, c_void_p]),
+    "mla_preabsorb_out_weights": (c_int32, [PD, c_int32, c_void_p, c_void_p, c_int32, c_void_p, c_void_p]),
+    "mla_out_proj_preabsorbed": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_int32, c_void_p,
+                                           c_void_p]),
     "mla_check_status": (c_int32, [c_void_p]),
     "mla_status_string": (c_char_p, [c_int32]),
     "mla_build_info": (c_char_p, []),

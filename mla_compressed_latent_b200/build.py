@@ -12,6 +12,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmla.so")
+# the same sources with test hooks compiled in (a switch that stalls a kernel's bounded wait on
+# purpose); loaded only by the tests of the wait-expiry path
+TEST_LIB = os.path.join(PKG, "libmla_testhooks.so")
 
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",
@@ -33,19 +36,24 @@ def sources():
                   glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
-    """Compile csrc/mla_api.cu (which includes every kernel) into libmla.so; return its path."""
-    if not force and up_to_date():
-        return LIB
+def build_test_hooks(force: bool = False, verbose: bool = False) -> str:
+    """Compile the test-hooks variant of the library (-DMLA_TEST_HOOKS) into libmla_testhooks.so."""
+    return build(force, verbose, ["-DMLA_TEST_HOOKS"], TEST_LIB)
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags=None, lib: str = LIB) -> str:
+    """Compile csrc/mla_api.cu (which includes every kernel) into `lib` (libmla.so); return its path."""
+    if not force and up_to_date(lib):
+        return lib
     cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC,
-           "-o", LIB + ".tmp", os.path.join(CSRC, "mla_api.cu")]
+           "-o", lib + ".tmp", os.path.join(CSRC, "mla_api.cu")]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -53,8 +61,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose and (res.stdout or res.stderr):
         print(res.stdout, res.stderr, file=sys.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -124,45 +124,15 @@ struct Params {
 };
 
 // One tile of the online softmax for rows r0 and r0 + 8 of a thread (register layout of the 16x256b
-// shape, see above): the rows' maxima over the tile's valid columns (the 4 threads of a row meet by
-// shuffles), the lazy update of the running maxima m (rescale factors al, 1 when m did not move), and
-// the exponentials packed as bf16 pairs (pk0 row r0, pk1 row r1; column block j) with their sums in l.
-// kMask: the tile has fewer than 64 valid columns (the last page of a sequence).
+// shape, see above): the exponentials packed as bf16 pairs (pk0 row r0, pk1 row r1; column block j)
+// with their sums added to l, and the lazy update of the running maxima m (rescale factors al, 1 when
+// m did not move). The running maximum moves only when the tile's exceeds it by 2^kRescaleLog2, so
+// the exponentials are first taken against the current m, alongside the tile's maxima (the 4 threads
+// of a row meet by shuffles); only a tile that moves a maximum (the first of a segment, then rarely)
+// takes them again. kMask: the tile has fewer than 64 visible columns.
 template <bool kMask>
-__device__ __forceinline__ void softmax_rows(const uint32_t (&sr)[32], int valid, int t4, float scale2, float& m0,
-                                             float& m1, float& l0, float& l1, float& al0, float& al1,
-                                             uint32_t (&pk0)[8], uint32_t (&pk1)[8]) {
-  float a0 = -INFINITY, a1 = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int c = 8 * j + 2 * t4;
-    if (!kMask || c < valid) {
-      a0 = fmaxf(a0, __uint_as_float(sr[4 * j]));
-      a1 = fmaxf(a1, __uint_as_float(sr[4 * j + 2]));
-    }
-    if (!kMask || c + 1 < valid) {
-      a0 = fmaxf(a0, __uint_as_float(sr[4 * j + 1]));
-      a1 = fmaxf(a1, __uint_as_float(sr[4 * j + 3]));
-    }
-  }
-  a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
-  a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
-  a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 2));
-  a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
-  // lazy rescale: the running maximum moves only when the tile's exceeds it by 2^kRescaleLog2
-  al0 = 1.f;
-  al1 = 1.f;
-  const float mt0 = a0 * scale2, mt1 = a1 * scale2;
-  if (mt0 > m0 + kRescaleLog2) {
-    al0 = (m0 == -INFINITY) ? 0.f : ptx::ex2_approx(m0 - mt0);
-    l0 *= al0;
-    m0 = mt0;
-  }
-  if (mt1 > m1 + kRescaleLog2) {
-    al1 = (m1 == -INFINITY) ? 0.f : ptx::ex2_approx(m1 - mt1);
-    l1 *= al1;
-    m1 = mt1;
-  }
+__device__ __forceinline__ void exps_rows(const uint32_t (&sr)[32], int valid, int t4, float scale2, float m0,
+                                          float m1, float& ls_0, float& ls_1, uint32_t (&pk0)[8], uint32_t (&pk1)[8]) {
   float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -181,8 +151,52 @@ __device__ __forceinline__ void softmax_rows(const uint32_t (&sr)[32], int valid
     pk0[j] = ptx::pack_bf16x2(e00, e01);
     pk1[j] = ptx::pack_bf16x2(e10, e11);
   }
-  l0 += ls0 + ls1;
-  l1 += ls2 + ls3;
+  ls_0 = ls0 + ls1;
+  ls_1 = ls2 + ls3;
+}
+
+template <bool kMask>
+__device__ __forceinline__ void softmax_rows(const uint32_t (&sr)[32], int valid, int t4, float scale2, float& m0,
+                                             float& m1, float& l0, float& l1, float& al0, float& al1,
+                                             uint32_t (&pk0)[8], uint32_t (&pk1)[8]) {
+  float ls0, ls1;
+  exps_rows<kMask>(sr, valid, t4, scale2, m0, m1, ls0, ls1, pk0, pk1);
+  float a0 = -INFINITY, a1 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int c = 8 * j + 2 * t4;
+    if (!kMask || c < valid) {
+      a0 = fmaxf(a0, __uint_as_float(sr[4 * j]));
+      a1 = fmaxf(a1, __uint_as_float(sr[4 * j + 2]));
+    }
+    if (!kMask || c + 1 < valid) {
+      a0 = fmaxf(a0, __uint_as_float(sr[4 * j + 1]));
+      a1 = fmaxf(a1, __uint_as_float(sr[4 * j + 3]));
+    }
+  }
+  a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
+  a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+  a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 2));
+  a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
+  al0 = 1.f;
+  al1 = 1.f;
+  const float mt0 = a0 * scale2, mt1 = a1 * scale2;
+  const bool up0 = mt0 > m0 + kRescaleLog2, up1 = mt1 > m1 + kRescaleLog2;
+  if (__any_sync(0xffffffffu, up0 || up1)) {
+    if (up0) {
+      al0 = (m0 == -INFINITY) ? 0.f : ptx::ex2_approx(m0 - mt0);
+      l0 *= al0;
+      m0 = mt0;
+    }
+    if (up1) {
+      al1 = (m1 == -INFINITY) ? 0.f : ptx::ex2_approx(m1 - mt1);
+      l1 *= al1;
+      m1 = mt1;
+    }
+    exps_rows<kMask>(sr, valid, t4, scale2, m0, m1, ls0, ls1, pk0, pk1);
+  }
+  l0 += ls0;
+  l1 += ls1;
 }
 
 // A warp's P rows into a P tile at `ptile` (K-major, 128-byte swizzle: row r at (r / 8) * 1024 +
@@ -339,8 +353,8 @@ __device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, uin
 }
 
 // ---- the kernel ------------------------------------------------------------------------------------
-// Warp roles.  Score CTA: 0 TMA producer | 1 S-MMA issuer for even tiles, and lane 0 of warp 2 for odd
-// tiles (one issuing thread cannot keep the tensor core busy at N = 64) | 2 TMEM | 3 copier (one bulk
+// Warp roles.  Score CTA: 0 TMA producer | 1 S-MMA issuer for even tiles, warp 2 for odd tiles (each
+// warp waits as a whole and one elected lane issues) | 2 TMEM | 3 copier (one bulk
 // copy per tile into the output CTA) | 4-11 row warps: softmax of their 16 rows each; all of them
 // copy Q̃ into TMEM at a segment start.
 // Output CTA: 0 TMA producer | 1 O-MMA issuer | 2 TMEM, then receiver (returns the score CTA's
@@ -472,27 +486,30 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           wait_bar(bar(STG_FREE + k % kStaging), (k / kStaging) & 1u, abort_addr, true, false);
       }
     } else if (warp == 1 || warp == 2) {
-      if (lane == 0) {   // ---- S-MMA issuers: S = Q̃ · [c ; k_r]ᵀ, K = 576 in 36 steps of 16
-        const uint32_t parity = warp == 1 ? 0u : 1u;
-        const uint64_t k_desc = ptx::smem_desc_sw128(base + kOffK, 16, 1024);
-        uint32_t it = 0, seg = 0, gq = 0;
-        bool ok = true;
-        while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
-          if (!(ok = wait_bar(bar(Q_FULL), seg & 1u, abort_addr, false))) break;
-          if (parity == 0)   // every row-warp thread has copied its part of the query out of the ring
-            for (int qg = 0; qg < kQGroups; ++qg) ptx::mbar_arrive(bar(K_EMPTY + (gq + qg) % kRing));
-          ++seg;
-          gq += kQGroups;
-          for (int t = t_lo; t < t_hi && ok; ++t, ++it, gq += kGroupsPerTile) {
-            if ((it & 1u) != parity) continue;
-            const uint32_t sb = it % kSBufs;
-            const uint32_t g0 = gq;
-            if (!(ok = wait_bar(bar(S_EMPTY + sb), ((it / kSBufs) & 1u) ^ 1u, abort_addr, false))) break;
-            const uint32_t d = tmem + kSCol0 + 64u * sb;
+      // ---- S-MMA issuers: S = Q̃ · [c ; k_r]ᵀ, K = 576 in 36 steps of 16. The whole warp runs the
+      // loop and waits; one elected lane issues each group's 12 MMAs and their commits.
+      const uint32_t parity = warp == 1 ? 0u : 1u;
+      const uint64_t k_desc = ptx::smem_desc_sw128(base + kOffK, 16, 1024);
+      uint32_t it = 0, seg = 0, gq = 0;
+      bool ok = true;
+      while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
+        if (!(ok = wait_bar_warp(bar(Q_FULL), seg & 1u, abort_addr, false))) break;
+        if (parity == 0 && lane == 0)   // every row-warp thread has copied its part of the query out of the ring
+          for (int qg = 0; qg < kQGroups; ++qg) ptx::mbar_arrive(bar(K_EMPTY + (gq + qg) % kRing));
+        __syncwarp();
+        ++seg;
+        gq += kQGroups;
+        for (int t = t_lo; t < t_hi && ok; ++t, ++it, gq += kGroupsPerTile) {
+          if ((it & 1u) != parity) continue;
+          const uint32_t sb = it % kSBufs;
+          const uint32_t g0 = gq;
+          if (!(ok = wait_bar_warp(bar(S_EMPTY + sb), ((it / kSBufs) & 1u) ^ 1u, abort_addr, false))) break;
+          const uint32_t d = tmem + kSCol0 + 64u * sb;
 #pragma unroll
-            for (int q = 0; q < kGroupsPerTile; ++q) {
-              const uint32_t gi = g0 + q, s = gi % kRing;
-              if (!(ok = wait_bar(bar(K_FULL + s), (gi / kRing) & 1u, abort_addr, false))) break;
+          for (int q = 0; q < kGroupsPerTile; ++q) {
+            const uint32_t gi = g0 + q, s = gi % kRing;
+            if (!(ok = wait_bar_warp(bar(K_FULL + s), (gi / kRing) & 1u, abort_addr, false))) break;
+            if (ptx::elect_one()) {
               ptx::tc_fence_after();
               const uint64_t gd = k_desc + (uint64_t)(s * (kGroupBytes >> 4));
 #pragma unroll
@@ -504,9 +521,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
                 for (int k = 0; k < 4; ++k) ptx::mma_ts(d, a + 8u * k, bd + 2 * k, kIdescS, (q | j | k) ? 1u : 0u);
               }
               ptx::mma_commit(bar(K_EMPTY + s));
+              if (q == kGroupsPerTile - 1) ptx::mma_commit(bar(S_FULL + sb));
             }
-            if (!ok) break;
-            ptx::mma_commit(bar(S_FULL + sb));
+            __syncwarp();
           }
         }
       }
@@ -556,29 +573,42 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
         }
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         gq += kGroupsPerTile * (t_hi - t_lo);
+        // software pipeline: a tile's scores are read from TMEM while the previous tile's P goes out
+        uint32_t sr[32];
+        if (t_lo < t_hi) {
+          const uint32_t s = it % kSBufs;
+          if (!wait_bar_warp(bar(S_FULL + s), (it / kSBufs) & 1u, abort_addr, false)) { ok = false; break; }
+          ptx::tc_fence_after();
+          ptx::tmem_ld_16x256b_x8(tmem + s_lane + kSCol0 + 64u * s, sr);
+          ptx::tmem_wait_ld_regs(sr);
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar(S_EMPTY + s));
+        }
         for (int t = t_lo; t < t_hi; ++t, ++it) {
-          const uint32_t s = it % kSBufs, stg = it % kStaging;
+          const uint32_t stg = it % kStaging;
           if (nb >= 0 && t == max(t_lo, t_hi - 3)) {   // the next segment's query row into L2
             const char* nq = reinterpret_cast<const char*>(p.q_abs + ((size_t)vrow(nb) * kH + h) * kRow);
             for (int k = g ? 5 : 0; k < (g ? 9 : 5); ++k) ptx::prefetch_l2(nq + 128 * k);
           }
           // probe this tile's staging buffer now; the answer is used after the arithmetic
           const bool stg_free = ptx::mbar_test_wait_cluster(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u);
-          if (!wait_bar_warp(bar(S_FULL + s), (it / kSBufs) & 1u, abort_addr, false)) { ok = false; break; }
-          uint32_t sr[32];
-          ptx::tc_fence_after();
-          ptx::tmem_ld_16x256b_x8(tmem + s_lane + kSCol0 + 64u * s, sr);
-          ptx::tmem_wait_ld();
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(bar(S_EMPTY + s));
           uint32_t pk0[8], pk1[8];
           float al0 = 1.f, al1 = 1.f;
           const int valid = L - t * kTile;
           if (valid >= kTile) softmax_rows<false>(sr, kTile, t4, scale2, m0, m1, l0, l1, al0, al1, pk0, pk1);
           else softmax_rows<true>(sr, valid, t4, scale2, m0, m1, l0, l1, al0, al1, pk0, pk1);
+          // the next tile's scores into the same registers (issued now, waited for after the P store)
+          const bool more = t + 1 < t_hi;
+          const uint32_t sn = (it + 1) % kSBufs;
+          if (more) {
+            if (!wait_bar_warp(bar(S_FULL + sn), ((it + 1) / kSBufs) & 1u, abort_addr, false)) { ok = false; break; }
+            ptx::tc_fence_after();
+            ptx::tmem_ld_16x256b_x8(tmem + s_lane + kSCol0 + 64u * sn, sr);
+          }
           // this tile's staging buffer must have been copied out (tile it - kStaging)
           if (!__all_sync(0xffffffffu, stg_free) &&
               !wait_bar_warp(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u, abort_addr, true)) {
+            if (more) ptx::tmem_wait_ld_regs(sr);
             ok = false;
             break;
           }
@@ -592,6 +622,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           // visible to the bulk copy (async proxy), then handed to the copier
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(bar(P_WRITTEN + stg));
+          if (more) {
+            ptx::tmem_wait_ld_regs(sr);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar(S_EMPTY + sn));
+          }
         }
         if (!ok) break;
         {
@@ -651,7 +686,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           wait_bar(bar(V_FULL + k % kVStages), (k / kVStages) & 1u, abort_addr, false, false);
       }
     } else if (warp == 1) {
-      // ---- MMA issuer (lane 0) with the warp's help for masking: O += P · C, K = 64 positions in
+      // ---- MMA issuer (an elected lane) with the warp's help for masking: O += P · C, K = 64 positions in
       // 4 steps of 16, N = 512 in 2 halves. A tile's P is complete (and O rescaled for it) once the
       // row warps arrived on P_LOCAL.
       const uint64_t v_desc0 = ptx::smem_desc_sw128(base + kOffV, kChunkBytes, 1024);
@@ -683,7 +718,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
               __syncwarp();
             }
           }
-          if (lane == 0) {
+          if (ptx::elect_one()) {
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_after();
             const uint64_t pd = p_desc0 + (uint64_t)(slot * (kSlotStride >> 4));

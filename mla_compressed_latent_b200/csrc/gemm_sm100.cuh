@@ -55,20 +55,33 @@ struct Params {
   int M2;
   __nv_bfloat16* y2;
   int64_t y2_tok_stride;
+  // Layouts: a_kmajor = the weights are stored [H, M, K] (K contiguous: W[h] transposed), read
+  // K-major; x_shared = X is [n_tok, K], one row per token shared by every head.
+  int a_kmajor, x_shared;
 };
 
 __host__ __device__ constexpr int stage_bytes(int tn) { return kABytes + tn * 128; }
 __host__ __device__ constexpr int smem_bytes(int tn, int stages) { return 1024 + kBarBytes + stages * stage_bytes(tn); }
 
-__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
+#ifdef MLA_TEST_HOOKS
+// Test builds only: with g_test_stall set, each CTA's MMA issuer first waits for a barrier phase that
+// nothing completes, with a 10 ms limit, so that the bounded-wait path (status, abort, drain) runs.
+__device__ int g_test_stall;
+#endif
+
+// Waits for the phase of `parity`. Gives up (false) after limit_ns, recording MLA_ERR_TIMEOUT, or as
+// soon as *abort is set (when abort is given).
+__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, const volatile int* abort = nullptr,
+                                     uint64_t limit_ns = kTimeoutNs) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = 0;
   for (uint32_t n = 0;; ++n) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if ((n & 15u) == 15u) {
+      if (abort && *abort) return false;
       const uint64_t now = ptx::globaltimer();
       if (t0 == 0) t0 = now;
-      else if (now - t0 > kTimeoutNs) { report(MLA_ERR_TIMEOUT); return false; }
+      else if (now - t0 > limit_ns) { report(MLA_ERR_TIMEOUT); return false; }
     }
   }
 }
@@ -96,6 +109,7 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
   const int S = p.stages;
   const uint32_t full0 = base, empty0 = base + 8u * kMaxStages, done = base + 16u * kMaxStages;
   const uint32_t slot = done + 8u;
+  volatile int* abort = reinterpret_cast<volatile int*>(smem_raw + (done + 16u - raw));   // the issuer gave up
   const uint32_t ring = base + kBarBytes;
   const uint32_t sbytes = (uint32_t)stage_bytes(p.tn);
   const uint32_t tmem_cols = p.tn <= 32 ? 32u : (p.tn <= 64 ? 64u : 128u);
@@ -103,6 +117,7 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { ptx::mbar_init(full0 + 8u * s, 1); ptx::mbar_init(empty0 + 8u * s, 1); }
     ptx::mbar_init(done, 1);
+    *abort = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(tw);
     ptx::prefetch_tmap(&tm_x);
@@ -117,34 +132,55 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
 
   if (warp == 0 && lane == 0) {
     // ---- TMA producer: per K chunk two weight boxes (64 k x 64 features) and one token box
-    for (int i = 0; i < nk; ++i) {
+    int i = 0;
+    for (; i < nk; ++i) {
       const int s = i % S;
-      if (!wait(empty0 + 8u * s, ((i / S) & 1u) ^ 1u)) break;
+      if (!wait(empty0 + 8u * s, ((i / S) & 1u) ^ 1u, abort)) break;
       const uint32_t st = ring + s * sbytes;
-      const int k = h * p.K + (kc0 + i) * kBK;
+      const int kk = (kc0 + i) * kBK, k = h * p.K + kk;
       ptx::mbar_arrive_expect_tx(full0 + 8u * s, sbytes);
-      ptx::tma_load_2d(st, tw, mt * kBM, k, full0 + 8u * s);
-      ptx::tma_load_2d(st + kABytes / 2, tw, mt * kBM + 64, k, full0 + 8u * s);
-      ptx::tma_load_2d(st + kABytes, &tm_x, k, tok0, full0 + 8u * s);
+      if (p.a_kmajor) {   // rows m of W[h]ᵀ: two boxes of 64 rows x 64 k
+        ptx::tma_load_2d(st, tw, kk, h * M + mt * kBM, full0 + 8u * s);
+        ptx::tma_load_2d(st + kABytes / 2, tw, kk, h * M + mt * kBM + 64, full0 + 8u * s);
+      } else {
+        ptx::tma_load_2d(st, tw, mt * kBM, k, full0 + 8u * s);
+        ptx::tma_load_2d(st + kABytes / 2, tw, mt * kBM + 64, k, full0 + 8u * s);
+      }
+      ptx::tma_load_2d(st + kABytes, &tm_x, p.x_shared ? kk : k, tok0, full0 + 8u * s);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer: M = 128, N = tn, four K = 16 steps per chunk
-    const uint32_t idesc = ptx::idesc_bf16_f32_ab(kBM, p.tn, true, false);
-    for (int i = 0; i < nk; ++i) {
+    // every load issued must land before the CTA may exit (waited for even after a give-up)
+    for (int k = (i > S ? i - S : 0); k < i; ++k) wait(full0 + 8u * (k % S), (k / S) & 1u);
+  } else if (warp == 1) {
+    // ---- MMA issuer: M = 128, N = tn, four K = 16 steps per chunk; the warp waits, an elected lane issues
+    const uint32_t idesc = ptx::idesc_bf16_f32_ab(kBM, p.tn, !p.a_kmajor, false);
+    bool live = true;
+#ifdef MLA_TEST_HOOKS
+    // phase 0 of `done` completes only through this warp's own commit below: nothing else can end the wait
+    if (g_test_stall) live = __all_sync(0xffffffffu, wait(done, 0u, nullptr, 10000000ull));
+#endif
+    for (int i = 0; i < nk && live; ++i) {
       const int s = i % S;
-      if (!wait(full0 + 8u * s, (i / S) & 1u)) break;
-      ptx::tc_fence_after();
-      const uint32_t st = ring + s * sbytes;
-      // A, MN-major: 8-row K groups 1024 B apart (SBO), the two 64-feature halves one box apart (LBO).
-      // B, K-major: 8-token groups 1024 B apart; a K step of 16 moves 32 B inside the swizzle row.
-      const uint64_t ad = ptx::smem_desc_sw128(st, kABytes / 2, 1024);
-      const uint64_t bd = ptx::smem_desc_sw128(st + kABytes, 16, 1024);
+      if (!__all_sync(0xffffffffu, wait(full0 + 8u * s, (i / S) & 1u))) { live = false; break; }
+      if (ptx::elect_one()) {
+        ptx::tc_fence_after();
+        const uint32_t st = ring + s * sbytes;
+        // A, MN-major: 8-row K groups 1024 B apart (SBO), the two 64-feature halves one box apart (LBO);
+        // a K step of 16 moves 16 rows = 2048 B. A, K-major: 8-feature groups 1024 B apart (the two
+        // 64-row boxes are contiguous); a K step moves 32 B inside the swizzle row.
+        // B, K-major: 8-token groups 1024 B apart; a K step of 16 moves 32 B inside the swizzle row.
+        const uint64_t ad = p.a_kmajor ? ptx::smem_desc_sw128(st, 16, 1024) : ptx::smem_desc_sw128(st, kABytes / 2, 1024);
+        const uint64_t a_step = p.a_kmajor ? 2u : (uint64_t)(2048 >> 4);
+        const uint64_t bd = ptx::smem_desc_sw128(st + kABytes, 16, 1024);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        ptx::mma_ss(tmem, ad + (uint64_t)(k * (2048 >> 4)), bd + (uint64_t)(2 * k), idesc, (i | k) ? 1u : 0u);
-      ptx::mma_commit(empty0 + 8u * s);
+        for (int k = 0; k < 4; ++k)
+          ptx::mma_ss(tmem, ad + (uint64_t)k * a_step, bd + (uint64_t)(2 * k), idesc, (i | k) ? 1u : 0u);
+        ptx::mma_commit(empty0 + 8u * s);
+      }
+      __syncwarp();
     }
-    ptx::mma_commit(done);
+    if (!live && lane == 0) *abort = 1;   // the producer stops waiting for stages that will not be freed
+    if (ptx::elect_one()) ptx::mma_commit(done);
+    __syncwarp();
   } else if (warp >= 4) {
     // ---- epilogue: thread = output feature (TMEM lane), 32 tokens (TMEM columns) per load
     const int row = threadIdx.x - 128;
@@ -254,12 +290,17 @@ struct Problem {
   const void* w2 = nullptr;  // optional second weight [K, M2] (H = 1, mode 0; output p.y2)
   int M2 = 0;
   int num_sms = 0;           // SMs of the device (0: unknown)
+  bool a_kmajor = false;     // w is [H * M, K] (each head's weight transposed), read K-major
+  bool x_shared = false;     // x is [n_tok, K], the same row for every head
 };
 
 // Launches on `st`; returns MLA_OK, or an error status with nothing launched.
 inline int run(const Problem& pr, Params p, cudaStream_t st) {
   if (!supported(pr.K, pr.M) || pr.n_tok <= 0 || pr.H <= 0 || pr.splits <= 0) return MLA_ERR_UNSUPPORTED;
   const bool two = pr.w2 != nullptr;
+  if ((pr.a_kmajor || pr.x_shared) && (two || p.rope_in != nullptr)) return MLA_ERR_UNSUPPORTED;
+  p.a_kmajor = pr.a_kmajor ? 1 : 0;
+  p.x_shared = pr.x_shared ? 1 : 0;
   if (two && (pr.H != 1 || pr.splits != 1 || p.mode != 0 || p.rope_in != nullptr || !p.y2 || !supported(pr.K, pr.M2)))
     return MLA_ERR_UNSUPPORTED;
   p.M = pr.M;
@@ -278,10 +319,14 @@ inline int run(const Problem& pr, Params p, cudaStream_t st) {
   if (pr.num_sms > 0 && ctas > pr.num_sms)
     p.stages = std::max(1, std::min(p.stages, (kSmemMax / 2 - 2048) / stage_bytes(p.tn)));
   CUtensorMap tm_w, tm_x, tm_w2;
-  if (!tmap::make_bf16_sw128(&tm_w, pr.w, pr.M, (int64_t)pr.H * pr.K, pr.M, kBK)) return MLA_ERR_INVALID_ARG;
-  if (two && !tmap::make_bf16_sw128(&tm_w2, pr.w2, pr.M2, pr.K, pr.M2, kBK)) return MLA_ERR_INVALID_ARG;
-  if (!tmap::make_bf16_sw128(&tm_x, pr.x, (int64_t)pr.H * pr.K, pr.n_tok, (int64_t)pr.H * pr.K, p.tn))
+  if (pr.a_kmajor) {
+    if (!tmap::make_bf16_sw128(&tm_w, pr.w, pr.K, (int64_t)pr.H * pr.M, pr.K, kBK)) return MLA_ERR_INVALID_ARG;
+  } else if (!tmap::make_bf16_sw128(&tm_w, pr.w, pr.M, (int64_t)pr.H * pr.K, pr.M, kBK)) {
     return MLA_ERR_INVALID_ARG;
+  }
+  if (two && !tmap::make_bf16_sw128(&tm_w2, pr.w2, pr.M2, pr.K, pr.M2, kBK)) return MLA_ERR_INVALID_ARG;
+  const int64_t x_cols = pr.x_shared ? (int64_t)pr.K : (int64_t)pr.H * pr.K;
+  if (!tmap::make_bf16_sw128(&tm_x, pr.x, x_cols, pr.n_tok, x_cols, p.tn)) return MLA_ERR_INVALID_ARG;
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);

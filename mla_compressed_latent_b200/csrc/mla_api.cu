@@ -160,6 +160,14 @@ const char* mla_status_string(int s) {
 
 uint64_t mla_launch_count(void) { return mla::g_launches.load(std::memory_order_relaxed); }
 
+#ifdef MLA_TEST_HOOKS
+// Test builds only (not declared in mla.h): makes every per-head GEMM's MMA issuer wait for a phase
+// that nothing completes, so that a test can watch a bounded wait run out on the GPU.
+int mla_test_set_stall(int on) {
+  return cudaMemcpyToSymbol(mla::gemm::g_test_stall, &on, sizeof(int)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+#endif
+
 const char* mla_build_info(void) {
   return "libmla: sm_100a; kernels: simt (fp32/bf16 all steps), sm100 absorbed decode, GQLA grouped decode and per-head projections (tcgen05/TMA)";
 }
@@ -220,10 +228,10 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     p.mode = 1;
     p.part = reinterpret_cast<float*>(workspace);
     if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, ks}), p, st))) return rc;
-    const int fin_threads = std::min(1024, (N + 31) / 32 * 32);   // one thread per output column
+    const int fin_threads = std::max(64, std::min(1024, (N / 4 + 31) / 32 * 32));   // four columns per thread
     mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)p.part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
-           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);
+           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0);
     return launch_status();
   }
   const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
@@ -237,7 +245,7 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, 
         part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
         block_table, max_pages, (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride,
-        cache->num_pages);
+        cache->num_pages, 0);
   } else {
     using T = __nv_bfloat16;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, 
@@ -245,7 +253,7 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, 
         part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
         block_table, max_pages, (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride,
-        cache->num_pages);
+        cache->num_pages, 0);
   }
   return launch_status();
 }
@@ -465,9 +473,18 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
     p.y_head_stride = d_v;
     if ((rc = mla::gemm::run(with_sms({w_uv, o_lat, H, d_c, d_v, n_tok, 1}), p, st))) return rc;
     if (w_o) {
-      using T = __nv_bfloat16;
-      launch(mla::simt::proj_partial_kernel<T>, ogrid, mla::simt::PROJ_COLS, 0, st, (const T*)out, n_tok, K,
-             (const T*)w_o, C, K, nullptr, (T*)out_model);
+      if (mla::gemm::supported(K, C)) {   // the heads concatenated, times W_O, on the tensor cores
+        mla::gemm::Params po{};
+        po.mode = 0;
+        po.y = reinterpret_cast<__nv_bfloat16*>(out_model);
+        po.y_tok_stride = C;
+        po.y_head_stride = 0;
+        if ((rc = mla::gemm::run(with_sms({w_o, out, 1, K, C, n_tok, 1}), po, st))) return rc;
+      } else {
+        using T = __nv_bfloat16;
+        launch(mla::simt::proj_partial_kernel<T>, ogrid, mla::simt::PROJ_COLS, 0, st, (const T*)out, n_tok, K,
+               (const T*)w_o, C, K, nullptr, (T*)out_model);
+      }
     }
     return launch_status();
   }
@@ -488,6 +505,172 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
       launch(mla::simt::proj_partial_kernel<T>, ogrid, mla::simt::PROJ_COLS, 0, st, (const T*)out, n_tok, K, (const T*)w_o,
                                                                                C, K, nullptr, (T*)out_model);
   }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------------------------------------
+// f3: W_UV·W_O absorbed into one output weight, and the output projection through it
+// ------------------------------------------------------------------------------------------------
+int mla_preabsorb_out_weights(const mla_dims_t* dims, int32_t dtype, const void* w_uv, const void* w_o, int32_t C,
+                              void* w_uvo, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (C <= 0 || !w_uv || !w_o || !w_uvo) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(w_uv) || !aligned16(w_o) || !aligned16(w_uvo)) return MLA_ERR_INVALID_ARG;
+  const int H = dims->H, d_c = dims->d_c, d_v = dims->d_v;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = esize(dtype);
+  // head h: W_UVO[h] [d_c, C] = W_UV[h] [d_c, d_v] · W_O[h*d_v : (h+1)*d_v, :]
+  for (int h = 0; h < H; ++h) {
+    const char* wuv_h = static_cast<const char*>(w_uv) + (size_t)h * d_c * d_v * es;
+    const char* wo_h = static_cast<const char*>(w_o) + (size_t)h * d_v * C * es;
+    char* y_h = static_cast<char*>(w_uvo) + (size_t)h * d_c * C * es;
+    if (dtype == MLA_BF16 && mla::gemm::supported(d_v, C) && aligned16(wuv_h) && aligned16(wo_h) && aligned16(y_h) &&
+        ((size_t)d_v * es) % 16 == 0) {
+      mla::gemm::Params p{};
+      p.mode = 0;
+      p.y = reinterpret_cast<__nv_bfloat16*>(y_h);
+      p.y_tok_stride = C;
+      p.y_head_stride = 0;
+      if ((rc = mla::gemm::run(with_sms({wo_h, wuv_h, 1, d_v, C, d_c, 1}), p, st))) return rc;
+    } else {
+      dim3 grid((C + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS, (d_c + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK, 1);
+      if (dtype == MLA_F32)
+        launch(mla::simt::proj_partial_kernel<float>, grid, mla::simt::PROJ_COLS, 0, st, (const float*)wuv_h, d_c, d_v,
+               (const float*)wo_h, C, d_v, nullptr, (float*)y_h);
+      else
+        launch(mla::simt::proj_partial_kernel<__nv_bfloat16>, grid, mla::simt::PROJ_COLS, 0, st,
+               (const __nv_bfloat16*)wuv_h, d_c, d_v, (const __nv_bfloat16*)wo_h, C, d_v, nullptr, (__nv_bfloat16*)y_h);
+    }
+  }
+  return launch_status();
+}
+
+int mla_out_proj_preabsorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* o_lat,
+                             const void* w_uvo, int32_t C, void* out_model, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (!tokens_ok(B, s_q) || C <= 0 || !o_lat || !w_uvo || !out_model) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o_lat) || !aligned16(w_uvo) || !aligned16(out_model)) return MLA_ERR_INVALID_ARG;
+  const int n_tok = B * s_q, K = dims->H * dims->d_c;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // out_model[tok, :] = concat_h(o_lat[tok, h, :]) · W_UVO, W_UVO = [H*d_c, C]
+  if (dtype == MLA_BF16 && mla::gemm::supported(K, C)) {
+    mla::gemm::Params p{};
+    p.mode = 0;
+    p.y = reinterpret_cast<__nv_bfloat16*>(out_model);
+    p.y_tok_stride = C;
+    p.y_head_stride = 0;
+    if ((rc = mla::gemm::run(with_sms({w_uvo, o_lat, 1, K, C, n_tok, 1}), p, st))) return rc;
+    return launch_status();
+  }
+  dim3 grid((C + mla::simt::PROJ_COLS - 1) / mla::simt::PROJ_COLS, (n_tok + mla::simt::PROJ_TOK - 1) / mla::simt::PROJ_TOK, 1);
+  if (dtype == MLA_F32)
+    launch(mla::simt::proj_partial_kernel<float>, grid, mla::simt::PROJ_COLS, 0, st, (const float*)o_lat, n_tok, K,
+           (const float*)w_uvo, C, K, nullptr, (float*)out_model);
+  else
+    launch(mla::simt::proj_partial_kernel<__nv_bfloat16>, grid, mla::simt::PROJ_COLS, 0, st, (const __nv_bfloat16*)o_lat,
+           n_tok, K, (const __nv_bfloat16*)w_uvo, C, K, nullptr, (__nv_bfloat16*)out_model);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------------------------------------
+// f3: append to the expanded (GQA) cache
+// ------------------------------------------------------------------------------------------------
+namespace {
+struct GqaAppendLayout { int ks; size_t part, cbuf, kbuf, vbuf, total; };
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+GqaAppendLayout gqa_append_layout(const mla_dims_t* d, int n_tok, int C) {
+  GqaAppendLayout L{};
+  const int N = d->d_c + d->d_r;
+  L.ks = append_tc_splits(n_tok, C, N);
+  L.part = 0;
+  L.cbuf = up256((size_t)L.ks * n_tok * N * sizeof(float));
+  L.kbuf = L.cbuf + up256((size_t)n_tok * d->d_c * 2);
+  L.vbuf = L.kbuf + up256((size_t)n_tok * d->g * d->D * 2);
+  L.total = L.vbuf + up256((size_t)n_tok * d->g * d->d_v * 2);
+  return L;
+}
+bool gqa_append_supported(const mla_dims_t* d, int32_t dtype, int C) {
+  return dtype == MLA_BF16 && d->g > 0 && d->H % d->g == 0 && mla::gemm::supported(C, d->d_c + d->d_r) &&
+         mla::gemm::supported(d->d_c, d->D) && mla::gemm::supported(d->d_c, d->d_v);
+}
+}  // namespace
+
+size_t mla_gqa_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C) {
+  if (check_dims(dims) || !tokens_ok(B, s_q) || C <= 0 || !gqa_append_supported(dims, MLA_BF16, C)) return 0;
+  return gqa_append_layout(dims, B * s_q, C).total;
+}
+
+int mla_append_gqa_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x, int32_t C,
+                         const void* w_dkv_kr, const void* gamma, const void* w_uk_g, const void* w_uv_g,
+                         const int32_t* seqlens, const int32_t* block_table, int32_t max_pages,
+                         const mla_gqa_cache_t* cache, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (dims->g <= 0 || dims->H % dims->g) return MLA_ERR_INVALID_ARG;
+  if (!tokens_ok(B, s_q) || C <= 0 || max_pages <= 0 || !x || !w_dkv_kr || !w_uk_g || !w_uv_g || !seqlens ||
+      !block_table || !cache)
+    return MLA_ERR_INVALID_ARG;
+  if (!cache->k || !cache->v || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_dkv_kr) || (gamma && !aligned16(gamma)) || !aligned16(w_uk_g) ||
+      !aligned16(w_uv_g) || !aligned16(seqlens) || !aligned16(block_table) || !aligned16(cache->k) ||
+      !aligned16(cache->v) || !aligned16(cache->rope))
+    return MLA_ERR_INVALID_ARG;
+  if (!stride_ok(cache->k_stride, dtype, (int64_t)dims->g * dims->D) ||
+      !stride_ok(cache->v_stride, dtype, (int64_t)dims->g * dims->d_v) || !stride_ok(cache->rope_stride, dtype, dims->d_r))
+    return MLA_ERR_INVALID_ARG;
+  if (!gqa_append_supported(dims, dtype, C)) return MLA_ERR_UNSUPPORTED;
+  const int n_tok = B * s_q, N = dims->d_c + dims->d_r, g = dims->g;
+  const GqaAppendLayout lay = gqa_append_layout(dims, n_tok, C);
+  if (!workspace || ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLA_ERR_INVALID_ARG;
+  using T = __nv_bfloat16;
+  char* ws = static_cast<char*>(workspace);
+  float* part = reinterpret_cast<float*>(ws + lay.part);
+  T* cbuf = reinterpret_cast<T*>(ws + lay.cbuf);
+  T* kbuf = reinterpret_cast<T*>(ws + lay.kbuf);
+  T* vbuf = reinterpret_cast<T*>(ws + lay.vbuf);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t fin_smem = (size_t)N * sizeof(float);
+  if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
+  // 1. z = x · [W_DKV | W_KR] (split-K partial sums)
+  mla::gemm::Params p{};
+  p.mode = 1;
+  p.part = part;
+  if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, lay.ks}), p, st))) return rc;
+  // 2. c = RMSNorm(z_c)·gamma into a plain buffer (rounded to the storage type, as a latent cache row
+  //    would be); k_r = RoPE(z_r) into the cache's RoPE rows
+  const int fin_threads = std::max(64, std::min(1024, (N / 4 + 31) / 32 * 32));
+  mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)part,
+                  lay.ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
+                  block_table, max_pages, cbuf, (int64_t)dims->d_c, (T*)cache->rope, cache->rope_stride,
+                  cache->num_pages, 1);
+  // 3. K_g = W_UK[g] · c (W_UK stored [g, D, d_c]: read K-major), V_g = c · W_UV[g], every group
+  mla::gemm::Problem pk{w_uk_g, cbuf, g, dims->d_c, dims->D, n_tok, 1};
+  pk.a_kmajor = true;
+  pk.x_shared = true;
+  mla::gemm::Params pkp{};
+  pkp.mode = 0;
+  pkp.y = kbuf;
+  pkp.y_tok_stride = (int64_t)g * dims->D;
+  pkp.y_head_stride = dims->D;
+  if ((rc = mla::gemm::run(with_sms(pk), pkp, st))) return rc;
+  mla::gemm::Problem pv{w_uv_g, cbuf, g, dims->d_c, dims->d_v, n_tok, 1};
+  pv.x_shared = true;
+  mla::gemm::Params pvp{};
+  pvp.mode = 0;
+  pvp.y = vbuf;
+  pvp.y_tok_stride = (int64_t)g * dims->d_v;
+  pvp.y_head_stride = dims->d_v;
+  if ((rc = mla::gemm::run(with_sms(pv), pvp, st))) return rc;
+  // 4. the rows into the cache slots of their positions
+  mla::launch_pdl(mla::simt::gqa_scatter_kernel<T>, dim3(n_tok), dim3(128), 0, st, (const T*)kbuf, (const T*)vbuf, s_q,
+                  g * dims->D, g * dims->d_v, seqlens, block_table, max_pages, cache->num_pages, (T*)cache->k,
+                  cache->k_stride, (T*)cache->v, cache->v_stride);
   return launch_status();
 }
 
@@ -628,11 +811,11 @@ extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, i
     p.mode = 1;
     p.part = part;
     if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, ks}), p, st))) return rc;
-    const int fin_threads = std::min(1024, (N + 31) / 32 * 32);
+    const int fin_threads = std::max(64, std::min(1024, (N / 4 + 31) / 32 * 32));
     mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st,
                     (const float*)part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps,
                     dims->rope_base, seqlens, block_table, max_pages, (T*)cache->latent, cache->latent_stride,
-                    (T*)cache->rope, cache->rope_stride, cache->num_pages);
+                    (T*)cache->rope, cache->rope_stride, cache->num_pages, 0);
     return launch_status();
   }
   const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
@@ -644,14 +827,14 @@ extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, i
            (const T*)w_dkv_kr, N, k_chunk, part, (T*)nullptr);
     launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
-           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);
+           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0);
   } else {
     using T = __nv_bfloat16;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, (const T*)x, n_tok, C,
            (const T*)w_dkv_kr, N, k_chunk, part, (T*)nullptr);
     launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
-           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages);
+           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0);
   }
   return launch_status();
 }

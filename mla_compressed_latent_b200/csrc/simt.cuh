@@ -72,15 +72,39 @@ __device__ __forceinline__ float sum_slices(const float* src, int ksplit, int64_
 
 // =============================================================================================
 // a1 epilogue: sum the K slices, RMSNorm the latent part, rotate the RoPE part, store the row.
-// One block per new token.
+// One block per new token. The partial sums are read 16 bytes at a time (4 columns per thread and
+// slice, several slices in flight) and the latent row is written 16 bytes at a time. With
+// latent_by_token the latent row of token tok goes to latent + tok * lat_stride (a plain buffer)
+// instead of its cache slot; the RoPE key always goes to its cache slot.
 // =============================================================================================
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+  static constexpr int n = 4;
+  static __device__ __forceinline__ void store(float* p, const float* v) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <> struct Vec16<__nv_bfloat16> {
+  static constexpr int n = 8;
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float* v) {
+    uint4 u;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]), h3 = __floats2bfloat162_rn(v[6], v[7]);
+    u.x = *reinterpret_cast<uint32_t*>(&h0);
+    u.y = *reinterpret_cast<uint32_t*>(&h1);
+    u.z = *reinterpret_cast<uint32_t*>(&h2);
+    u.w = *reinterpret_cast<uint32_t*>(&h3);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+
 template <typename T>
 __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit, int n_tok, int s_q,
                                      int d_c, int d_r, const T* __restrict__ gamma, float eps,
                                      float rope_base, const int32_t* __restrict__ seqlens,
                                      const int32_t* __restrict__ block_table, int max_pages,
                                      T* latent, int64_t lat_stride, T* rope, int64_t rope_stride,
-                                     int num_pages) {
+                                     int num_pages, int latent_by_token) {
   extern __shared__ float z[];
   __shared__ float red[32];
   grid_dependency_wait();   // launched with programmatic dependent launch after the projection
@@ -88,8 +112,31 @@ __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit,
   const int tok = blockIdx.x;
   const int b = tok / s_q, t = tok % s_q;
   const int N = d_c + d_r;
-  for (int i = threadIdx.x; i < N; i += blockDim.x)
-    z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
+  if ((N & 3) == 0) {
+    const float4* src = reinterpret_cast<const float4*>(part + (int64_t)tok * N);
+    const int64_t step4 = (int64_t)n_tok * N / 4;
+    for (int i4 = threadIdx.x; i4 < N / 4; i4 += blockDim.x) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      int ks = 0;
+      for (; ks + 4 <= ksplit; ks += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = src[(ks + u) * step4 + i4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+        }
+      }
+      for (; ks < ksplit; ++ks) {
+        const float4 v = src[ks * step4 + i4];
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      z[4 * i4] = acc.x; z[4 * i4 + 1] = acc.y; z[4 * i4 + 2] = acc.z; z[4 * i4 + 3] = acc.w;
+    }
+  } else {
+    for (int i = threadIdx.x; i < N; i += blockDim.x)
+      z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
+  }
   __syncthreads();
   float ss = 0.f;
   for (int i = threadIdx.x; i < d_c; i += blockDim.x) ss = fmaf(z[i], z[i], ss);
@@ -102,9 +149,17 @@ __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit,
   }
   const int64_t row = cache_row(block_table + (int64_t)b * max_pages, pos, num_pages);
   if (row < 0) return;
-  for (int i = threadIdx.x; i < d_c; i += blockDim.x) {
-    const float gm = gamma ? ld(gamma + i) : 1.f;
-    st(latent + row * lat_stride + i, z[i] * inv * gm);
+  T* lrow = latent + (latent_by_token ? (int64_t)tok : row) * lat_stride;
+  constexpr int V = Vec16<T>::n;
+  if (d_c % V == 0) {   // row starts are 16-byte aligned (aligned base, stride a multiple of 16 bytes)
+    for (int i = threadIdx.x * V; i < d_c; i += blockDim.x * V) {
+      float v[V];
+#pragma unroll
+      for (int u = 0; u < V; ++u) v[u] = z[i + u] * inv * (gamma ? ld(gamma + i + u) : 1.f);
+      Vec16<T>::store(lrow + i, v);
+    }
+  } else {
+    for (int i = threadIdx.x; i < d_c; i += blockDim.x) st(lrow + i, z[i] * inv * (gamma ? ld(gamma + i) : 1.f));
   }
   for (int i = threadIdx.x; i < d_r / 2; i += blockDim.x) {
     float cs, sn;
@@ -113,6 +168,58 @@ __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit,
     st(rope + row * rope_stride + 2 * i, a * cs - bb * sn);
     st(rope + row * rope_stride + 2 * i + 1, a * sn + bb * cs);
   }
+}
+
+// =============================================================================================
+// f3 epilogue of the expanded (GQA) cache append: token tok's expanded keys [g*D] and values
+// [g*d_v], computed into plain buffers, copied into the cache rows of its position, 16 bytes at a
+// time (row widths are multiples of 16 bytes). One block per new token.
+// =============================================================================================
+template <typename T>
+__global__ void gqa_scatter_kernel(const T* __restrict__ kbuf, const T* __restrict__ vbuf, int s_q, int kw, int vw,
+                                   const int32_t* __restrict__ seqlens, const int32_t* __restrict__ block_table,
+                                   int max_pages, int num_pages, T* k, int64_t k_stride, T* v, int64_t v_stride) {
+  grid_dependency_wait();
+  allow_dependents();
+  const int tok = blockIdx.x;
+  const int b = tok / s_q, t = tok % s_q;
+  const int pos = seqlens[b] - s_q + t;
+  if (pos < 0 || (pos >> 6) >= max_pages) {
+    if (threadIdx.x == 0) report(MLA_ERR_DEVICE_CHECK);
+    return;
+  }
+  const int64_t row = cache_row(block_table + (int64_t)b * max_pages, pos, num_pages);
+  if (row < 0) return;
+  const uint4* ks = reinterpret_cast<const uint4*>(kbuf + (int64_t)tok * kw);
+  const uint4* vs = reinterpret_cast<const uint4*>(vbuf + (int64_t)tok * vw);
+  uint4* kd = reinterpret_cast<uint4*>(k + row * k_stride);
+  uint4* vd = reinterpret_cast<uint4*>(v + row * v_stride);
+  const int nk = kw * (int)sizeof(T) / 16, nv = vw * (int)sizeof(T) / 16;
+  for (int i = threadIdx.x; i < nk; i += blockDim.x) kd[i] = ks[i];
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) vd[i] = vs[i];
+}
+
+// =============================================================================================
+// Sum of K slices: out[tok, m] = sum_s part[s, tok, m], stored in T (split-K GEMM epilogue).
+// Four columns per thread (M a multiple of 4), one block row of tokens per blockIdx.y.
+// =============================================================================================
+template <typename T>
+__global__ void reduce_slices_kernel(const float* __restrict__ part, int ksplit, int n_tok, int M, T* out,
+                                     int64_t out_stride) {
+  grid_dependency_wait();
+  allow_dependents();
+  const int tok = blockIdx.y;
+  const int i4 = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i4 >= M / 4) return;
+  const float4* src = reinterpret_cast<const float4*>(part + (int64_t)tok * M) + i4;
+  const int64_t step4 = (int64_t)n_tok * M / 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < ksplit; ++s) {
+    const float4 v = src[s * step4];
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  T* o = out + (int64_t)tok * out_stride + 4 * i4;
+  st(o, acc.x); st(o + 1, acc.y); st(o + 2, acc.z); st(o + 3, acc.w);
 }
 
 // =============================================================================================

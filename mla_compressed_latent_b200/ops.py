@@ -227,6 +227,50 @@ def mla_decode_gqla_grouped(dims: Dims, q_nope, q_rope_raw, cache: GqaCache, blo
     return out, lse
 
 
+def mla_append_gqa_cache(dims: Dims, x, w_dkv_kr, gamma, w_uk_g, w_uv_g, seqlens, block_table, cache: GqaCache,
+                         workspace=None, stream=None):
+    """Append this step's tokens to the expanded GQA cache: k_r and, per group, K = W_UK[g]·c and
+    V = c·W_UV[g] of c = RMSNorm(x·W_DKV) (x [B, s_q, C], w_uk_g [g, D, d_c], w_uv_g [g, d_c, d_v])."""
+    lib = L.load()
+    B, s_q, C = x.shape
+    d = dims.c()
+    need = lib.mla_gqa_append_workspace_size(ctypes.byref(d), B, s_q, C)
+    workspace, wsb = _workspace(need, x.device, workspace)
+    cc = cache.c()
+    rc = lib.mla_append_gqa_cache(ctypes.byref(d), _dt(x), B, s_q, _ptr(x), C, _ptr(w_dkv_kr), _ptr(gamma),
+                                  _ptr(w_uk_g), _ptr(w_uv_g), _ptr(_i32(seqlens)), _ptr(_i32(block_table)),
+                                  block_table.shape[1], ctypes.byref(cc),
+                                  _ptr(workspace) if workspace is not None else None, wsb, _stream(stream))
+    _check("mla_append_gqa_cache", rc)
+
+
+def mla_preabsorb_out_weights(dims: Dims, w_uv, w_o, w_uvo=None, stream=None):
+    """W_UVO [H, d_c, C] with W_UVO[h] = W_UV[h] · W_O[h*d_v:(h+1)*d_v] (w_uv [H, d_c, d_v], w_o [H*d_v, C])."""
+    lib = L.load()
+    C = w_o.shape[1]
+    if w_uvo is None:
+        w_uvo = torch.empty(dims.H, dims.d_c, C, dtype=w_uv.dtype, device=w_uv.device)
+    d = dims.c()
+    rc = lib.mla_preabsorb_out_weights(ctypes.byref(d), _dt(w_uv), _ptr(w_uv), _ptr(w_o), C, _ptr(w_uvo),
+                                       _stream(stream))
+    _check("mla_preabsorb_out_weights", rc)
+    return w_uvo
+
+
+def mla_out_proj_preabsorbed(dims: Dims, o_lat, w_uvo, out_model=None, stream=None):
+    """out_model [B, s_q, C] = concat_h(o_lat[..., h, :]) · W_UVO (o_lat [B, s_q, H, d_c], w_uvo [H, d_c, C])."""
+    lib = L.load()
+    B, s_q, H, _ = o_lat.shape
+    C = w_uvo.shape[-1]
+    if out_model is None:
+        out_model = torch.empty(B, s_q, C, dtype=o_lat.dtype, device=o_lat.device)
+    d = dims.c()
+    rc = lib.mla_out_proj_preabsorbed(ctypes.byref(d), _dt(o_lat), B, s_q, _ptr(o_lat), _ptr(w_uvo), C,
+                                      _ptr(out_model), _stream(stream))
+    _check("mla_out_proj_preabsorbed", rc)
+    return out_model
+
+
 def mla_check_status(stream=None) -> int:
     return L.load().mla_check_status(_stream(stream))
 

@@ -238,6 +238,23 @@ def out_projection(o_lat, W_UV, W_O=None):
     return out.reshape(s_q, -1) @ np.asarray(W_O, f64)
 
 
+def preabsorbed_out_weights(W_UV, W_O):
+    """The value up-projection absorbed into the output projection ([P4] « Chemin MQA-Absorbé »: the
+    up-projections are absorbed into the query and output projections): head h's block of W_O
+    (rows h·d_v .. h·d_v + d_v - 1) premultiplied by W_UV[h]. W_UV [H, d_c, d_v], W_O [H·d_v, C]
+    -> W_UVO [H, d_c, C]."""
+    W_UV = np.asarray(W_UV, f64)
+    H, d_c, d_v = W_UV.shape
+    W_O = np.asarray(W_O, f64).reshape(H, d_v, -1)
+    return np.einsum("hce,heo->hco", W_UV, W_O)
+
+
+def out_projection_preabsorbed(o_lat, W_UVO):
+    """The layer output straight from the weighted latents: sum over heads of o_lat_h · W_UVO[h].
+    o_lat [s_q, H, d_c], W_UVO [H, d_c, C] -> [s_q, C]."""
+    return np.einsum("thc,hco->to", np.asarray(o_lat, f64), np.asarray(W_UVO, f64))
+
+
 def merge_partials(o_parts, lse_parts):
     """Combine softmax partials computed over disjoint position sets.
 

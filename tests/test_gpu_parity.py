@@ -397,6 +397,55 @@ def test_full_step_dsv3_against_oracle():
 
 # ------------------------------------------------------------------------------------------------
 # a6: GQLA grouped path
+def test_dsv3_context_built_from_hidden_states():
+    """The DeepSeek shape with its configured cache recipe: two whole 4096-position contexts written
+    by mla_append_cache from hidden states x ~ N(0, 1) (4095 positions as one prefill call, then the
+    new token as a decode step, random page table), then absorb -> decode -> out_proj. The oracle
+    builds the same rows from the same x (rms(x·W_DKV), RoPE(x·W_KR)), keeps them in the cache's
+    type, and runs its own absorbed decode and projection on them."""
+    L, B = 4096, 2
+    w = synth.workload("dsv3_b64_l4096", B=B, lengths=("fixed", L), pages="random")
+    case = Case(w)
+    dev = case.to_device()
+    dims = Dims.of(w)
+    dev["pool"].zero_()
+    cache = _cache(dev, case)
+    xs, x64 = [], []
+    for b in range(B):
+        t, t64 = _stored_bf16(synth.context_hidden_states(w, L, b))
+        xs.append(t)
+        x64.append(t64)
+    xt = torch.stack(xs).cuda()
+    prefill = torch.full((B,), L - 1, dtype=torch.int32, device="cuda")
+    ops.mla_append_cache(dims, xt[:, :L - 1].contiguous(), dev["w_dkv_kr"], None, prefill, dev["table"], cache)
+    ops.mla_append_cache(dims, xt[:, L - 1:].contiguous(), dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache)
+    q_abs = ops.mla_absorb_q(dims, dev["q_nope"], dev["q_rope_raw"], dev["W_UK"], dev["seqlens"])
+    o_lat, lse = ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"])
+    out = ops.mla_out_proj(dims, o_lat, dev["W_UV"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    pool = dev["pool"].cpu()
+    got = out.double().cpu().numpy()
+    got_lse = lse.cpu().numpy()
+    for b in range(B):
+        c, kr = O.latent_rows(x64[b], case.W64["W_DKV"], case.W64["W_KR"], np.arange(L))
+        gc, gkr = case.seq_rows64(b, pool)
+        _assert_close(gc, c, "bf16", f"latent rows seq {b}")
+        _assert_close(gkr, kr, "bf16", f"rope rows seq {b}")
+        c_s, kr_s = as_stored(c, "bf16"), as_stored(kr, "bf16")
+        q = as_stored(O.absorb_query(case.q_nope64[b], case.q_rope_raw64[b], case.W64["W_UK"],
+                                     O.token_positions(L, 1)), "bf16")
+        ol, l = O.absorbed_decode(q, c_s, kr_s, L, w.sm_scale)
+        ref = O.out_projection(as_stored(ol, "bf16"), case.W64["W_UV"])
+        _assert_close(got[b], ref, "bf16", f"out seq {b}")
+        _assert_lse(got_lse[b], l, "bf16", f"lse seq {b}")
+
+
+def _stored_bf16(a):
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+    return t, t.to(torch.float64).numpy()
+
+
 # ------------------------------------------------------------------------------------------------
 
 def test_gqla_grouped_equals_absorbed_on_same_weights():
@@ -439,6 +488,79 @@ def test_gqla_grouped_equals_absorbed_on_same_weights():
         _, ref_la = O.absorbed_decode(qa, rows[idx, :w.d_c], rows[idx, w.d_c:], L, w.sm_scale)
         _assert_lse(lse_a[b].cpu().numpy(), ref_la, "bf16", f"absorbed lse seq {b}")
         assert np.abs(ref_la - ref_l).max() < 5e-3      # the two paths agree up to bf16 storage
+
+
+def test_gqa_cache_append_from_hidden_states_then_grouped_decode():
+    """f3: the expanded GQA cache written by the GPU from hidden states (a prefill call, then the new
+    token as a decode step, random page table): K = W_UK[g]·c, V = c·W_UV[g] and k_r per row against
+    the oracle's expansion of its own rows (one bf16 rounding of c, then of K and V), and the
+    grouped decode over that cache against the oracle's grouped attention on its own rows."""
+    lens = (300, 65, 1000)
+    w = synth.workload("gqla_g8_b32_l8192", B=3, lengths=("list", lens), pages="random")
+    case = Case(w)
+    dev = case.to_device()
+    dims = Dims.of(w)
+    n = case.num_pages * 64
+    K = torch.zeros(n, w.g, w.D, dtype=torch.bfloat16, device="cuda")
+    V = torch.zeros(n, w.g, w.d_v, dtype=torch.bfloat16, device="cuda")
+    R = torch.zeros(n, w.d_r, dtype=torch.bfloat16, device="cuda")
+    gcache = GqaCache(K, V, R, case.num_pages)
+    W_UK_g, W_UV_g = dev["W_UK_g"], dev["W_UV_g"]
+    Lmax = max(lens)
+    xs = [_stored_bf16(synth.context_hidden_states(w, Lmax, b)) for b in range(w.B)]
+    xt = torch.stack([t for t, _ in xs]).cuda()
+    # prefill: the first len - 1 positions of every sequence, as s_q = 64 steps of a common length
+    # where possible, then token by token; finally the new token
+    done = np.zeros(w.B, np.int64)
+    while True:
+        todo = np.asarray(lens) - 1 - done
+        if (todo <= 0).all():
+            break
+        step = 64 if (todo >= 64).all() else 1
+        act = [b for b in range(w.B) if todo[b] >= step]
+        sl = torch.from_numpy((done[act] + step).astype(np.int32)).cuda()
+        xb = torch.stack([xt[b, done[b]:done[b] + step] for b in act]).contiguous()
+        tb = dev["table"][torch.tensor(act, device="cuda")].contiguous()
+        ops.mla_append_gqa_cache(dims, xb, dev["w_dkv_kr"], None, W_UK_g, W_UV_g, sl, tb, gcache)
+        done[act] += step
+    x_new = torch.stack([xt[b, lens[b] - 1:lens[b]] for b in range(w.B)]).contiguous()
+    ops.mla_append_gqa_cache(dims, x_new, dev["w_dkv_kr"], None, W_UK_g, W_UV_g, dev["seqlens"], dev["table"], gcache)
+    out, lse = ops.mla_decode_gqla_grouped(dims, dev["q_nope"], dev["q_rope_raw"], gcache, dev["table"], dev["seqlens"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    Kh, Vh, Rh = (t.double().cpu().numpy() for t in (K, V, R))
+    for b, L in enumerate(lens):
+        p = np.arange(L)
+        idx = case.table[b, p // 64].astype(np.int64) * 64 + p % 64
+        c, kr = O.latent_rows(xs[b][1][:L], case.W64["W_DKV"], case.W64["W_KR"], p)
+        Kr, Vr = O.gqla_expand(as_stored(c, "bf16"), case.W64["W_UK_g"], case.W64["W_UV_g"])
+        _assert_close(Kh[idx], Kr, "bf16", f"expanded keys seq {b}")
+        _assert_close(Vh[idx], Vr, "bf16", f"expanded values seq {b}")
+        _assert_close(Rh[idx], kr, "bf16", f"rope keys seq {b}")
+        q_rot = O.rope(case.q_rope_raw64[b], np.full((1, w.H), L - 1))
+        ref, ref_l = O.gqla_grouped_decode(case.q_nope64[b], q_rot, as_stored(Kr, "bf16"), as_stored(Vr, "bf16"),
+                                           as_stored(kr, "bf16"), L, w.sm_scale, w.g)
+        _assert_close(out[b].double().cpu().numpy(), ref, "bf16", f"grouped out seq {b}")
+        _assert_lse(lse[b].cpu().numpy(), ref_l, "bf16", f"grouped lse seq {b}")
+
+
+@pytest.mark.parametrize("name", ["dsv3_b64_l4096", "smallem_fp32"])
+def test_output_projection_through_preabsorbed_weights(name):
+    """f3: W_UVO[h] = W_UV[h]·W_O[h] built on the GPU, then the layer output straight from the
+    weighted latents, against the oracle's two-step projection (o_lat·W_UV[h], concatenated, ·W_O)."""
+    over = dict(B=3, s_q=1, H=16) if name == "dsv3_b64_l4096" else dict(B=2, s_q=2)
+    w = synth.workload(name, **over)
+    case = Case(w)
+    dev = case.to_device()
+    dims = Dims.of(w)
+    w_uvo = ops.mla_preabsorb_out_weights(dims, dev["W_UV"], dev["W_O"])
+    out_model = ops.mla_out_proj_preabsorbed(dims, dev["o_lat"], w_uvo)
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    ref = O.out_projection(case.o_lat64.reshape(-1, w.H, w.d_c), case.W64["W_UV"], case.W64["W_O"])
+    _assert_close(out_model.double().cpu().numpy().reshape(ref.shape), ref, w.dtype, "layer output")
+    ref_w = O.preabsorbed_out_weights(case.W64["W_UV"], case.W64["W_O"])
+    _assert_close(w_uvo.double().cpu().numpy(), ref_w, w.dtype, "absorbed weights")
 
 
 def test_gqla_ragged_lengths_and_splits():

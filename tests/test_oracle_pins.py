@@ -256,6 +256,38 @@ def test_gqla_grouped_equals_absorbed_on_group_shared_weights():
     assert np.abs(lse_g - lse_a).max() <= 1e-12
 
 
+def test_preabsorbed_output_equals_two_step_projection():
+    """« Chemin MQA-Absorbé »: projecting the weighted latents through W_UV[h]·W_O[h] at once equals
+    projecting each head through W_UV[h], concatenating and projecting through W_O (associativity;
+    the two sides sum in different orders)."""
+    r = _rng(44)
+    s_q, H, d_c, d_v, C = 3, 4, 6, 5, 7
+    o_lat = r.standard_normal((s_q, H, d_c))
+    W_UV = r.standard_normal((H, d_c, d_v))
+    W_O = r.standard_normal((H * d_v, C))
+    two_step = O.out_projection(o_lat, W_UV, W_O)
+    one_step = O.out_projection_preabsorbed(o_lat, O.preabsorbed_out_weights(W_UV, W_O))
+    np.testing.assert_allclose(one_step, two_step, rtol=1e-12, atol=1e-12)
+    # by hand for one output: sum over heads, latents and value columns
+    want = sum(o_lat[1, h, c] * W_UV[h, c, e] * W_O[h * d_v + e, 2]
+               for h in range(H) for c in range(d_c) for e in range(d_v))
+    assert abs(one_step[1, 2] - want) < 1e-12 * max(1.0, abs(want))
+
+
+def test_planted_head_minor_output_blocks_are_caught(monkeypatch):
+    good = O.preabsorbed_out_weights
+
+    def bad(W_UV, W_O):
+        # W_O's rows taken head-minor (row e·H + h) instead of head-major (row h·d_v + e)
+        W_UV = np.asarray(W_UV, float)
+        H, d_c, d_v = W_UV.shape
+        W_Ob = np.asarray(W_O, float).reshape(d_v, H, -1).transpose(1, 0, 2).reshape(H * d_v, -1)
+        return good(W_UV, W_Ob)
+    monkeypatch.setattr(O, "preabsorbed_out_weights", bad)
+    with pytest.raises(AssertionError):
+        test_preabsorbed_output_equals_two_step_projection()
+
+
 def test_merge_of_disjoint_parts_equals_whole():
     L = _layer(seed=21, L=50)
     d_c = L["c"].shape[1]

@@ -72,7 +72,16 @@ CALLS = {
     # B, s_q, q_nope, q_rope_raw, cache, table, max_pages, seqlens, out, lse, ws, ws_bytes, stream
     "mla_decode_gqla_grouped": ([32, 1, P, P, "GC", P, 128, P, P, P, P, BIG_WS, None],
                                 [2, 3, 5, 7, 8, 9], [0, 1, 6], 10, []),
+    # B, s_q, x, C, w_dkv_kr, gamma, w_uk_g, w_uv_g, seqlens, table, max_pages, cache, ws, ws_bytes, stream
+    "mla_append_gqa_cache": ([32, 1, P, 7168, P, P, P, P, P, P, 128, "GC", P, BIG_WS, None],
+                             [2, 4, 6, 7, 8, 9], [0, 1, 3, 10], 12, [5]),
+    # w_uv, w_o, C, w_uvo, stream
+    "mla_preabsorb_out_weights": ([P, P, 7168, P, None], [0, 1, 3], [2], None, []),
+    # B, s_q, o_lat, w_uvo, C, out_model, stream
+    "mla_out_proj_preabsorbed": ([64, 1, P, P, 7168, P, None], [2, 3, 5], [0, 1, 4], None, []),
 }
+# calls without a token count (B, s_q): the overflow check does not apply
+NO_TOKENS = {"mla_preabsorb_out_weights"}
 
 
 def _call(lib, name, args, dims=None, dtype=1):
@@ -123,7 +132,7 @@ def test_bad_dtype_and_dims_are_rejected(lib, name):
         assert _call(lib, name, tmpl, dims=bad) == L.MLA_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("name", list(CALLS))
+@pytest.mark.parametrize("name", [n for n in CALLS if n not in NO_TOKENS])
 def test_token_count_past_int32_is_rejected(lib, name):
     """B * s_q is formed in 32 bits: a product past INT32_MAX is an invalid argument, found before
     any size is computed from it."""
