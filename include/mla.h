@@ -42,6 +42,14 @@
 extern "C" {
 #endif
 
+/* The library exports these calls only (it is built with hidden visibility): two builds loaded in
+ * one process never share internal state. */
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
 enum mla_status {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer or stride */
@@ -99,8 +107,8 @@ typedef struct mla_gqa_cache {
  * workspace: at least mla_append_workspace_size(...) bytes of device memory (fp32 partial sums);
  * its contents need not be initialised.
  * ------------------------------------------------------------------------------------------- */
-size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C);
-int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+MLA_API size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C);
+MLA_API int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                      const void* x, int32_t C, const void* w_dkv_kr, const void* gamma,
                      const int32_t* seqlens, const int32_t* block_table, int32_t max_pages,
                      const mla_latent_cache_t* cache, void* workspace, size_t ws_bytes, void* stream);
@@ -121,7 +129,7 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
  * buffer: calls that overlap on the GPU (streams with no ordering between them) race on it.
  * Nothing in it needs to start at zero.
  * ------------------------------------------------------------------------------------------- */
-int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+MLA_API int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                              const void* x, int32_t C, const void* w_dkv_kr, const void* gamma,
                              const int32_t* seqlens, const int32_t* block_table, int32_t max_pages,
                              const mla_latent_cache_t* cache, void* stream);
@@ -141,8 +149,8 @@ int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, int32_t B, i
  * misaligned pointers and non-positive sizes, MLA_ERR_WORKSPACE, MLA_ERR_CUDA (see the conventions
  * above: the chain enqueues three or four kernels).
  * ------------------------------------------------------------------------------------------- */
-size_t mla_query_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C, int32_t d_q);
-int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+MLA_API size_t mla_query_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C, int32_t d_q);
+MLA_API int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                       const void* x, int32_t C, int32_t d_q, const void* w_dq, const void* gamma_q,
                       const void* w_uq, const void* w_qr, void* q_nope, void* q_rope_raw,
                       void* workspace, size_t ws_bytes, void* stream);
@@ -154,7 +162,7 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
  *   q_nope [B, s_q, H, D]   q_rope_raw [B, s_q, H, d_r]   w_uk [H, D, d_c]   seqlens [B] int32
  *   q_abs  [B, s_q, H, d_c + d_r]   (all dtype)
  * ------------------------------------------------------------------------------------------- */
-int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+MLA_API int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                  const void* q_nope, const void* q_rope_raw, const void* w_uk,
                  const int32_t* seqlens, void* q_abs, void* stream);
 
@@ -170,9 +178,9 @@ int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
  * sequence the table can describe is max_pages*64 positions).
  * Requires every seqlens[b] >= s_q (a token always sees itself).
  * ------------------------------------------------------------------------------------------- */
-size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+MLA_API size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                                  int32_t max_pages);
-int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+MLA_API int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                         const void* q_abs, const mla_latent_cache_t* cache,
                         const int32_t* block_table, int32_t max_pages, const int32_t* seqlens,
                         void* o_lat, float* lse, void* workspace, size_t ws_bytes, void* stream);
@@ -185,7 +193,7 @@ int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_
  *   H*d_v a multiple of 64 and C of 8 this second product runs on the tensor cores too)
  *   o_lat [B, s_q, H, d_c]  w_uv [H, d_c, d_v]  out [B, s_q, H, d_v]  out_model [B, s_q, C] (dtype)
  * ------------------------------------------------------------------------------------------- */
-int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+MLA_API int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                  const void* o_lat, const void* w_uv, void* out,
                  const void* w_o, int32_t C, void* out_model, void* stream);
 
@@ -199,9 +207,9 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
  * Requires every seqlens[b] >= s_q, as a3 does: a sequence shorter than that is reported on the
  * device (MLA_ERR_DEVICE_CHECK) and its outputs are undefined.
  * ------------------------------------------------------------------------------------------- */
-size_t mla_gqla_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+MLA_API size_t mla_gqla_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                                int32_t max_pages);
-int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+MLA_API int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
                             const void* q_nope, const void* q_rope_raw, const mla_gqa_cache_t* cache,
                             const int32_t* block_table, int32_t max_pages, const int32_t* seqlens,
                             void* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
@@ -219,8 +227,8 @@ int mla_decode_gqla_grouped(const mla_dims_t* dims, int32_t dtype, int32_t B, in
  * workspace: at least mla_gqa_append_workspace_size(...) bytes (fp32 partial sums, then c, K and V of
  * the new tokens); contents need not be initialised. The call enqueues five kernels.
  * ------------------------------------------------------------------------------------------- */
-size_t mla_gqa_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C);
-int mla_append_gqa_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x, int32_t C,
+MLA_API size_t mla_gqa_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t C);
+MLA_API int mla_append_gqa_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x, int32_t C,
                          const void* w_dkv_kr, const void* gamma, const void* w_uk_g, const void* w_uv_g,
                          const int32_t* seqlens, const int32_t* block_table, int32_t max_pages,
                          const mla_gqa_cache_t* cache, void* workspace, size_t ws_bytes, void* stream);
@@ -235,9 +243,9 @@ int mla_append_gqa_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32
  * which equals mla_out_proj with w_o up to rounding. Note the weight is H*d_c x C: it pays off only
  * when d_c * H * C is small against the two projections it replaces.
  * ------------------------------------------------------------------------------------------- */
-int mla_preabsorb_out_weights(const mla_dims_t* dims, int32_t dtype, const void* w_uv, const void* w_o, int32_t C,
+MLA_API int mla_preabsorb_out_weights(const mla_dims_t* dims, int32_t dtype, const void* w_uv, const void* w_o, int32_t C,
                               void* w_uvo, void* stream);
-int mla_out_proj_preabsorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* o_lat,
+MLA_API int mla_out_proj_preabsorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* o_lat,
                              const void* w_uvo, int32_t C, void* out_model, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
@@ -249,10 +257,10 @@ int mla_out_proj_preabsorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, i
  * mla_launch_count: kernels this process has launched through the library so far (host counter,
  * incremented at every launch; used to report how many kernels a timed region ran).
  * ------------------------------------------------------------------------------------------- */
-int mla_check_status(void* stream);
-const char* mla_status_string(int status);
-const char* mla_build_info(void);
-uint64_t mla_launch_count(void);
+MLA_API int mla_check_status(void* stream);
+MLA_API const char* mla_status_string(int status);
+MLA_API const char* mla_build_info(void);
+MLA_API uint64_t mla_launch_count(void);
 
 #ifdef __cplusplus
 }

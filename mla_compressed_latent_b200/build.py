@@ -21,6 +21,9 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-Xcompiler", "-fPIC", "-shared",
     "--expt-relaxed-constexpr",
+    # only the C ABI is exported: internal symbols (inline statics, kernels' host stubs) stay private
+    # to each build, so two builds loaded in one process never share state
+    "-Xcompiler", "-fvisibility=hidden",
 ]
 
 

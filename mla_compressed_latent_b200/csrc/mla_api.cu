@@ -163,7 +163,7 @@ uint64_t mla_launch_count(void) { return mla::g_launches.load(std::memory_order_
 #ifdef MLA_TEST_HOOKS
 // Test builds only (not declared in mla.h): makes every per-head GEMM's MMA issuer wait for a phase
 // that nothing completes, so that a test can watch a bounded wait run out on the GPU.
-int mla_test_set_stall(int on) {
+MLA_API int mla_test_set_stall(int on) {
   return cudaMemcpyToSymbol(mla::gemm::g_test_stall, &on, sizeof(int)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 #endif

@@ -38,6 +38,21 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in _declared():
         assert hasattr(lib, name), name
+
+
+def test_library_exports_nothing_else():
+    """Built with hidden visibility: the dynamic symbol table holds the declared C calls and no C++
+    symbol, so two builds loaded in one process (the library and its test-hooks build) cannot bind
+    each other's inline statics (a kernel-attribute cache shared that way made a launch fail)."""
+    import shutil
+    import subprocess
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("nm not available")
+    path = B.build()
+    out = subprocess.run([nm, "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    funcs = sorted(ln.split()[-1] for ln in out.splitlines() if len(ln.split()) == 3 and ln.split()[1] in "TtWw")
+    assert funcs == _declared(), sorted(set(funcs) ^ set(_declared()))
     # and the binding knows each of them with a signature
     assert set(_declared()) <= set(L.SIGNATURES)
 
