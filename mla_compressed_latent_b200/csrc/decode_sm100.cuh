@@ -10,11 +10,12 @@
 //   CTA 0 ("score CTA") keeps Q̃ [128 x 576] bf16 in TMEM (288 columns) as the A operand and
 //         computes S = Q̃ · [c;k_r]ᵀ for 64-position tiles into three TMEM buffers.
 //   CTA 1 ("output CTA") holds O in TMEM and issues O += P · C for each tile.
-// The score CTA's eight row warps turn S into bf16 P (two softmax warps per SM sub-partition: one
-// alone is bound by its own latency) and each tile's P crosses to the output CTA as one bulk DSMEM
-// copy; the output CTA's row warps rescale their rows of O when a running maximum moved (lazily: only
-// past 2^8) and run the epilogue. No FLOP is done twice; each CTA TMA-loads the rows it needs (the
-// second read hits L2).
+// The score CTA's eight row warps turn S into bf16 P: two sets of four warps take alternate tiles, a
+// thread holding a whole row of a tile, so the two warps of an SM sub-partition work on different
+// tiles and their exponentials overlap the other's hand-off; each tile's P crosses to the output CTA
+// as one bulk DSMEM copy. The output CTA's row warps rescale their rows of O when a running maximum
+// moved (lazily: only past 2^8) and run the epilogue. No FLOP is done twice; each CTA TMA-loads the
+// rows it needs (the second read hits L2).
 // Work: the tiles of all sequences are laid end to end and cut into one contiguous range per
 // pair; a sequence cut between pairs is written as fp32 partials and merged afterwards. When the
 // batch has no more sequences than pairs and they are close in length, each pair takes one whole
@@ -38,7 +39,7 @@ constexpr int kKChunks = kRow / 64;                    // 9 chunks per tile on t
 constexpr int kVChunks = kDC / 64;                     // 8 chunks per tile on the output CTA
 constexpr int kGroupChunks = 3;                       // score CTA: a ring of 3-chunk groups (24 KB),
 constexpr int kGroupsPerTile = kKChunks / kGroupChunks;// 3 per tile, each released as soon as its
-constexpr int kRing = 8;                               // 12 MMAs are done
+constexpr int kRing = 7;                               // 12 MMAs are done
 constexpr int kGroupBytes = kGroupChunks * kChunkBytes;// 24576
 constexpr int kQGroups = 6;                            // a sequence's Q̃ travels the ring first: 18 boxes of
                                                        // 64 heads x 64 columns in 6 groups
@@ -69,12 +70,14 @@ constexpr int kStaging = 2;                            // P tiles assembled on t
 static_assert(kCopyBytes <= kSlotStride && kSlotStride % 1024 == 0 && kCopyBytes % 16 == 0, "P slot layout");
 
 // shared memory map (offsets from a 1024-byte aligned base)
-//   score CTA:  K group ring [7] | staging [2]
+//   score CTA:  K group ring [7] | staging [2] | per-tile maxima [2][128] | set sums [2][2][2][128]
 //   output CTA: V stages [2] | P slots [4] | epilogue transpose buffers [8 x 2 KB]
 //   both:       1/l per row (two segments) | barriers | TMEM address | abort flag | work range
 constexpr int kOffK = 0;
 constexpr int kOffStaging = kRing * kGroupBytes;                       // 172032
-constexpr int kRegion0 = kOffStaging + kStaging * kStgStride;         // 205824
+constexpr int kOffDec = kOffStaging + kStaging * kStgStride;          // 205824: float [2][128]
+constexpr int kOffSetSums = kOffDec + 2 * kH * 4;                      // float [2][2][2][128]
+constexpr int kRegion0 = kOffSetSums + 8 * kH * 4;                     // 210944
 constexpr int kOffV = 0;
 constexpr int kOffPSlots = kVStages * kVStageBytes;                    // 131072
 constexpr int kOffEpi = kOffPSlots + kPSlots * kSlotStride;           // 200704
@@ -93,7 +96,7 @@ enum Bar : int {
   K_FULL = 0, K_EMPTY = K_FULL + kRing, S_FULL = K_EMPTY + kRing, S_EMPTY = S_FULL + kSBufs,
   Q_FULL = S_EMPTY + kSBufs, P_EMPTY = Q_FULL + 1, P_WRITTEN = P_EMPTY + kPSlots,
   STG_FREE = P_WRITTEN + kStaging, STATS_EMPTY = STG_FREE + kStaging,
-  V_FULL = STATS_EMPTY + 1, V_EMPTY = V_FULL + kVStages, P_FULL = V_EMPTY + kVStages,
+  DEC_FULL = STATS_EMPTY + 1, V_FULL = DEC_FULL + 2, V_EMPTY = V_FULL + kVStages, P_FULL = V_EMPTY + kVStages,
   P_LOCAL = P_FULL + kPSlots, STATS_FULL = P_LOCAL + kPSlots, NUM_BARS = STATS_FULL + 1
 };
 constexpr int kOffTmemSlot = kOffBar + NUM_BARS * 8;
@@ -122,98 +125,6 @@ struct Params {
   float* part_lse;             // [2 * pairs, 128]
   float sm_scale_log2;         // sm_scale * log2(e)
 };
-
-// One tile of the online softmax for rows r0 and r0 + 8 of a thread (register layout of the 16x256b
-// shape, see above): the exponentials packed as bf16 pairs (pk0 row r0, pk1 row r1; column block j)
-// with their sums added to l, and the lazy update of the running maxima m (rescale factors al, 1 when
-// m did not move). The running maximum moves only when the tile's exceeds it by 2^kRescaleLog2, so
-// the exponentials are first taken against the current m, alongside the tile's maxima (the 4 threads
-// of a row meet by shuffles); only a tile that moves a maximum (the first of a segment, then rarely)
-// takes them again. kMask: the tile has fewer than 64 visible columns.
-template <bool kMask>
-__device__ __forceinline__ void exps_rows(const uint32_t (&sr)[32], int valid, int t4, float scale2, float m0,
-                                          float m1, float& ls_0, float& ls_1, uint32_t (&pk0)[8], uint32_t (&pk1)[8]) {
-  float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int c = 8 * j + 2 * t4;
-    const float e00 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j]), scale2, -m0)) : 0.f;
-    const float e01 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 1]), scale2, -m0)) : 0.f;
-    const float e10 = (!kMask || c < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 2]), scale2, -m1)) : 0.f;
-    const float e11 = (!kMask || c + 1 < valid) ? ptx::ex2_approx(fmaf(__uint_as_float(sr[4 * j + 3]), scale2, -m1)) : 0.f;
-    if (j & 1) {
-      ls1 += e00 + e01;
-      ls3 += e10 + e11;
-    } else {
-      ls0 += e00 + e01;
-      ls2 += e10 + e11;
-    }
-    pk0[j] = ptx::pack_bf16x2(e00, e01);
-    pk1[j] = ptx::pack_bf16x2(e10, e11);
-  }
-  ls_0 = ls0 + ls1;
-  ls_1 = ls2 + ls3;
-}
-
-template <bool kMask>
-__device__ __forceinline__ void softmax_rows(const uint32_t (&sr)[32], int valid, int t4, float scale2, float& m0,
-                                             float& m1, float& l0, float& l1, float& al0, float& al1,
-                                             uint32_t (&pk0)[8], uint32_t (&pk1)[8]) {
-  float ls0, ls1;
-  exps_rows<kMask>(sr, valid, t4, scale2, m0, m1, ls0, ls1, pk0, pk1);
-  float a0 = -INFINITY, a1 = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int c = 8 * j + 2 * t4;
-    if (!kMask || c < valid) {
-      a0 = fmaxf(a0, __uint_as_float(sr[4 * j]));
-      a1 = fmaxf(a1, __uint_as_float(sr[4 * j + 2]));
-    }
-    if (!kMask || c + 1 < valid) {
-      a0 = fmaxf(a0, __uint_as_float(sr[4 * j + 1]));
-      a1 = fmaxf(a1, __uint_as_float(sr[4 * j + 3]));
-    }
-  }
-  a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
-  a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
-  a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 2));
-  a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
-  al0 = 1.f;
-  al1 = 1.f;
-  const float mt0 = a0 * scale2, mt1 = a1 * scale2;
-  const bool up0 = mt0 > m0 + kRescaleLog2, up1 = mt1 > m1 + kRescaleLog2;
-  if (__any_sync(0xffffffffu, up0 || up1)) {
-    if (up0) {
-      al0 = (m0 == -INFINITY) ? 0.f : ptx::ex2_approx(m0 - mt0);
-      l0 *= al0;
-      m0 = mt0;
-    }
-    if (up1) {
-      al1 = (m1 == -INFINITY) ? 0.f : ptx::ex2_approx(m1 - mt1);
-      l1 *= al1;
-      m1 = mt1;
-    }
-    exps_rows<kMask>(sr, valid, t4, scale2, m0, m1, ls0, ls1, pk0, pk1);
-  }
-  l0 += ls0;
-  l1 += ls1;
-}
-
-// A warp's P rows into a P tile at `ptile` (K-major, 128-byte swizzle: row r at (r / 8) * 1024 +
-// (r % 8) * 128, 16-byte chunk j at (j ^ (r % 8)) * 16). The warp's rows are [rw, rw + 16); pk0[j] /
-// pk1[j] are the thread's element pairs of the 8x8 blocks (rows rw + [0, 8) / rw + [8, 16), chunk j),
-// which is exactly the stmatrix fragment layout: four stmatrix.x4 store all sixteen blocks.
-__device__ __forceinline__ void store_p_rows(uint32_t ptile, int rw, int lane, const uint32_t (&pk0)[8],
-                                             const uint32_t (&pk1)[8]) {
-  const int m = lane >> 3, row = rw + (lane & 7) + 8 * (m & 1);
-  const uint32_t row_addr = ptile + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
-  const uint32_t sw = (uint32_t)(row & 7);
-#pragma unroll
-  for (int j = 0; j < 8; j += 2) {
-    const uint32_t chunk = (uint32_t)(j + (m >> 1));
-    ptx::stmatrix_x4(row_addr + ((chunk ^ sw) << 4), pk0[j], pk1[j], pk0[j + 1], pk1[j + 1]);
-  }
-}
 
 // ---- work split -----------------------------------------------------------------------------------
 __device__ __forceinline__ int tiles_of(int L, int max_tiles) { return L > 0 ? min((L + kTile - 1) / kTile, max_tiles) : 0; }
@@ -378,17 +289,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
   if (threadIdx.x == 0) {
     // arrival counts: TMA producers and tcgen05.commit arrive once; thread groups one by one
     for (int i = 0; i < kRing; ++i) { ptx::mbar_init(bar(K_FULL + i), 1); ptx::mbar_init(bar(K_EMPTY + i), 1); }
-    for (int i = 0; i < kSBufs; ++i) { ptx::mbar_init(bar(S_FULL + i), 1); ptx::mbar_init(bar(S_EMPTY + i), kGroup); }
+    for (int i = 0; i < kSBufs; ++i) { ptx::mbar_init(bar(S_FULL + i), 1); ptx::mbar_init(bar(S_EMPTY + i), kH); }
     ptx::mbar_init(bar(Q_FULL), kGroup);
     for (int i = 0; i < kPSlots; ++i) {
       ptx::mbar_init(bar(P_EMPTY + i), 1);
       ptx::mbar_init(bar(P_FULL + i), 1);
       ptx::mbar_init(bar(P_LOCAL + i), kGroup);
     }
-    for (int i = 0; i < kStaging; ++i) { ptx::mbar_init(bar(P_WRITTEN + i), kGroup); ptx::mbar_init(bar(STG_FREE + i), 1); }
+    for (int i = 0; i < kStaging; ++i) { ptx::mbar_init(bar(P_WRITTEN + i), kH); ptx::mbar_init(bar(STG_FREE + i), 1); }
+    for (int i = 0; i < 2; ++i) ptx::mbar_init(bar(DEC_FULL + i), kH);   // one set's 128 row threads
     ptx::mbar_init(bar(STATS_EMPTY), kGroup);
     for (int i = 0; i < kVStages; ++i) { ptx::mbar_init(bar(V_FULL + i), 1); ptx::mbar_init(bar(V_EMPTY + i), 1); }
-    ptx::mbar_init(bar(STATS_FULL), kH / 2);   // one arrival per score-CTA row thread with t % 4 = 0
+    ptx::mbar_init(bar(STATS_FULL), kH);   // one arrival per row (set 0 of the score CTA)
     *reinterpret_cast<volatile int*>(gbase + kOffAbort) = 0;
     ptx::fence_mbar_init();
   }
@@ -528,32 +440,39 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
         }
       }
     } else if (warp >= 4) {
-      // ---- row warps: the softmax of their 16 rows
-      const int g = (warp - 4) >> 2;                      // Q̃ copy: head h, column half g
-      const int h = ((warp & 3) << 5) | lane;
+      // ---- row warps: two sets of four warps take alternate tiles (set = it % 2); in a set, thread =
+      // one head row of its warp's TMEM lane quarter, the whole 64-position row of S in registers
+      // (32x32b loads), so a row's maximum and sum need no shuffle. The lazy running maximum m of a
+      // row moves only when a tile's maximum exceeds it by 2^kRescaleLog2; each tile's decision (m
+      // after the tile) is published for the next tile, which the other set processes. Each set keeps
+      // its own partial row sums, combined at the segment end.
+      const int set = (warp - 4) >> 2;                    // also the Q̃ column half this warp copies
+      const int row = ((warp & 3) << 5) | lane;           // head = TMEM lane
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const uint32_t stats_remote = ptx::map_to_cta(base + kOffStats, 1);
+      float* dec = reinterpret_cast<float*>(gbase + kOffDec);          // [2][128] m after a tile
+      float* part_ml = reinterpret_cast<float*>(gbase + kOffSetSums);  // [2 segments][2 sets][2][128] (m, l)
       uint32_t it = 0, seg = 0, gq = 0;
       bool ok = true;
       while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
         const int L = vlen(b);
-        // Q̃ of this sequence into TMEM columns [0, 288), from the 6 ring groups that carry it (the
-        // previous segment's S MMAs are done: their last result was read below). Half g fills
-        // column blocks [5g, 5 + 4g) of 64 values (32 TMEM columns).
+        // Q̃ of this sequence into TMEM columns [0, 288), from the 6 ring groups that carry it (every
+        // S MMA of the previous segment is done: the row warps met after its last result). Set g
+        // fills column blocks [5g, 5 + 4g) of 64 values (32 TMEM columns).
         {
           bool qok = true;
           for (int qg = 0; qg < kQGroups; ++qg)
             qok = qok && wait_bar_warp(bar(K_FULL + (gq + qg) % kRing), ((gq + qg) / kRing) & 1u, abort_addr, false);
-          if (!qok) { ok = false; break; }
-          const int r = h & 63, rh = h >> 6;
+          ok = ok && qok;   // after a failure every row warp still meets the others at the segment end
+          const int r = row & 63, rh = row >> 6;
 #pragma unroll 1
-          for (int cb = g ? 5 : 0; cb < (g ? 9 : 5); ++cb) {
+          for (int cb = set ? 5 : 0; cb < (set ? 9 : 5) && ok; ++cb) {
             const int qc = 2 * cb + rh, qg = qc / kGroupChunks, j = qc % kGroupChunks;
-            const uint32_t row = base + kOffK + ((gq + qg) % kRing) * kGroupBytes + j * kChunkBytes + r * 128;
+            const uint32_t srow = base + kOffK + ((gq + qg) % kRing) * kGroupBytes + j * kChunkBytes + r * 128;
             uint32_t v[32];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              const uint4 x = ptx::ld_shared_v4(row + ((uint32_t)(k ^ (r & 7)) << 4));
+              const uint4 x = ptx::ld_shared_v4(srow + ((uint32_t)(k ^ (r & 7)) << 4));
               v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
             }
             ptx::tmem_st32(tmem + lane_off + 32u * cb, v);
@@ -563,7 +482,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           // tiles then hands the query groups back to the producer
           gq += kQGroups;
           ptx::tc_fence_before();
-          ptx::mbar_arrive(bar(Q_FULL));
+          if (ok) ptx::mbar_arrive(bar(Q_FULL));
         }
         int nb = -1;
         {
@@ -571,88 +490,115 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           int x0, x1, x2;
           if (!peek.next(p.seqlens, p.B, p.max_tiles, nb, x0, x1, x2)) nb = -1;
         }
-        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         gq += kGroupsPerTile * (t_hi - t_lo);
-        // software pipeline: a tile's scores are read from TMEM while the previous tile's P goes out
-        uint32_t sr[32];
-        if (t_lo < t_hi) {
-          const uint32_t s = it % kSBufs;
-          if (!wait_bar_warp(bar(S_FULL + s), (it / kSBufs) & 1u, abort_addr, false)) { ok = false; break; }
-          ptx::tc_fence_after();
-          ptx::tmem_ld_16x256b_x8(tmem + s_lane + kSCol0 + 64u * s, sr);
-          ptx::tmem_wait_ld_regs(sr);
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(bar(S_EMPTY + s));
-        }
+        float m_own = -INFINITY, l_own = 0.f;   // this set's running maximum and partial row sum
         for (int t = t_lo; t < t_hi; ++t, ++it) {
-          const uint32_t stg = it % kStaging;
+          if ((it & 1u) != (uint32_t)set || !ok) continue;   // the other set's tile (or give up: meet below)
+          const uint32_t sb = it % kSBufs, stg = it % kStaging, sp = it & 1u;
           if (nb >= 0 && t == max(t_lo, t_hi - 3)) {   // the next segment's query row into L2
-            const char* nq = reinterpret_cast<const char*>(p.q_abs + ((size_t)vrow(nb) * kH + h) * kRow);
-            for (int k = g ? 5 : 0; k < (g ? 9 : 5); ++k) ptx::prefetch_l2(nq + 128 * k);
+            const char* nq = reinterpret_cast<const char*>(p.q_abs + ((size_t)vrow(nb) * kH + row) * kRow);
+            for (int k = set ? 5 : 0; k < (set ? 9 : 5); ++k) ptx::prefetch_l2(nq + 128 * k);
           }
           // probe this tile's staging buffer now; the answer is used after the arithmetic
           const bool stg_free = ptx::mbar_test_wait_cluster(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u);
-          uint32_t pk0[8], pk1[8];
-          float al0 = 1.f, al1 = 1.f;
-          const int valid = L - t * kTile;
-          if (valid >= kTile) softmax_rows<false>(sr, kTile, t4, scale2, m0, m1, l0, l1, al0, al1, pk0, pk1);
-          else softmax_rows<true>(sr, valid, t4, scale2, m0, m1, l0, l1, al0, al1, pk0, pk1);
-          // the next tile's scores into the same registers (issued now, waited for after the P store)
-          const bool more = t + 1 < t_hi;
-          const uint32_t sn = (it + 1) % kSBufs;
-          if (more) {
-            if (!wait_bar_warp(bar(S_FULL + sn), ((it + 1) / kSBufs) & 1u, abort_addr, false)) { ok = false; break; }
+          if (!wait_bar_warp(bar(S_FULL + sb), (it / kSBufs) & 1u, abort_addr, false)) { ok = false; continue; }
+          uint32_t v[64];
+          {
+            uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(v);
+            uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(v + 32);
             ptx::tc_fence_after();
-            ptx::tmem_ld_16x256b_x8(tmem + s_lane + kSCol0 + 64u * sn, sr);
+            ptx::tmem_ld32(tmem + lane_off + kSCol0 + 64u * sb, v0);
+            ptx::tmem_ld32(tmem + lane_off + kSCol0 + 64u * sb + 32u, v1);
+            ptx::tmem_wait_ld_regs(v0);
+            ptx::tmem_wait_ld_regs(v1);
           }
-          // this tile's staging buffer must have been copied out (tile it - kStaging)
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar(S_EMPTY + sb));
+          const int valid = L - t * kTile;
+          // the tile's maximum over its visible positions
+          float a4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int j = 0; j < 64; ++j)
+            if (valid >= kTile || j < valid) a4[j & 3] = fmaxf(a4[j & 3], __uint_as_float(v[j]));
+          const float mt = fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3])) * scale2;
+          // m after the previous tile (the other set's decision), then this tile's
+          float m_prev = -INFINITY;
+          if (t > t_lo) {
+            const uint32_t pi = it - 1;
+            if (!wait_bar_warp(bar(DEC_FULL + (pi & 1u)), (pi >> 1) & 1u, abort_addr, true)) { ok = false; continue; }
+            m_prev = dec[(pi & 1u) * kH + row];
+          }
+          float al = 1.f, m_new = m_prev;
+          if (mt > m_prev + kRescaleLog2) {
+            al = (m_prev == -INFINITY) ? 0.f : ptx::ex2_approx(m_prev - mt);
+            m_new = mt;
+          }
+          dec[sp * kH + row] = m_new;
+          ptx::mbar_arrive(bar(DEC_FULL + sp));
+          if (m_new != m_own) {   // this set's partial sum to the new maximum
+            l_own = (m_own == -INFINITY) ? 0.f : l_own * ptx::ex2_approx(m_own - m_new);
+            m_own = m_new;
+          }
+          // exponentials, their sum, bf16 pairs
+          uint32_t pk[32];
+          float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            const bool in0 = valid >= kTile || j < valid, in1 = valid >= kTile || j + 1 < valid;
+            const float x0 = fmaf(__uint_as_float(v[j]), scale2, -m_new);
+            const float x1 = fmaf(__uint_as_float(v[j + 1]), scale2, -m_new);
+            const float e0 = in0 ? ptx::ex2_approx(x0) : 0.f;
+            const float e1 = in1 ? ptx::ex2_approx(x1) : 0.f;
+            ls[(j >> 1) & 3] += e0 + e1;
+            pk[j >> 1] = ptx::pack_bf16x2(e0, e1);
+          }
+          l_own += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          // this tile's staging buffer must have been copied out (this set's tile two before)
           if (!__all_sync(0xffffffffu, stg_free) &&
               !wait_bar_warp(bar(STG_FREE + stg), ((it / kStaging) & 1u) ^ 1u, abort_addr, true)) {
-            if (more) ptx::tmem_wait_ld_regs(sr);
             ok = false;
-            break;
+            continue;
           }
+          // P row into the K-major, 128-byte swizzled tile (row r at (r / 8) * 1024 + (r % 8) * 128,
+          // 16-byte chunk c at (c ^ (r % 8)) * 16), and its rescale factor
           const uint32_t st0 = base + kOffStaging + stg * kStgStride;
-          store_p_rows(st0, 32 * qd + 16 * sub, lane, pk0, pk1);
-          if (t4 == 0) {
-            float* alpha_s = reinterpret_cast<float*>(gbase + kOffStaging + stg * kStgStride + kAlphaOff);
-            alpha_s[r0] = al0;
-            alpha_s[r0 + 8] = al1;
-          }
+          const uint32_t prow = st0 + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            ptx::st_shared_v4(prow + (((uint32_t)c ^ (uint32_t)(row & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                              pk[4 * c + 3]);
+          reinterpret_cast<float*>(gbase + kOffStaging + stg * kStgStride + kAlphaOff)[row] = al;
           // visible to the bulk copy (async proxy), then handed to the copier
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(bar(P_WRITTEN + stg));
-          if (more) {
-            ptx::tmem_wait_ld_regs(sr);
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(bar(S_EMPTY + sn));
-          }
         }
-        if (!ok) break;
-        {
-          // segment end: each row's sum over its four threads; 1/l to the output CTA, lse to memory
-          l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-          l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-          l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-          l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-          if (!wait_bar_warp(bar(STATS_EMPTY), (seg & 1u) ^ 1u, abort_addr, true)) { ok = false; break; }
-          if (t4 == 0) {
+        // segment end: the two sets' partial sums combined. All row warps meet here (and agree
+        // whether to go on); after it, every S MMA of the segment is known to be done.
+        float* pml = part_ml + (seg & 1u) * 4 * kH;   // by segment parity: a set may run one segment ahead
+        pml[(set * 2) * kH + row] = m_own;
+        pml[(set * 2 + 1) * kH + row] = l_own;
+        if (ptx::named_bar_or(2, kGroup, !ok)) { ok = false; break; }
+        if (set == 0) {
+          const float m1 = pml[2 * kH + row], l1 = pml[3 * kH + row];
+          const float m_fin = fmaxf(m_own, m1);
+          float l = 0.f;
+          if (m_own != -INFINITY) l += l_own * ptx::ex2_approx(m_own - m_fin);
+          if (m1 != -INFINITY) l += l1 * ptx::ex2_approx(m1 - m_fin);
+          if (!wait_bar_warp(bar(STATS_EMPTY), (seg & 1u) ^ 1u, abort_addr, true)) ok = false;
+          if (ok) {
             const bool partial = !(t_lo == 0 && t_hi == tiles_b);
             float* lse_dst = partial ? p.part_lse + ((size_t)pair * 2 + (seg > 0)) * kH : p.lse + (size_t)vrow(b) * kH;
             // a segment with no visible position (a token's masked last tile alone) has l = 0:
             // lse -inf and a zero part, which the merge weighs by 0
-            lse_dst[r0] = (m0 + log2f(l0)) * 0.69314718055994531f;
-            lse_dst[r0 + 8] = (m1 + log2f(l1)) * 0.69314718055994531f;
-            const uint32_t st = stats_remote;
-            ptx::st_cluster_f32(st + r0 * 4u, l0 > 0.f ? 1.f / l0 : 0.f);
-            ptx::st_cluster_f32(st + (r0 + 8) * 4u, l1 > 0.f ? 1.f / l1 : 0.f);
+            lse_dst[row] = (m_fin + log2f(l)) * 0.69314718055994531f;
+            ptx::st_cluster_f32(stats_remote + row * 4u, l > 0.f ? 1.f / l : 0.f);
             ptx::mbar_arrive_remote(bar(STATS_FULL), 1);
           }
         }
         ++seg;
       }
       // before leaving: the output CTA's last release of the stats must have landed here
-      if (t4 == 0 && seg > 0) wait_bar(bar(STATS_EMPTY), (seg - 1) & 1u, abort_addr, true, false);
+      if (set == 0 && seg > 0) wait_bar(bar(STATS_EMPTY), (seg - 1) & 1u, abort_addr, true, false);
     }
   } else {
     // ============================== output CTA ==============================
