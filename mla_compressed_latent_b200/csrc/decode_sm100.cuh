@@ -39,7 +39,7 @@ constexpr int kKChunks = kRow / 64;                    // 9 chunks per tile on t
 constexpr int kVChunks = kDC / 64;                     // 8 chunks per tile on the output CTA
 constexpr int kGroupChunks = 3;                       // score CTA: a ring of 3-chunk groups (24 KB),
 constexpr int kGroupsPerTile = kKChunks / kGroupChunks;// 3 per tile, each released as soon as its
-constexpr int kRing = 7;                               // 12 MMAs are done
+constexpr int kRing = 8;                               // 12 MMAs are done
 constexpr int kGroupBytes = kGroupChunks * kChunkBytes;// 24576
 constexpr int kQGroups = 6;                            // a sequence's Q̃ travels the ring first: 18 boxes of
                                                        // 64 heads x 64 columns in 6 groups
@@ -70,22 +70,22 @@ constexpr int kStaging = 2;                            // P tiles assembled on t
 static_assert(kCopyBytes <= kSlotStride && kSlotStride % 1024 == 0 && kCopyBytes % 16 == 0, "P slot layout");
 
 // shared memory map (offsets from a 1024-byte aligned base)
-//   score CTA:  K group ring [7] | staging [2] | per-tile maxima [2][128] | set sums [2][2][2][128]
+//   score CTA:  K group ring [8] | staging [2]
 //   output CTA: V stages [2] | P slots [4] | epilogue transpose buffers [8 x 2 KB]
 //   both:       1/l per row (two segments) | barriers | TMEM address | abort flag | work range
 constexpr int kOffK = 0;
-constexpr int kOffStaging = kRing * kGroupBytes;                       // 172032
-constexpr int kOffDec = kOffStaging + kStaging * kStgStride;          // 205824: float [2][128]
-constexpr int kOffSetSums = kOffDec + 2 * kH * 4;                      // float [2][2][2][128]
-constexpr int kRegion0 = kOffSetSums + 8 * kH * 4;                     // 210944
+constexpr int kOffStaging = kRing * kGroupBytes;                       // 196608
+constexpr int kRegion0 = kOffStaging + kStaging * kStgStride;         // 230400
 constexpr int kOffV = 0;
 constexpr int kOffPSlots = kVStages * kVStageBytes;                    // 131072
 constexpr int kOffEpi = kOffPSlots + kPSlots * kSlotStride;           // 200704
 constexpr int kEpiWarpBytes = 2048;
 constexpr int kRegion1 = kOffEpi + 8 * kEpiWarpBytes;                 // 217088
 constexpr int kRegion = kRegion0 > kRegion1 ? kRegion0 : kRegion1;
-// float [128] 1/l per row (output CTA). One buffer is enough: the score CTA writes a segment's
-// values only after the output CTA released the previous segment's (STATS_EMPTY).
+// float [128] per row. Output CTA: 1/l (one buffer is enough: the score CTA writes a segment's values
+// only after the output CTA released the previous segment's, STATS_EMPTY). Score CTA: the running
+// maximum after the latest tile, handed from one softmax set to the other; at a segment end, set 1's
+// partial row sums.
 constexpr int kOffStats = kRegion;
 constexpr int kOffBar = kOffStats + kH * 4;
 // Barriers. Score CTA: K_*, S_*, Q_FULL, P_EMPTY, P_WRITTEN, STG_FREE, STATS_EMPTY. Output CTA:
@@ -96,7 +96,7 @@ enum Bar : int {
   K_FULL = 0, K_EMPTY = K_FULL + kRing, S_FULL = K_EMPTY + kRing, S_EMPTY = S_FULL + kSBufs,
   Q_FULL = S_EMPTY + kSBufs, P_EMPTY = Q_FULL + 1, P_WRITTEN = P_EMPTY + kPSlots,
   STG_FREE = P_WRITTEN + kStaging, STATS_EMPTY = STG_FREE + kStaging,
-  DEC_FULL = STATS_EMPTY + 1, V_FULL = DEC_FULL + 2, V_EMPTY = V_FULL + kVStages, P_FULL = V_EMPTY + kVStages,
+  DEC_FULL = STATS_EMPTY + 1, V_FULL = DEC_FULL + 1, V_EMPTY = V_FULL + kVStages, P_FULL = V_EMPTY + kVStages,
   P_LOCAL = P_FULL + kPSlots, STATS_FULL = P_LOCAL + kPSlots, NUM_BARS = STATS_FULL + 1
 };
 constexpr int kOffTmemSlot = kOffBar + NUM_BARS * 8;
@@ -297,7 +297,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
       ptx::mbar_init(bar(P_LOCAL + i), kGroup);
     }
     for (int i = 0; i < kStaging; ++i) { ptx::mbar_init(bar(P_WRITTEN + i), kH); ptx::mbar_init(bar(STG_FREE + i), 1); }
-    for (int i = 0; i < 2; ++i) ptx::mbar_init(bar(DEC_FULL + i), kH);   // one set's 128 row threads
+    ptx::mbar_init(bar(DEC_FULL), kH);   // one set's 128 row threads, once per tile
     ptx::mbar_init(bar(STATS_EMPTY), kGroup);
     for (int i = 0; i < kVStages; ++i) { ptx::mbar_init(bar(V_FULL + i), 1); ptx::mbar_init(bar(V_EMPTY + i), 1); }
     ptx::mbar_init(bar(STATS_FULL), kH);   // one arrival per row (set 0 of the score CTA)
@@ -318,14 +318,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
   if (warp == 3) plan_range(p.seqlens, p.B, p.s_q, p.max_tiles, pair, npairs, work);
   ptx::tc_fence_before();
   __syncthreads();
-  // (no early allow_dependents(): the merge that follows would park its blocks on these SMs)
+  // (allow_dependents() only at the end: the merge that follows would park its blocks on these SMs)
   ptx::cluster_sync();      // the peer's barriers are initialised before any remote arrive
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffTmemSlot);
   SegIter segs{work[0], work[1], work[2], (int)work[3]};
   int b, t_lo, t_hi, tiles_b;
   // row-warp geometry (warps 4-11)
-  const int qd = warp & 3, sub = (warp - 4) >> 2, t4 = lane & 3;
+  const int qd = warp & 3, sub = (warp - 4) >> 2;
   const int r0 = 32 * qd + 16 * sub + (lane >> 2);                       // and r0 + 8
   const uint32_t s_lane = (uint32_t)(32 * qd + 16 * sub) << 16;          // TMEM lane field of the warp
   const float scale2 = p.sm_scale_log2;
@@ -450,8 +450,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
       const int row = ((warp & 3) << 5) | lane;           // head = TMEM lane
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const uint32_t stats_remote = ptx::map_to_cta(base + kOffStats, 1);
-      float* dec = reinterpret_cast<float*>(gbase + kOffDec);          // [2][128] m after a tile
-      float* part_ml = reinterpret_cast<float*>(gbase + kOffSetSums);  // [2 segments][2 sets][2][128] (m, l)
+      float* dec = reinterpret_cast<float*>(gbase + kOffStats);   // [128]: m after the latest tile
       uint32_t it = 0, seg = 0, gq = 0;
       bool ok = true;
       while (ok && segs.next(p.seqlens, p.B, p.max_tiles, b, t_lo, t_hi, tiles_b)) {
@@ -494,7 +493,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
         float m_own = -INFINITY, l_own = 0.f;   // this set's running maximum and partial row sum
         for (int t = t_lo; t < t_hi; ++t, ++it) {
           if ((it & 1u) != (uint32_t)set || !ok) continue;   // the other set's tile (or give up: meet below)
-          const uint32_t sb = it % kSBufs, stg = it % kStaging, sp = it & 1u;
+          const uint32_t sb = it % kSBufs, stg = it % kStaging;
           if (nb >= 0 && t == max(t_lo, t_hi - 3)) {   // the next segment's query row into L2
             const char* nq = reinterpret_cast<const char*>(p.q_abs + ((size_t)vrow(nb) * kH + row) * kRow);
             for (int k = set ? 5 : 0; k < (set ? 9 : 5); ++k) ptx::prefetch_l2(nq + 128 * k);
@@ -523,18 +522,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           const float mt = fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3])) * scale2;
           // m after the previous tile (the other set's decision), then this tile's
           float m_prev = -INFINITY;
-          if (t > t_lo) {
-            const uint32_t pi = it - 1;
-            if (!wait_bar_warp(bar(DEC_FULL + (pi & 1u)), (pi >> 1) & 1u, abort_addr, true)) { ok = false; continue; }
-            m_prev = dec[(pi & 1u) * kH + row];
+          if (t > t_lo) {   // phase it - 1 of DEC_FULL: the previous tile's decision (one slot: each
+                            // tile's set reads its predecessor's value before writing its own)
+            if (!wait_bar_warp(bar(DEC_FULL), (it - 1) & 1u, abort_addr, true)) { ok = false; continue; }
+            m_prev = dec[row];
           }
           float al = 1.f, m_new = m_prev;
           if (mt > m_prev + kRescaleLog2) {
             al = (m_prev == -INFINITY) ? 0.f : ptx::ex2_approx(m_prev - mt);
             m_new = mt;
           }
-          dec[sp * kH + row] = m_new;
-          ptx::mbar_arrive(bar(DEC_FULL + sp));
+          dec[row] = m_new;
+          ptx::mbar_arrive(bar(DEC_FULL));
           if (m_new != m_own) {   // this set's partial sum to the new maximum
             l_own = (m_own == -INFINITY) ? 0.f : l_own * ptx::ex2_approx(m_own - m_new);
             m_own = m_new;
@@ -572,18 +571,23 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(bar(P_WRITTEN + stg));
         }
-        // segment end: the two sets' partial sums combined. All row warps meet here (and agree
-        // whether to go on); after it, every S MMA of the segment is known to be done.
-        float* pml = part_ml + (seg & 1u) * 4 * kH;   // by segment parity: a set may run one segment ahead
-        pml[(set * 2) * kH + row] = m_own;
-        pml[(set * 2 + 1) * kH + row] = l_own;
+        // segment end: the two sets' partial sums combined at the maximum after the segment's last
+        // tile (the set that did not process that tile reads its decision), set 1's sums handed to set
+        // 0 through the same slot. All row warps meet here (and agree whether to go on); after it,
+        // every S MMA of the segment is known to be done.
+        float m_fin = -INFINITY;
+        if (ok && t_hi > t_lo) {
+          const uint32_t last = it - 1;
+          if ((last & 1u) == (uint32_t)set) m_fin = m_own;
+          else if (wait_bar_warp(bar(DEC_FULL), last & 1u, abort_addr, true)) m_fin = dec[row];
+          else ok = false;
+        }
+        const float l_fin = (m_own == -INFINITY) ? 0.f : l_own * ptx::ex2_approx(m_own - m_fin);
         if (ptx::named_bar_or(2, kGroup, !ok)) { ok = false; break; }
+        if (set == 1) dec[row] = l_fin;
+        ptx::named_bar_sync(2, kGroup);
         if (set == 0) {
-          const float m1 = pml[2 * kH + row], l1 = pml[3 * kH + row];
-          const float m_fin = fmaxf(m_own, m1);
-          float l = 0.f;
-          if (m_own != -INFINITY) l += l_own * ptx::ex2_approx(m_own - m_fin);
-          if (m1 != -INFINITY) l += l1 * ptx::ex2_approx(m1 - m_fin);
+          const float l = l_fin + dec[row];
           if (!wait_bar_warp(bar(STATS_EMPTY), (seg & 1u) ^ 1u, abort_addr, true)) ok = false;
           if (ok) {
             const bool partial = !(t_lo == 0 && t_hi == tiles_b);
@@ -796,9 +800,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
     }
   }
 
-  // teardown: TMEM back, then leave together so no remote access can target an exited CTA
+  // teardown: TMEM back, then leave together so no remote access can target an exited CTA. The
+  // merge that follows may be scheduled from here on (it waits for this grid's completion and its
+  // writes before reading anything), so its launch overlaps the last CTAs' exit.
   ptx::tc_fence_before();
   __syncthreads();
+  allow_dependents();
   if (warp == 2) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);

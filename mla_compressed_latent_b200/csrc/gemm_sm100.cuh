@@ -150,18 +150,19 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
     }
     // every load issued must land before the CTA may exit (waited for even after a give-up)
     for (int k = (i > S ? i - S : 0); k < i; ++k) wait(full0 + 8u * (k % S), (k / S) & 1u);
-  } else if (warp == 1) {
-    // ---- MMA issuer: M = 128, N = tn, four K = 16 steps per chunk; the warp waits, an elected lane issues
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer: M = 128, N = tn, four K = 16 steps per chunk (one thread: with two to four K
+    // chunks per CTA at decode batch sizes, a warp-wide wait costs more than the issue rate gains)
     const uint32_t idesc = ptx::idesc_bf16_f32_ab(kBM, p.tn, !p.a_kmajor, false);
     bool live = true;
 #ifdef MLA_TEST_HOOKS
     // phase 0 of `done` completes only through this warp's own commit below: nothing else can end the wait
-    if (g_test_stall) live = __all_sync(0xffffffffu, wait(done, 0u, nullptr, 10000000ull));
+    if (g_test_stall) live = wait(done, 0u, nullptr, 10000000ull);
 #endif
     for (int i = 0; i < nk && live; ++i) {
       const int s = i % S;
-      if (!__all_sync(0xffffffffu, wait(full0 + 8u * s, (i / S) & 1u))) { live = false; break; }
-      if (ptx::elect_one()) {
+      if (!wait(full0 + 8u * s, (i / S) & 1u)) { live = false; break; }
+      {
         ptx::tc_fence_after();
         const uint32_t st = ring + s * sbytes;
         // A, MN-major: 8-row K groups 1024 B apart (SBO), the two 64-feature halves one box apart (LBO);
@@ -176,11 +177,9 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
           ptx::mma_ss(tmem, ad + (uint64_t)k * a_step, bd + (uint64_t)(2 * k), idesc, (i | k) ? 1u : 0u);
         ptx::mma_commit(empty0 + 8u * s);
       }
-      __syncwarp();
     }
-    if (!live && lane == 0) *abort = 1;   // the producer stops waiting for stages that will not be freed
-    if (ptx::elect_one()) ptx::mma_commit(done);
-    __syncwarp();
+    if (!live) *abort = 1;   // the producer stops waiting for stages that will not be freed
+    ptx::mma_commit(done);
   } else if (warp >= 4) {
     // ---- epilogue: thread = output feature (TMEM lane), 32 tokens (TMEM columns) per load
     const int row = threadIdx.x - 128;

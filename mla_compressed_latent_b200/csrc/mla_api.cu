@@ -228,7 +228,7 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     p.mode = 1;
     p.part = reinterpret_cast<float*>(workspace);
     if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, ks}), p, st))) return rc;
-    const int fin_threads = std::max(64, std::min(1024, (N / 4 + 31) / 32 * 32));   // four columns per thread
+    const int fin_threads = std::min(1024, (N + 31) / 32 * 32);   // one thread per output column
     mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)p.part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
            (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0);
@@ -644,7 +644,7 @@ int mla_append_gqa_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32
   if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, lay.ks}), p, st))) return rc;
   // 2. c = RMSNorm(z_c)·gamma into a plain buffer (rounded to the storage type, as a latent cache row
   //    would be); k_r = RoPE(z_r) into the cache's RoPE rows
-  const int fin_threads = std::max(64, std::min(1024, (N / 4 + 31) / 32 * 32));
+  const int fin_threads = std::min(1024, (N + 31) / 32 * 32);
   mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)part,
                   lay.ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
                   block_table, max_pages, cbuf, (int64_t)dims->d_c, (T*)cache->rope, cache->rope_stride,
@@ -811,7 +811,7 @@ extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, i
     p.mode = 1;
     p.part = part;
     if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, ks}), p, st))) return rc;
-    const int fin_threads = std::max(64, std::min(1024, (N / 4 + 31) / 32 * 32));
+    const int fin_threads = std::min(1024, (N + 31) / 32 * 32);
     mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st,
                     (const float*)part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps,
                     dims->rope_base, seqlens, block_table, max_pages, (T*)cache->latent, cache->latent_stride,

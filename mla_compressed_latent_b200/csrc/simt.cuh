@@ -72,8 +72,8 @@ __device__ __forceinline__ float sum_slices(const float* src, int ksplit, int64_
 
 // =============================================================================================
 // a1 epilogue: sum the K slices, RMSNorm the latent part, rotate the RoPE part, store the row.
-// One block per new token. The partial sums are read 16 bytes at a time (4 columns per thread and
-// slice, several slices in flight) and the latent row is written 16 bytes at a time. With
+// One block per new token (a thread per column sums that column's K slices, many loads in flight);
+// the latent row is written 16 bytes at a time. With
 // latent_by_token the latent row of token tok goes to latent + tok * lat_stride (a plain buffer)
 // instead of its cache slot; the RoPE key always goes to its cache slot.
 // =============================================================================================
@@ -112,31 +112,9 @@ __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit,
   const int tok = blockIdx.x;
   const int b = tok / s_q, t = tok % s_q;
   const int N = d_c + d_r;
-  if ((N & 3) == 0) {
-    const float4* src = reinterpret_cast<const float4*>(part + (int64_t)tok * N);
-    const int64_t step4 = (int64_t)n_tok * N / 4;
-    for (int i4 = threadIdx.x; i4 < N / 4; i4 += blockDim.x) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      int ks = 0;
-      for (; ks + 4 <= ksplit; ks += 4) {
-        float4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) v[u] = src[(ks + u) * step4 + i4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
-        }
-      }
-      for (; ks < ksplit; ++ks) {
-        const float4 v = src[ks * step4 + i4];
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
-      z[4 * i4] = acc.x; z[4 * i4 + 1] = acc.y; z[4 * i4 + 2] = acc.z; z[4 * i4 + 3] = acc.w;
-    }
-  } else {
-    for (int i = threadIdx.x; i < N; i += blockDim.x)
-      z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
-  }
+  // one column per thread, up to 32 slices' loads in flight per thread
+  for (int i = threadIdx.x; i < N; i += blockDim.x)
+    z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
   __syncthreads();
   float ss = 0.f;
   for (int i = threadIdx.x; i < d_c; i += blockDim.x) ss = fmaf(z[i], z[i], ss);
