@@ -44,6 +44,9 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="bound on the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-secondary", action="store_true", help="skip the other configurations' decode timings")
+    p.add_argument("--decode-only", action="store_true",
+                   help="time the workload's decode call alone (inputs drawn on the GPU) and print its line; "
+                        "a per-configuration diagnostic, not the whole step")
     return p.parse_args()
 
 
@@ -656,6 +659,23 @@ def main():
 
     w = synth.workload(args.workload)
     dims = Dims.of(w)
+    if args.decode_only:
+        peaks, peak_kind = load_peaks()
+        with ClockSampler(local) as clk:
+            r = time_decode_alone(w.name, device, args.steps, args.warmup, peaks)
+        ms = max_over_ranks(r["decode_us"] / 1e3, world, device)
+        r["roofline"]["peak_source"] = peak_kind
+        line = {"metric": METRIC, "value": world * r["positions_per_s"] * (r["decode_us"] / 1e3) / ms, "unit": UNIT,
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+                "config": {"workload": w.name, **r["config"], "step": "the decode call alone"},
+                "tokens_per_s": world * r["tokens_per_s"] * (r["decode_us"] / 1e3) / ms, "decode_us": r["decode_us"],
+                "roofline": r["roofline"], "clocks": clk.summary()}
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
     if w.g:
         return run_grouped(args, w, dims, device, world, rank, local)
     dev = build_inputs(w, device)
