@@ -73,6 +73,20 @@ def quantize_rows(c):
     return codes, scale
 
 
+def quantize_rows_f32(c):
+    """The same quantisation with the arithmetic that decides each code done in float32, the
+    precision a kernel takes that decision in: s_j = fl32(max|c_j| / 448) and code = the nearest
+    E4M3 value of fl32(c_j / s_j), each operation rounded once to float32. `c` holds
+    float32-representable values (bf16 rows are). Returns (codes uint8 [n, d_c], scales [n] as the
+    float32 values, widened)."""
+    c32 = np.asarray(c, np.float32)
+    amax = np.abs(c32).max(axis=1)
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    quot = (c32 / safe[:, None]).astype(np.float32)
+    return e4m3_encode(quot.astype(f64)), scale.astype(f64)
+
+
 def dequantize_rows(codes, scale):
     return e4m3_decode(codes) * np.asarray(scale, f64)[:, None]
 

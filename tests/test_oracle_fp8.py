@@ -80,6 +80,40 @@ def test_decode_over_the_8bit_cache_stays_close_to_the_16bit_one():
     assert np.abs(l8 - l).max() < 0.05
 
 
+def test_float32_decision_equals_the_exact_one_where_no_rounding_intervenes():
+    """Rows whose largest magnitude is 448·2^k and whose values are E4M3 values times 2^k: the scale
+    2^k and every quotient are exact in float32, so both quantisations give the same codes, and
+    dequantising gives the rows back."""
+    r = np.random.default_rng(53)
+    codes = r.integers(0, 0x7F, (16, 512)).astype(np.uint8) | (r.integers(0, 2, (16, 512)).astype(np.uint8) << 7)
+    codes[:, 0] = 0x7E                                     # each row reaches 448
+    k = r.integers(-20, 20, 16)
+    c = F.e4m3_decode(codes) * np.ldexp(1.0, k)[:, None]
+    c32, s32 = F.quantize_rows_f32(c)
+    c64, s64 = F.quantize_rows(c)
+    assert np.array_equal(s32, np.ldexp(1.0, k)) and np.array_equal(s32, s64)
+    assert np.array_equal(F.e4m3_decode(c32), F.e4m3_decode(c64))   # +0 and -0 may differ as codes
+    np.testing.assert_array_equal(F.dequantize_rows(c32, s32), c)
+
+
+def test_float32_decision_differs_from_the_exact_one_only_at_ties():
+    """On bf16-valued random rows the two precisions agree except where the exact quotient lies within
+    a float32 rounding of a midpoint between two E4M3 values (a tie that float32 can move)."""
+    r = np.random.default_rng(54)
+    c = torch.from_numpy(r.standard_normal((256, 512)) * r.uniform(0.01, 30, (256, 1))).to(torch.bfloat16)
+    c = c.to(torch.float64).numpy()
+    c32, s32 = F.quantize_rows_f32(c)
+    c64, s64 = F.quantize_rows(c)
+    np.testing.assert_allclose(s32, s64, rtol=2.0 ** -24)
+    diff = F.e4m3_decode(c32) != F.e4m3_decode(c64)
+    assert diff.mean() < 1e-3
+    if diff.any():
+        exact = np.abs(c / s64[:, None])[diff]
+        v32, v64 = np.abs(F.e4m3_decode(c32)[diff]), np.abs(F.e4m3_decode(c64)[diff])
+        mid = (v32 + v64) / 2                                # the two candidates are neighbours
+        assert (np.abs(exact - mid) <= 2.0 ** -22 * mid).all()
+
+
 # planted slips ------------------------------------------------------------------------------
 
 def test_planted_wrong_exponent_bias_is_caught(monkeypatch):
