@@ -32,6 +32,9 @@ UNIT = "positions/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # nominal B200 figures (context for the measured fractions): HBM3e ~8 TB/s, dense bf16 2.25 PFLOP/s
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+# fp32 FMA throughput of the CUDA cores (the roof of a kernel that does its contractions there):
+# 148 SMs x 128 fp32 lanes x 2 FLOPs per FMA x 1965 MHz (the maximum SM clock)
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def parse():
@@ -104,7 +107,10 @@ def decode_counts(w, lens):
     total = int(sum(int(L) for L in lens))
     e = 2 if w.dtype == "bf16" else 4
     n_tok = w.B * w.s_q
-    bytes_ = total * (w.d_c + w.d_r) * e + n_tok * w.H * ((w.d_c + w.d_r) + w.d_c) * e + n_tok * w.H * 4
+    # a cached row: the latent in e bytes per value (or one E4M3 byte plus a 4-byte scale per row),
+    # the RoPE key in e bytes per value
+    row = (w.d_c * e if getattr(w, "latent_bits", 16) == 16 else w.d_c + 4) + w.d_r * e
+    bytes_ = total * row + n_tok * w.H * ((w.d_c + w.d_r) + w.d_c) * e + n_tok * w.H * 4
     visible = sum(int(L) * w.s_q - w.s_q * (w.s_q - 1) // 2 for L in lens)
     flops = 2 * w.H * (2 * w.d_c + w.d_r) * visible
     return bytes_, flops, total
@@ -340,7 +346,7 @@ def build_inputs(w, device):
 
 # configurations whose decode call the default run also times on its own: long-context split-KV,
 # the GQLA grouped path, multi-token steps with 2 and 4 new tokens
-SECONDARY = ("longctx_b8", "gqla_g8_b32_l8192", "mtp_sq2_b128", "mtp_sq4_b128")
+SECONDARY = ("longctx_b8", "gqla_g8_b32_l8192", "mtp_sq2_b128", "mtp_sq4_b128", "dsv3_fp8_b64_l4096")
 
 
 def run_e2e(args, w, dev, step, out, stream, device, world, from_x, e_steps):
@@ -493,13 +499,30 @@ def time_decode_alone(name, device, steps, warmup, peaks):
         q_abs = q_abs.to(torch.bfloat16)
         o_lat = torch.empty(w.B, w.s_q, w.H, w.d_c, dtype=torch.bfloat16, device=device)
         lse = torch.empty(w.B, w.s_q, w.H, dtype=torch.float32, device=device)
-        ws = torch.empty(max(16, ops.mla_decode_workspace_size(dims, torch.bfloat16, w.B, w.s_q, table.shape[1])),
-                         dtype=torch.uint8, device=device)
-
-        def call():
-            ops.mla_decode_absorbed(dims, q_abs, cache, tbl, seqlens, o_lat=o_lat, lse=lse, workspace=ws)
         bytes_, flops, _ = decode_counts(w, lens)
-        kernel = "mla_decode_absorbed (decode + split merge)"
+        if w.latent_bits == 8:
+            # the 16-bit pool converted once by the library's quantiser; the RoPE keys stay 16-bit
+            from mla_compressed_latent_b200.ops import LatentCacheFp8
+            cache8 = LatentCacheFp8.empty_like(cache)
+            ops.mla_quantize_latent_fp8(dims, cache.latent, cache8.codes, cache8.scales)
+            del pool, cache
+            import ctypes
+            from mla_compressed_latent_b200 import _lib as L
+            dc = dims.c()
+            ws = torch.empty(max(16, int(L.load().mla_decode_fp8_workspace_size(ctypes.byref(dc), w.B, w.s_q,
+                                                                                 table.shape[1]))),
+                             dtype=torch.uint8, device=device)
+
+            def call():
+                ops.mla_decode_absorbed_fp8(dims, q_abs, cache8, tbl, seqlens, o_lat=o_lat, lse=lse, workspace=ws)
+            kernel = "mla_decode_absorbed_fp8 (CUDA-core decode + split merge)"
+        else:
+            ws = torch.empty(max(16, ops.mla_decode_workspace_size(dims, torch.bfloat16, w.B, w.s_q, table.shape[1])),
+                             dtype=torch.uint8, device=device)
+
+            def call():
+                ops.mla_decode_absorbed(dims, q_abs, cache, tbl, seqlens, o_lat=o_lat, lse=lse, workspace=ws)
+            kernel = "mla_decode_absorbed (decode + split merge)"
     for _ in range(warmup):
         call()
     torch.cuda.synchronize()
@@ -515,7 +538,11 @@ def time_decode_alone(name, device, steps, warmup, peaks):
     sec = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
     gbs, tfs = bytes_ / sec / 1e9, flops / sec / 1e12
     t_hbm, t_tc = bytes_ / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)
-    if t_tc > t_hbm:
+    if getattr(w, "latent_bits", 16) == 8:   # the 8-bit decode runs its contractions on the CUDA cores
+        roof = {"bound": "alu", "achieved": tfs, "peak": ALU_FP32_TFLOPS, "unit": "TFLOP/s",
+                "frac": tfs / ALU_FP32_TFLOPS, "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                "peak_note": "fp32 FMA of 148 SMs x 128 lanes at 1965 MHz"}
+    elif t_tc > t_hbm:
         roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": tfs / peaks["bf16_tflops"],
                 "frac_sustained": tfs / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
@@ -524,7 +551,6 @@ def time_decode_alone(name, device, steps, warmup, peaks):
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm_gbs"], "frac_nominal": gbs / NOMINAL_PEAKS["hbm_gbs"], "tensor_tflops": tfs}
     roof.update({"traffic": None, "kernel": kernel, "bytes_per_launch": bytes_, "flops_per_launch": flops})
-    del cache
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return {"decode_us": sec * 1e6, "positions_per_s": total / sec, "tokens_per_s": n_tok / sec,

@@ -249,6 +249,46 @@ MLA_API int mla_out_proj_preabsorbed(const mla_dims_t* dims, int32_t dtype, int3
                              const void* w_uvo, int32_t C, void* out_model, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * 8-bit latent cache (« Cache KV, mémoire récurrente, MLA et bas rang », trainer notes of « Le
+ * problème — Cache KV standard »: one byte per cached value instead of two). Only the latent rows
+ * are narrowed; the RoPE keys stay in dtype. Each latent row j is stored as FP8 E4M3 codes (1 sign,
+ * 4 exponent bits of bias 7, 3 mantissa bits, subnormals, largest finite value 448) with one fp32
+ * scale s_j = max|c_j| / 448:
+ *   code_j = E4M3(c_j / s_j), round to nearest, ties to even, saturated at +-448 (s_j and the
+ *   quotients computed in fp32, each rounded once); a zero row stores s_j = 0 and zero codes.
+ * The decode attends the dequantised rows s_j * value(code_j) exactly as mla_decode_absorbed attends
+ * 16-bit rows (same q_abs, o_lat, lse, seqlens and table conventions).
+ *
+ * mla_quantize_latent_fp8: rows [0, rows) of `latent` (dtype, row stride `latent_stride` elements,
+ *   >= d_c) into codes [rows, d_c] (uint8, row stride `code_stride` bytes, >= d_c, multiple of 16)
+ *   and scales [rows] (fp32). Any row range of a pool can be converted (for example the rows that
+ *   mla_append_cache has just written, or a whole 16-bit pool once). Errors: MLA_ERR_INVALID_ARG
+ *   (null or misaligned pointers, bad strides, rows <= 0), MLA_ERR_UNSUPPORTED (d_c not a multiple
+ *   of 16).
+ * mla_decode_absorbed_fp8: a3 + a4 over that cache. The cache descriptor names the codes, the
+ *   scales and the dtype RoPE keys of the same num_pages*64 rows. workspace: at least
+ *   mla_decode_fp8_workspace_size(...) bytes (split partials; no initialisation needed). Runs on the
+ *   CUDA cores (fp32 arithmetic); requires every seqlens[b] >= s_q. Same errors as
+ *   mla_decode_absorbed.
+ * ------------------------------------------------------------------------------------------- */
+typedef struct mla_latent_cache_fp8 {
+  const uint8_t* codes;   /* device, [num_pages*64, >= d_c] E4M3 codes of the latent rows */
+  int64_t code_stride;    /* bytes from one row of codes to the next, >= d_c, multiple of 16 */
+  const float* scales;    /* device, [num_pages*64] one fp32 scale per row */
+  const void* rope;       /* device, dtype, [num_pages*64, >= d_r] RoPE keys */
+  int64_t rope_stride;    /* elements from one RoPE row to the next, >= d_r */
+  int32_t num_pages;      /* pages in the pool; page ids must be < num_pages */
+} mla_latent_cache_fp8_t;
+
+MLA_API int mla_quantize_latent_fp8(const mla_dims_t* dims, int32_t dtype, const void* latent, int64_t latent_stride,
+                                    int64_t rows, uint8_t* codes, int64_t code_stride, float* scales, void* stream);
+MLA_API size_t mla_decode_fp8_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t max_pages);
+MLA_API int mla_decode_absorbed_fp8(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_abs,
+                                    const mla_latent_cache_fp8_t* cache, const int32_t* block_table,
+                                    int32_t max_pages, const int32_t* seqlens, void* o_lat, float* lse,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Status.
  * mla_check_status: synchronises `stream`, returns the device status word of the current device
  * (MLA_OK when no kernel recorded an error since the last call) and clears it.

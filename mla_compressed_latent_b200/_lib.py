@@ -35,6 +35,11 @@ class MlaGqaCache(ctypes.Structure):
                 ("rope", c_void_p), ("rope_stride", c_int64), ("num_pages", c_int32)]
 
 
+class MlaLatentCacheFp8(ctypes.Structure):
+    _fields_ = [("codes", c_void_p), ("code_stride", c_int64), ("scales", c_void_p), ("rope", c_void_p),
+                ("rope_stride", c_int64), ("num_pages", c_int32)]
+
+
 PD = POINTER(MlaDims)
 PI = c_void_p  # int32 device pointers travel as void*
 
@@ -65,6 +70,11 @@ SIGNATURES = {
     "mla_preabsorb_out_weights": (c_int32, [PD, c_int32, c_void_p, c_void_p, c_int32, c_void_p, c_void_p]),
     "mla_out_proj_preabsorbed": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_int32, c_void_p,
                                            c_void_p]),
+    "mla_quantize_latent_fp8": (c_int32, [PD, c_int32, c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p,
+                                          c_void_p]),
+    "mla_decode_fp8_workspace_size": (c_size_t, [PD, c_int32, c_int32, c_int32]),
+    "mla_decode_absorbed_fp8": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, POINTER(MlaLatentCacheFp8), PI,
+                                          c_int32, PI, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "mla_check_status": (c_int32, [c_void_p]),
     "mla_status_string": (c_char_p, [c_int32]),
     "mla_build_info": (c_char_p, []),

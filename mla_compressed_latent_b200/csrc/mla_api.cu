@@ -123,15 +123,15 @@ size_t simt_decode_ws(int n_tok, int H, int Dv, int max_pages) {
 template <typename T>
 int launch_decode_simt(DecodeArgs A, int n_tok, void* ws, size_t ws_bytes, cudaStream_t st) {
   const int W = A.Dk + A.d_r;
-  const size_t smem = ((size_t)8 * W + (size_t)32 * (W + 1) + (A.kv_shared ? 0 : (size_t)32 * A.Dv) + 256) * 4 + 32 * 8;
-  int rc = set_smem(mla::simt::decode_simt_kernel<T>, smem);
-  if (rc) return rc;
-  if (A.nsplit > 1) {
+  const size_t smem = ((size_t)8 * W + (size_t)32 * (W + 1) + (A.kv_shared ? 0 : (size_t)32 * A.Dv) + 256) * 4 + 32 * 8 + 32 * 4;
+  if (A.nsplit > 1) {   // argument errors before any CUDA call
     const size_t slots = (size_t)n_tok * A.H * A.nsplit;
     if (!ws || ws_bytes < slots * A.Dv * sizeof(float) + slots * sizeof(float)) return MLA_ERR_WORKSPACE;
     A.part_o = reinterpret_cast<float*>(ws);
     A.part_lse = A.part_o + slots * A.Dv;
   }
+  int rc = set_smem(mla::simt::decode_simt_kernel<T>, smem);
+  if (rc) return rc;
   dim3 grid(n_tok, A.H / mla::simt::DEC_HEADS, A.nsplit);
   launch(mla::simt::decode_simt_kernel<T>, grid, 256, smem, st, A);
   if (A.nsplit > 1) {
@@ -434,6 +434,73 @@ int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_
   A.q_rope_raw = nullptr;
   A.kpart = cache->latent; A.k_stride = cache->latent_stride; A.k_group_off = 0;
   A.vpart = cache->latent; A.v_stride = cache->latent_stride; A.v_group_off = 0;
+  A.rope = cache->rope; A.rope_stride = cache->rope_stride;
+  A.Dk = dims->d_c; A.Dv = dims->d_c; A.d_r = dims->d_r; A.H = dims->H; A.heads_per_group = dims->H;
+  A.kv_shared = 1;
+  A.block_table = block_table; A.max_pages = max_pages; A.num_pages = cache->num_pages;
+  A.seqlens = seqlens; A.s_q = s_q; A.sm_scale = score_scale(dims); A.rope_base = dims->rope_base;
+  A.out = o_lat; A.out_head_stride = dims->d_c; A.lse = lse;
+  SimtSplit sp = simt_split(n_tok, dims->H, max_pages);
+  A.nsplit = sp.nsplit; A.chunk = sp.chunk;
+  return dtype == MLA_F32 ? launch_decode_simt<float>(A, n_tok, workspace, ws_bytes, st)
+                          : launch_decode_simt<__nv_bfloat16>(A, n_tok, workspace, ws_bytes, st);
+}
+
+// ------------------------------------------------------------------------------------------------
+// 8-bit latent cache
+// ------------------------------------------------------------------------------------------------
+int mla_quantize_latent_fp8(const mla_dims_t* dims, int32_t dtype, const void* latent, int64_t latent_stride,
+                            int64_t rows, uint8_t* codes, int64_t code_stride, float* scales, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (!latent || !codes || !scales || rows <= 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(latent) || !aligned16(codes) || !aligned16(scales)) return MLA_ERR_INVALID_ARG;
+  if (!stride_ok(latent_stride, dtype, dims->d_c) || code_stride < dims->d_c || code_stride % 16) return MLA_ERR_INVALID_ARG;
+  if (dims->d_c % 16) return MLA_ERR_UNSUPPORTED;
+  if ((rows + 7) / 8 > INT32_MAX) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid((unsigned)((rows + 7) / 8));
+  if (dtype == MLA_F32)
+    launch(mla::simt::quantize_e4m3_kernel<float>, grid, 256, 0, st, (const float*)latent, latent_stride, rows,
+           dims->d_c, codes, code_stride, scales);
+  else
+    launch(mla::simt::quantize_e4m3_kernel<__nv_bfloat16>, grid, 256, 0, st, (const __nv_bfloat16*)latent,
+           latent_stride, rows, dims->d_c, codes, code_stride, scales);
+  return launch_status();
+}
+
+size_t mla_decode_fp8_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t max_pages) {
+  if (check_dims(dims) || !tokens_ok(B, s_q) || max_pages <= 0) return 0;
+  return simt_decode_ws(B * s_q, dims->H, dims->d_c, max_pages);
+}
+
+int mla_decode_absorbed_fp8(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_abs,
+                            const mla_latent_cache_fp8_t* cache, const int32_t* block_table, int32_t max_pages,
+                            const int32_t* seqlens, void* o_lat, float* lse, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  if (!tokens_ok(B, s_q) || max_pages <= 0 || !q_abs || !cache || !block_table || !seqlens || !o_lat || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if (!cache->codes || !cache->scales || !cache->rope || cache->num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_abs) || !aligned16(cache->codes) || !aligned16(cache->scales) || !aligned16(cache->rope) ||
+      !aligned16(block_table) || !aligned16(seqlens) || !aligned16(o_lat) || !aligned16(lse) ||
+      (workspace && !aligned16(workspace)))
+    return MLA_ERR_INVALID_ARG;
+  if (cache->code_stride < dims->d_c || cache->code_stride % 16 || !stride_ok(cache->rope_stride, dtype, dims->d_r))
+    return MLA_ERR_INVALID_ARG;
+  if (dims->H % mla::simt::DEC_HEADS || dims->d_c % 32 || dims->d_c > 32 * mla::simt::DEC_MAX_OV)
+    return MLA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int n_tok = B * s_q;
+  DecodeArgs A{};
+  A.q = q_abs;
+  A.q_head_stride = dims->d_c + dims->d_r;
+  A.q_rope_raw = nullptr;
+  A.kpart = cache->codes; A.k_stride = cache->code_stride; A.k_group_off = 0; A.kscale = cache->scales;
+  A.vpart = cache->codes; A.v_stride = cache->code_stride; A.v_group_off = 0;
   A.rope = cache->rope; A.rope_stride = cache->rope_stride;
   A.Dk = dims->d_c; A.Dv = dims->d_c; A.d_r = dims->d_r; A.H = dims->H; A.heads_per_group = dims->H;
   A.kv_shared = 1;

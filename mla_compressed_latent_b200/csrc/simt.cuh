@@ -299,6 +299,8 @@ struct DecodeArgs {
   int64_t q_head_stride;
   const void* q_rope_raw;  // grouped path: [n_tok, H, d_r] un-rotated; nullptr for absorbed
   const void* kpart; int64_t k_stride; int64_t k_group_off;
+  const float* kscale;     // 8-bit latent cache: kpart holds E4M3 codes (k_stride in bytes), one fp32
+                           // scale per row here; nullptr for a dtype cache
   const void* vpart; int64_t v_stride; int64_t v_group_off;
   const void* rope; int64_t rope_stride;
   int Dk, Dv, d_r, H, heads_per_group;
@@ -310,10 +312,21 @@ struct DecodeArgs {
   float* part_o; float* part_lse; int nsplit; int chunk;
 };
 
+// Value of an E4M3 code from the format's definition: sign, exponent field e (bias 7), mantissa m;
+// (1 + m/8) * 2^(e-7) for e >= 1 (written straight into fp32's fields), m * 2^-9 for e = 0, NaN for
+// e = 15, m = 7.
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
+  if (e == 15u && m == 7u) v = __uint_as_float(0x7fc00000u);
+  return (c & 0x80u) ? -v : v;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 decode_simt_kernel(DecodeArgs A) {
   extern __shared__ float sm[];
+  __shared__ float lut[256];   // E4M3 code -> value, for an 8-bit latent cache
   const int W = A.Dk + A.d_r;
   const int WP = W + 1;  // padded key row: conflict-free column reads
   float* qs = sm;                              // [8][W]
@@ -321,6 +334,9 @@ decode_simt_kernel(DecodeArgs A) {
   float* vs = A.kv_shared ? ks : ks + DEC_TILE * WP;   // [32][Dv] (or aliases ks)
   float* ps = ks + DEC_TILE * WP + (A.kv_shared ? 0 : DEC_TILE * A.Dv);  // [8][32]
   int64_t* rows = reinterpret_cast<int64_t*>(ps + DEC_HEADS * DEC_TILE);  // [32]
+  float* rscale = reinterpret_cast<float*>(rows + DEC_TILE);             // [32] (8-bit cache)
+  const bool fp8 = A.kscale != nullptr;
+  if (fp8) lut[threadIdx.x] = e4m3_value(threadIdx.x);   // 256 threads, one code each
 
   const int tok = blockIdx.x;
   const int h0 = blockIdx.y * DEC_HEADS;
@@ -369,16 +385,20 @@ decode_simt_kernel(DecodeArgs A) {
     __syncthreads();
     if (threadIdx.x < DEC_TILE) {
       const int p = p0 + threadIdx.x;
-      rows[threadIdx.x] = (p < hi) ? cache_row(table, p, A.num_pages) : -1;
+      const int64_t row = (p < hi) ? cache_row(table, p, A.num_pages) : -1;
+      rows[threadIdx.x] = row;
+      if (fp8) rscale[threadIdx.x] = row >= 0 ? A.kscale[row] : 0.f;
     }
     __syncthreads();
+    const uint8_t* k8 = reinterpret_cast<const uint8_t*>(A.kpart);
     for (int i = threadIdx.x; i < DEC_TILE * W; i += blockDim.x) {
       const int r = i / W, d = i % W;
       const int64_t row = rows[r];
       float v = 0.f;
       if (row >= 0) {
-        v = (d < A.Dk) ? ld(kp + row * A.k_stride + grp * A.k_group_off + d)
-                       : ld(rp + row * A.rope_stride + (d - A.Dk));
+        if (d >= A.Dk) v = ld(rp + row * A.rope_stride + (d - A.Dk));
+        else if (fp8) v = lut[k8[row * A.k_stride + d]] * rscale[r];   // the dequantised latent
+        else v = ld(kp + row * A.k_stride + grp * A.k_group_off + d);
       }
       ks[r * WP + d] = v;
     }
@@ -435,6 +455,35 @@ decode_simt_kernel(DecodeArgs A) {
       if (k < nov) po[lane + 32 * k] = o[k] * inv_l;
     if (lane == 0) A.part_lse[slot] = lse;
   }
+}
+
+// 8-bit latent cache: row j of `lat` becomes the E4M3 codes of c_j / s_j, s_j = max|c_j| / 448 (both
+// in fp32, each operation rounded once; round to nearest, ties to even, saturated at 448 by the
+// conversion instruction; a zero magnitude is stored as +0). One warp per row, 8 rows per block.
+template <typename T>
+__global__ void __launch_bounds__(256)
+quantize_e4m3_kernel(const T* __restrict__ lat, int64_t lat_stride, int64_t rows, int d_c, uint8_t* __restrict__ codes,
+                     int64_t code_stride, float* __restrict__ scales) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const T* src = lat + row * lat_stride;
+  float amax = 0.f;
+  for (int i = lane; i < d_c; i += 32) amax = fmaxf(amax, fabsf(ld(src + i)));
+  amax = warp_max(amax);
+  const float s = __fdiv_rn(amax, 448.f);
+  const float safe = s > 0.f ? s : 1.f;
+  uint8_t* dst = codes + row * code_stride;
+  for (int i = 2 * lane; i < d_c; i += 64) {
+    const float a = __fdiv_rn(ld(src + i), safe), b = __fdiv_rn(ld(src + i + 1), safe);
+    uint16_t pr;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(b), "f"(a));   // a -> low byte
+    uint32_t lo = pr & 0xffu, hi = pr >> 8;
+    if ((lo & 0x7fu) == 0u) lo = 0u;   // -0 -> +0
+    if ((hi & 0x7fu) == 0u) hi = 0u;
+    *reinterpret_cast<uint16_t*>(dst + i) = (uint16_t)(lo | (hi << 8));
+  }
+  if (lane == 0) scales[row] = s;
 }
 
 // a4: combine the split partials of every (token, head): weights exp(lse_s - LSE).

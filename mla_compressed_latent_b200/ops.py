@@ -108,6 +108,28 @@ class GqaCache:
                              self.rope.data_ptr(), self.rope.stride(0), self.num_pages)
 
 
+@dataclass
+class LatentCacheFp8:
+    """8-bit latent pool: E4M3 codes [num_pages*64, d_c] uint8 + fp32 scales [num_pages*64] + the
+    16-bit RoPE-key pool [num_pages*64, d_r]."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    rope: torch.Tensor
+    num_pages: int
+
+    @staticmethod
+    def empty_like(cache: "LatentCache") -> "LatentCacheFp8":
+        """Code and scale storage for every row of a 16-bit pool, sharing its RoPE keys."""
+        rows, d_c = cache.latent.shape
+        dev = cache.latent.device
+        return LatentCacheFp8(torch.empty(rows, d_c, dtype=torch.uint8, device=dev),
+                              torch.empty(rows, dtype=torch.float32, device=dev), cache.rope, cache.num_pages)
+
+    def c(self) -> L.MlaLatentCacheFp8:
+        return L.MlaLatentCacheFp8(self.codes.data_ptr(), self.codes.stride(0), self.scales.data_ptr(),
+                                   self.rope.data_ptr(), self.rope.stride(0), self.num_pages)
+
+
 def _workspace(nbytes, device, workspace):
     if nbytes == 0:
         return workspace, 0
@@ -186,6 +208,38 @@ def mla_decode_absorbed(dims: Dims, q_abs, cache: LatentCache, block_table, seql
                                  _ptr(_i32(block_table)), max_pages, _ptr(_i32(seqlens)), _ptr(o_lat), _ptr(lse),
                                  _ptr(workspace) if workspace is not None else None, wsb, _stream(stream))
     _check("mla_decode_absorbed", rc)
+    return o_lat, lse
+
+
+def mla_quantize_latent_fp8(dims: Dims, latent, codes, scales, stream=None):
+    """Rows of `latent` [rows, d_c] (dtype, rows may be a view of a pool) into E4M3 `codes` [rows, d_c]
+    (uint8) and fp32 `scales` [rows]."""
+    lib = L.load()
+    rows = latent.shape[0]
+    d = dims.c()
+    rc = lib.mla_quantize_latent_fp8(ctypes.byref(d), _dt(latent), _ptr(latent), latent.stride(0), rows, _ptr(codes),
+                                     codes.stride(0), _ptr(scales), _stream(stream))
+    _check("mla_quantize_latent_fp8", rc)
+    return codes, scales
+
+
+def mla_decode_absorbed_fp8(dims: Dims, q_abs, cache: LatentCacheFp8, block_table, seqlens, o_lat=None, lse=None,
+                            workspace=None, stream=None):
+    lib = L.load()
+    B, s_q, H, _ = q_abs.shape
+    if o_lat is None:
+        o_lat = torch.empty(B, s_q, H, dims.d_c, dtype=q_abs.dtype, device=q_abs.device)
+    if lse is None:
+        lse = torch.empty(B, s_q, H, dtype=torch.float32, device=q_abs.device)
+    d = dims.c()
+    max_pages = block_table.shape[1]
+    need = lib.mla_decode_fp8_workspace_size(ctypes.byref(d), B, s_q, max_pages)
+    workspace, wsb = _workspace(need, q_abs.device, workspace)
+    cc = cache.c()
+    rc = lib.mla_decode_absorbed_fp8(ctypes.byref(d), _dt(q_abs), B, s_q, _ptr(q_abs), ctypes.byref(cc),
+                                     _ptr(_i32(block_table)), max_pages, _ptr(_i32(seqlens)), _ptr(o_lat), _ptr(lse),
+                                     _ptr(workspace) if workspace is not None else None, wsb, _stream(stream))
+    _check("mla_decode_absorbed_fp8", rc)
     return o_lat, lse
 
 

@@ -63,6 +63,7 @@ class Workload:
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
     description: str = ""
+    latent_bits: int = 16      # 8: the latent rows are kept as E4M3 codes with one scale per row
 
     @property
     def d_qk(self) -> int:
@@ -102,6 +103,10 @@ WORKLOADS = {
         Workload("mtp_sq4_b128", "bf16", B=128, s_q=4, H=128, D=128, d_r=64, d_c=512, d_v=128,
                  C=7168, lengths=("uniform", 1024, 32768), pages="random",
                  description="multi-token absorbed decode, 4 tokens per step, random page table"),
+        Workload("dsv3_fp8_b64_l4096", "bf16", B=64, s_q=1, H=128, D=128, d_r=64, d_c=512, d_v=128, C=7168,
+                 latent_bits=8,
+                 description="the DeepSeek-shaped batch over an 8-bit latent cache (E4M3 codes, one fp32 scale "
+                             "per row, 16-bit RoPE keys)"),
     ]
 }
 

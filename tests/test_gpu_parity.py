@@ -10,10 +10,11 @@ import pytest
 import torch
 
 import synth
+from oracle import fp8_cache as F
 from oracle import mla_oracle as O
 from mla_compressed_latent_b200 import _lib as L
 from mla_compressed_latent_b200 import ops
-from mla_compressed_latent_b200.ops import Dims, LatentCache, GqaCache
+from mla_compressed_latent_b200.ops import Dims, LatentCache, LatentCacheFp8, GqaCache
 
 from _cases import TOL, Case, as_stored, max_rel_err
 
@@ -650,3 +651,91 @@ def test_invalid_arguments_raise():
     with pytest.raises(ops.MlaError):
         ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"],
                                 o_lat=torch.empty(1, 1, 128, 512, dtype=torch.bfloat16, device="cuda")[..., 1:])
+
+
+# ------------------------------------------------------------------------------------------------
+# f4: 8-bit latent cache. The decode checks take codes and scales made by the oracle on the host
+# (its float32-decision quantiser), never the GPU quantiser's, which has its own bit-exact test.
+# ------------------------------------------------------------------------------------------------
+
+def _fp8_rows(case):
+    """Oracle E4M3 codes and scales of every row of the case's 16-bit pool."""
+    lat = case.pool[:, :case.w.d_c].to(torch.float64).numpy()
+    return F.quantize_rows_f32(lat)
+
+
+def _seq_pool_index(case, b):
+    p = np.arange(int(case.lens[b]))
+    return case.table[b, p // 64].astype(np.int64) * 64 + p % 64
+
+
+@pytest.mark.parametrize("name,dtype", [("dsv3_b64_l4096", torch.bfloat16), ("smallem_fp32", torch.float32)])
+def test_quantize_latent_fp8_matches_the_oracle_bit_for_bit(name, dtype):
+    """Codes and scales of the GPU quantiser equal the oracle's (decision in float32), on rows read
+    through an interleaved pool's stride: varied magnitudes, a zero row, values far below their row's
+    scale (code +0), subnormal codes, a row whose largest value dwarfs the rest."""
+    w = synth.workload(name)
+    r = np.random.default_rng(60)
+    rows, d_c, stride = 700, w.d_c, w.d_c + w.d_r
+    c = r.standard_normal((rows, d_c)) * r.uniform(1e-3, 50, (rows, 1))
+    c[3] = 0.0
+    c[4] = 1e-30
+    c[4, 0] = 1.0
+    c[5] = r.uniform(-1, 1, d_c) * 2.0 ** -8
+    c[6, 7] = 448.0 * 3
+    pool = torch.zeros(rows, stride, dtype=dtype)
+    pool[:, :d_c] = torch.from_numpy(c).to(dtype)
+    ref_codes, ref_scales = F.quantize_rows_f32(pool[:, :d_c].to(torch.float64).numpy())
+    dev = pool.cuda()
+    codes = torch.empty(rows, d_c, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(rows, dtype=torch.float32, device="cuda")
+    ops.mla_quantize_latent_fp8(Dims.of(w), dev[:, :d_c], codes, scales)
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref_codes)
+    np.testing.assert_array_equal(scales.cpu().numpy().astype(np.float64), ref_scales)
+    assert (ref_codes[4, 1:] == 0).all() and ref_scales[3] == 0 and (ref_codes[3] == 0).all()
+
+
+FP8_DECODE = [
+    ([1], 1, "contiguous"),
+    ([64, 65], 1, "random"),
+    ([4096, 129, 2049, 64, 5000], 1, "contiguous"),
+    ([65, 129, 64 * 5 + 1, 2], 2, "random"),
+    ([131072], 1, "random"),
+]
+
+
+def _decode_fp8_case(w, heads=None, seqs=None):
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    codes, scales = _fp8_rows(case)
+    cache = LatentCacheFp8(torch.from_numpy(codes).cuda(), torch.from_numpy(scales.astype(np.float32)).cuda(),
+                           dev["pool"][:, w.d_c:], case.num_pages)
+    o_lat, lse = ops.mla_decode_absorbed_fp8(Dims.of(w), dev["q_abs"], cache, dev["table"], dev["seqlens"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    got_o, got_l = o_lat.float().cpu().numpy(), lse.cpu().numpy()
+    for b in (range(w.B) if seqs is None else seqs):
+        idx = _seq_pool_index(case, b)
+        kr = case.pool[torch.from_numpy(idx), w.d_c:].to(torch.float64).numpy()
+        q = case.q_abs64[b] if heads is None else case.q_abs64[b][:, heads]
+        ref_o, ref_l = F.absorbed_decode_fp8(q, codes[idx], scales[idx], kr, int(case.lens[b]), w.sm_scale)
+        go = got_o[b] if heads is None else got_o[b][:, heads]
+        gl = got_l[b] if heads is None else got_l[b][:, heads]
+        _assert_close(go, ref_o, "bf16", f"o_lat seq {b}")
+        _assert_lse(gl, ref_l, "bf16", f"lse seq {b}")
+
+
+@pytest.mark.parametrize("lens,s_q,pages", FP8_DECODE)
+def test_decode_absorbed_fp8(lens, s_q, pages):
+    _decode_fp8_case(synth.workload("dsv3_b64_l4096", B=len(lens), s_q=s_q, lengths=("list", tuple(lens)),
+                                    pages=pages))
+
+
+def test_decode_absorbed_fp8_full_size_sampled():
+    """The bench's 8-bit configuration (64 x 4096, DeepSeek widths), every sequence decoded, the
+    oracle on a seeded sample of sequences and heads."""
+    w = synth.workload("dsv3_b64_l4096")
+    r = np.random.default_rng(61)
+    _decode_fp8_case(w, heads=r.choice(w.H, 12, replace=False), seqs=r.choice(w.B, 6, replace=False))

@@ -47,6 +47,12 @@ def _gqa_cache(**kw):
     return L.MlaGqaCache(c["k"], c["k_stride"], c["v"], c["v_stride"], c["rope"], c["rope_stride"], c["num_pages"])
 
 
+def _fp8_cache(**kw):
+    c = dict(codes=GOOD, code_stride=512, scales=GOOD, rope=GOOD + 1024, rope_stride=576, num_pages=10)
+    c.update(kw)
+    return L.MlaLatentCacheFp8(c["codes"], c["code_stride"], c["scales"], c["rope"], c["rope_stride"], c["num_pages"])
+
+
 BIG_WS = 1 << 40   # larger than any workspace the calls ask for
 
 
@@ -79,9 +85,15 @@ CALLS = {
     "mla_preabsorb_out_weights": ([P, P, 7168, P, None], [0, 1, 3], [2], None, []),
     # B, s_q, o_lat, w_uvo, C, out_model, stream
     "mla_out_proj_preabsorbed": ([64, 1, P, P, 7168, P, None], [2, 3, 5], [0, 1, 4], None, []),
+    # latent, latent_stride, rows, codes, code_stride, scales, stream
+    "mla_quantize_latent_fp8": ([P, 576, 1000, P, 512, P, None], [0, 3, 5], [1, 2, 4], None, []),
+    # B, s_q, q_abs, cache, table, max_pages, seqlens, o_lat, lse, ws, ws_bytes, stream (one long
+    # sequence: the CUDA-core decode then splits it and needs a workspace)
+    "mla_decode_absorbed_fp8": ([1, 1, P, "FC", P, 2048, P, P, P, P, BIG_WS, None],
+                                [2, 4, 6, 7, 8], [0, 1, 5], 9, []),
 }
 # calls without a token count (B, s_q): the overflow check does not apply
-NO_TOKENS = {"mla_preabsorb_out_weights"}
+NO_TOKENS = {"mla_preabsorb_out_weights", "mla_quantize_latent_fp8"}
 
 
 def _call(lib, name, args, dims=None, dtype=1):
@@ -92,6 +104,8 @@ def _call(lib, name, args, dims=None, dtype=1):
             conv.append(ctypes.byref(_latent_cache()))
         elif a == "GC":
             conv.append(ctypes.byref(_gqa_cache()))
+        elif a == "FC":
+            conv.append(ctypes.byref(_fp8_cache()))
         elif a == P:
             conv.append(ctypes.c_void_p(GOOD))
         elif a == P_ODD:
@@ -174,3 +188,21 @@ def test_bad_gqa_cache_is_rejected(lib, field, value):
     rc = lib.mla_decode_gqla_grouped(ctypes.byref(d), 1, 32, 1, g, g, ctypes.byref(cache), g, 128, g, g, g, g,
                                      BIG_WS, None)
     assert rc == L.MLA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("field,value", [("codes", 0), ("scales", 0), ("rope", 0), ("codes", ODD), ("scales", ODD),
+                                         ("code_stride", 500), ("code_stride", 520), ("rope_stride", 63),
+                                         ("num_pages", 0)])
+def test_bad_fp8_cache_is_rejected(lib, field, value):
+    cache = _fp8_cache(**{field: value})
+    d = _dims()
+    g = ctypes.c_void_p(GOOD)
+    rc = lib.mla_decode_absorbed_fp8(ctypes.byref(d), 1, 64, 1, g, ctypes.byref(cache), g, 64, g, g, g, g, BIG_WS,
+                                     None)
+    assert rc == L.MLA_ERR_INVALID_ARG
+
+
+def test_fp8_quantiser_wants_whole_16_value_rows(lib):
+    g = ctypes.c_void_p(GOOD)
+    d = _dims(d_c=520)
+    assert lib.mla_quantize_latent_fp8(ctypes.byref(d), 1, g, 528, 10, g, 528, g, None) == L.MLA_ERR_UNSUPPORTED
