@@ -644,6 +644,38 @@ def test_page_id_outside_pool_is_reported_not_read():
     assert ops.mla_check_status() == 0       # cleared by the previous read
 
 
+def test_sequence_without_its_new_token_is_reported():
+    """seqlens[b] must count the step's own token: a zero length is reported by every decode path
+    (absorbed, grouped, 8-bit) as a device check, its outputs left unwritten, the others still right."""
+    w = synth.workload("dsv3_b64_l4096", B=2, lengths=("list", (200, 70)))
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    short = dev["seqlens"].clone()
+    short[1] = 0
+    o_lat, lse = ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), dev["table"], short)
+    assert ops.mla_check_status() == L.MLA_ERR_DEVICE_CHECK
+    ref_o, ref_l = _oracle_absorbed(case, case.q_abs64, seqs=[0])
+    _assert_close(o_lat[0].float().cpu().numpy(), ref_o[0], "bf16", "o_lat of the valid sequence")
+    _assert_lse(lse[0].cpu().numpy(), ref_l[0], "bf16", "lse of the valid sequence")
+    codes, scales = _fp8_rows(case)
+    cache8 = LatentCacheFp8(torch.from_numpy(codes).cuda(), torch.from_numpy(scales.astype(np.float32)).cuda(),
+                            dev["pool"][:, w.d_c:], case.num_pages)
+    ops.mla_decode_absorbed_fp8(Dims.of(w), dev["q_abs"], cache8, dev["table"], short)
+    assert ops.mla_check_status() == L.MLA_ERR_DEVICE_CHECK
+    wg = synth.workload("gqla_g8_b32_l8192", B=2, lengths=("list", (200, 70)))
+    cg = Case(wg)
+    dg = cg.to_device()
+    n = cg.num_pages * 64
+    gcache = GqaCache(torch.zeros(n, wg.g, wg.D, dtype=torch.bfloat16, device="cuda"),
+                      torch.zeros(n, wg.g, wg.d_v, dtype=torch.bfloat16, device="cuda"),
+                      torch.zeros(n, wg.d_r, dtype=torch.bfloat16, device="cuda"), cg.num_pages)
+    short_g = dg["seqlens"].clone()
+    short_g[1] = 0
+    ops.mla_decode_gqla_grouped(Dims.of(wg), dg["q_nope"], dg["q_rope_raw"], gcache, dg["table"], short_g)
+    assert ops.mla_check_status() == L.MLA_ERR_DEVICE_CHECK
+    assert ops.mla_check_status() == 0
+
+
 def test_invalid_arguments_raise():
     w = synth.workload("dsv3_b64_l4096", B=1, lengths=("list", (64,)))
     case = Case(w, with_weights=False)
