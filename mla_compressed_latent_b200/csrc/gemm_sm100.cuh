@@ -58,6 +58,9 @@ struct Params {
   // Layouts: a_kmajor = the weights are stored [H, M, K] (K contiguous: W[h] transposed), read
   // K-major; x_shared = X is [n_tok, K], one row per token shared by every head.
   int a_kmajor, x_shared;
+  // set by run(): every output row start is 16-byte aligned (base and strides), so the epilogue may
+  // store 16-byte pieces
+  int vec_out;
 };
 
 __host__ __device__ constexpr int stage_bytes(int tn) { return kABytes + tn * 128; }
@@ -222,7 +225,44 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
     }
     const bool ok = __all_sync(0xffffffffu, wait(done, 0));
     ptx::tc_fence_after();
-    if (ok) {
+    if (ok && p.vec_out) {
+      // 32 features (the warp's TMEM lanes) x 32 tokens at a time: each thread puts its feature's
+      // values in column `lane` of a [token][feature] tile in shared memory (the ring, free once the
+      // accumulator is done: 4 KB per warp), then the warp stores the tile's token rows in 16-byte
+      // pieces (features are contiguous in every output; M and the strides are multiples of 8).
+      uint8_t* tile = smem_raw + (ring - raw) + (uint32_t)(warp - 4) * 4096u;
+      const uint32_t tile_s = ring + (uint32_t)(warp - 4) * 4096u;
+      const int f0 = mt * kBM + (warp & 3) * 32;   // the warp's first feature
+      const bool f32_out = !second && p.mode != 0;
+      for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tmem + lane_off + (uint32_t)c, r);
+        ptx::tmem_wait_ld();
+        const int kn = min(32, p.n_tok - tok0 - c);
+        if (f32_out) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            reinterpret_cast<float*>(tile)[k * 32 + lane] = nk > 0 ? __uint_as_float(r[k]) : 0.f;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            reinterpret_cast<__nv_bfloat16*>(tile)[k * 32 + lane] = __float2bfloat16_rn(nk > 0 ? __uint_as_float(r[k]) : 0.f);
+        }
+        __syncwarp();
+        const int pieces = f32_out ? 8 : 4;   // 16-byte pieces per 32-feature token row
+        for (int i = lane; i < 32 * pieces; i += 32) {
+          const int t = i / pieces, f = f0 + (i % pieces) * (f32_out ? 4 : 8);
+          if (t >= kn || f >= M) continue;
+          const uint4 v = ptx::ld_shared_v4(tile_s + (uint32_t)i * 16u);
+          const int tok = tok0 + c + t;
+          void* dst = second ? (void*)(p.y2 + (int64_t)tok * p.y2_tok_stride + f)
+                    : p.mode == 0 ? (void*)(p.y + (int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + f)
+                                  : (void*)(p.part + ((int64_t)split * p.n_tok + tok) * p.M + f);
+          *reinterpret_cast<uint4*>(dst) = v;
+        }
+        __syncwarp();
+      }
+    } else if (ok) {   // any other output layout: one value per store
       for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
         uint32_t r[32];
         ptx::tmem_ld32(tmem + lane_off + (uint32_t)c, r);
@@ -304,6 +344,14 @@ inline int run(const Problem& pr, Params p, cudaStream_t st) {
     return MLA_ERR_UNSUPPORTED;
   p.M = pr.M;
   p.M2 = two ? pr.M2 : 0;
+  {
+    auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+    if (p.mode == 0)
+      p.vec_out = a16(p.y) && p.y_tok_stride % 8 == 0 && p.y_head_stride % 8 == 0 &&
+                  (!two || (a16(p.y2) && p.y2_tok_stride % 8 == 0)) ? 1 : 0;
+    else
+      p.vec_out = a16(p.part) && pr.M % 4 == 0 ? 1 : 0;
+  }
   p.K = pr.K;
   p.n_tok = pr.n_tok;
   p.H = pr.H;
