@@ -821,83 +821,91 @@ __device__ __forceinline__ int pair_of(long long x, long long T, int P) { return
 // Each warp finds the sequence's tile range itself (no block barrier), then issues all its
 // partial loads before combining them.
 constexpr int kMergeHeads = 4;
+constexpr int kMergeTokenBlocks = 8;   // blocks along the tokens; each strides over them
 __global__ void __launch_bounds__(32 * kMergeHeads)
 merge_kernel(const int32_t* __restrict__ seqlens, int B, int s_q, int max_tiles, int npairs, const float* __restrict__ part_o,
              const float* __restrict__ part_lse, __nv_bfloat16* __restrict__ o_lat, float* __restrict__ lse) {
-  // block x: new token v = b * s_q + tok of sequence b; its parts come from pair (group, tok) of the
-  // groups that covered the sequence's tiles
-  const int v = blockIdx.x, b = v / s_q, tok = v % s_q;
+  // blocks stride over the new tokens v = b * s_q + tok; a token's parts come from pair (group, tok) of
+  // the groups that covered its sequence's tiles
   const int G = npairs / s_q;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   grid_dependency_wait();
   allow_dependents();
-  // global tile offset of sequence b and the total: lane l sums sequences [l*per, (l+1)*per)
+  // the total of tiles and the longest sequence decide the split, the same for every token: lane l
+  // sums sequences [l*per, (l+1)*per)
   const int per = (B + 31) / 32;
   const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
-  long long local = 0, before = 0;
+  long long local = 0;
   int max_tb = 0;
   for (int x = b0; x < b1; ++x) {
     const int tb = tiles_of(__ldg(seqlens + x), max_tiles);
-    if (x < b) before += tb;
     local += tb;
     max_tb = max(max_tb, tb);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     local += __shfl_xor_sync(0xffffffffu, local, o);
-    before += __shfl_xor_sync(0xffffffffu, before, o);
     max_tb = max(max_tb, __shfl_xor_sync(0xffffffffu, max_tb, o));
   }
-  const long long T = local, off = before, tb = tiles_of(__ldg(seqlens + b), max_tiles);
-  if (tb == 0 || T == 0 || G == 0 || whole_sequences(B, G, T, max_tb)) return;   // nothing was cut
-  const int p0 = pair_of(off, T, G), p1 = pair_of(off + tb - 1, T, G);   // groups
-  if (p0 == p1) return;                       // written whole by one group
-  const int h = blockIdx.y * kMergeHeads + warp;
-  // a group with an empty range wrote nothing; the others' parts in order, lane q holds group p0 + q's lse
-  auto slot = [&](int q) -> int {
-    const long long start_q = (long long)q * T / G;
-    if ((long long)(q + 1) * T / G <= start_q) return -1;
-    return (q * s_q + tok) * 2 + (start_q < off ? 1 : 0);
-  };
-  float mx = -INFINITY;
-  for (int q0 = p0; q0 <= p1; q0 += 32) {
-    const int q = q0 + lane;
-    const int idx = q <= p1 ? slot(q) : -1;
-    mx = fmaxf(mx, warp_max(idx >= 0 ? part_lse[(size_t)idx * kH + h] : -INFINITY));
-  }
-  float tot = 0.f;
-  float acc[16];
+  const long long T = local;
+  if (T == 0 || G == 0 || whole_sequences(B, G, T, max_tb)) return;   // nothing was cut
+  for (int v = blockIdx.x; v < B * s_q; v += gridDim.x) {
+    const int b = v / s_q, tok = v % s_q;
+    long long before = 0;
+    for (int x = b0; x < min(b1, b); ++x) before += tiles_of(__ldg(seqlens + x), max_tiles);
 #pragma unroll
-  for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-  // lane covers columns [4 lane + 128 k, +4) for k < 4: every load instruction reads 512 contiguous bytes
-  for (int q = p0; q <= p1; q += 2) {
-    const int i0 = slot(q), i1 = q + 1 <= p1 ? slot(q + 1) : -1;
-    float4 x0[4], x1[4];
-    const float w0 = i0 >= 0 ? exp2f((part_lse[(size_t)i0 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
-    const float w1 = i1 >= 0 ? exp2f((part_lse[(size_t)i1 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
-    const float4* s0 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i0, 0) * kH + h) * kDC) + lane;
-    const float4* s1 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i1, 0) * kH + h) * kDC) + lane;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      x0[k] = i0 >= 0 ? s0[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
-      x1[k] = i1 >= 0 ? s1[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+    const long long off = before, tb = tiles_of(__ldg(seqlens + b), max_tiles);
+    if (tb == 0) continue;
+    const int p0 = pair_of(off, T, G), p1 = pair_of(off + tb - 1, T, G);   // groups
+    if (p0 == p1) continue;                     // written whole by one group
+    const int h = blockIdx.y * kMergeHeads + warp;
+    // a group with an empty range wrote nothing; the others' parts in order, lane q holds group p0 + q's lse
+    auto slot = [&](int q) -> int {
+      const long long start_q = (long long)q * T / G;
+      if ((long long)(q + 1) * T / G <= start_q) return -1;
+      return (q * s_q + tok) * 2 + (start_q < off ? 1 : 0);
+    };
+    float mx = -INFINITY;
+    for (int q0 = p0; q0 <= p1; q0 += 32) {
+      const int q = q0 + lane;
+      const int idx = q <= p1 ? slot(q) : -1;
+      mx = fmaxf(mx, warp_max(idx >= 0 ? part_lse[(size_t)idx * kH + h] : -INFINITY));
     }
-    tot += w0 + w1;
+    float tot = 0.f;
+    float acc[16];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      acc[4 * k] += w0 * x0[k].x + w1 * x1[k].x;
-      acc[4 * k + 1] += w0 * x0[k].y + w1 * x1[k].y;
-      acc[4 * k + 2] += w0 * x0[k].z + w1 * x1[k].z;
-      acc[4 * k + 3] += w0 * x0[k].w + w1 * x1[k].w;
+    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+    // lane covers columns [4 lane + 128 k, +4) for k < 4: every load instruction reads 512 contiguous bytes
+    for (int q = p0; q <= p1; q += 2) {
+      const int i0 = slot(q), i1 = q + 1 <= p1 ? slot(q + 1) : -1;
+      float4 x0[4], x1[4];
+      const float w0 = i0 >= 0 ? exp2f((part_lse[(size_t)i0 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
+      const float w1 = i1 >= 0 ? exp2f((part_lse[(size_t)i1 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
+      const float4* s0 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i0, 0) * kH + h) * kDC) + lane;
+      const float4* s1 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i1, 0) * kH + h) * kDC) + lane;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        x0[k] = i0 >= 0 ? s0[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+        x1[k] = i1 >= 0 ? s1[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      tot += w0 + w1;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[4 * k] += w0 * x0[k].x + w1 * x1[k].x;
+        acc[4 * k + 1] += w0 * x0[k].y + w1 * x1[k].y;
+        acc[4 * k + 2] += w0 * x0[k].z + w1 * x1[k].z;
+        acc[4 * k + 3] += w0 * x0[k].w + w1 * x1[k].w;
+      }
     }
-  }
-  const float inv = 1.f / tot;
-  uint2* dst = reinterpret_cast<uint2*>(o_lat + ((size_t)v * kH + h) * kDC) + lane;
+    const float inv = 1.f / tot;
+    uint2* dst = reinterpret_cast<uint2*>(o_lat + ((size_t)v * kH + h) * kDC) + lane;
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
-    dst[32 * k] = make_uint2(ptx::pack_bf16x2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
-                             ptx::pack_bf16x2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
-  if (lane == 0) lse[(size_t)v * kH + h] = mx + logf(tot);
+    for (int k = 0; k < 4; ++k)
+      dst[32 * k] = make_uint2(ptx::pack_bf16x2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
+                               ptx::pack_bf16x2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
+    if (lane == 0) lse[(size_t)v * kH + h] = mx + logf(tot);
+  }
 }
 
 // ---- host side -----------------------------------------------------------------------------------------
@@ -974,7 +982,7 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   prm.part_lse = prm.part_o + (size_t)2 * max_pairs(num_sms) * kH * kDC;
   prm.sm_scale_log2 = d->sm_scale * 1.4426950408889634f;
   launch_pdl(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
-  launch_pdl(merge_kernel, dim3(B * s_q, kH / kMergeHeads), dim3(32 * kMergeHeads), 0, st, seqlens, (int)B, (int)s_q, (int)max_pages, P, (const float*)prm.part_o,
+  launch_pdl(merge_kernel, dim3(std::min(B * s_q, kMergeTokenBlocks), kH / kMergeHeads), dim3(32 * kMergeHeads), 0, st, seqlens, (int)B, (int)s_q, (int)max_pages, P, (const float*)prm.part_o,
          (const float*)prm.part_lse, prm.o_lat, lse);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
