@@ -772,12 +772,11 @@ def main():
                                                    q_nope=qn_buf, q_rope_raw=qr_buf, workspace=ws_q)
             if every:
                 mark("project_q")
-        ops.mla_append_cache(dims, x, dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache, workspace=ws_app)
-        if every:
-            mark("append")
-        ops.mla_absorb_q(dims, q_nope, q_rope, dev["W_UK"], dev["seqlens"], q_abs=q_abs)
+        # a1 + a2: the cache append and the query absorption, their projections in one launch
+        ops.mla_append_cache_absorb_q(dims, x, dev["w_dkv_kr"], None, q_nope, q_rope, dev["W_UK"], dev["seqlens"],
+                                      dev["table"], cache, q_abs=q_abs, workspace=ws_app)
         if events:
-            mark("absorb_q")
+            mark("append_absorb")
         ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"], o_lat=o_lat, lse=lse, workspace=ws_dec)
         if events:
             mark("decode")
@@ -822,13 +821,13 @@ def main():
     if max_over_ranks(1.0 if clk.rejected() else 0.0, world, device) > 0:
         ms, launches, clk = timed_region()
         remeasured = True
-    dec_ms = statistics.mean(between(m, "absorb_q", "decode") for m in dec_ev)
+    dec_ms = statistics.mean(between(m, "append_absorb", "decode") for m in dec_ev)
     # per-call breakdown, outside the timed region (its events stop the calls' launches overlapping)
     dec_ev.clear()
     for _ in range(min(args.steps, 50)):
         step(dev["x"], dev["q_nope"], dev["q_rope_raw"], events="all")
     torch.cuda.synchronize()
-    calls = (("project_q",) if from_x else ()) + ("append", "absorb_q", "decode", "out_proj")
+    calls = (("project_q",) if from_x else ()) + ("append_absorb", "decode", "out_proj")
     order = ("start",) + calls
     breakdown = {c: statistics.mean(between(m, order[i], c) for m in dec_ev) * 1e3 for i, c in enumerate(calls)}
     assert ops.mla_check_status() == 0

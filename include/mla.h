@@ -167,6 +167,24 @@ MLA_API int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32
                  const int32_t* seqlens, void* q_abs, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * a1 and a2 of one decode step in one call: mla_append_cache, then mla_absorb_q, on one stream.
+ * The order is the one that overlaps best: the absorption's CTAs (one per head) stream W_UK while
+ * the append's finish (RMSNorm, RoPE, paged store) runs. Arguments, layouts and results are those of
+ * the two calls, bit for bit. workspace: at least mla_append_workspace_size(dims, B, s_q, C) bytes,
+ * no initialisation needed. Argument errors of either half return before anything is launched.
+ * Weights (w_dkv_kr, w_uk here, w_uv and w_o in mla_out_proj) may be read before the kernel
+ * launched just before on the stream has finished, when that kernel lets its successor start early
+ * (programmatic dependent launch): such a kernel must not write them. No kernel of this library
+ * writes an array that one of these calls takes as a weight.
+ * ------------------------------------------------------------------------------------------- */
+MLA_API int mla_append_cache_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                              const void* x, int32_t C, const void* w_dkv_kr, const void* gamma,
+                              const void* q_nope, const void* q_rope_raw, const void* w_uk,
+                              const int32_t* seqlens, const int32_t* block_table, int32_t max_pages,
+                              const mla_latent_cache_t* cache, void* q_abs, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * a3 + a4. Absorbed decode over the latent cache, split over the GPU's SMs, with the
  * log-sum-exp merge of split sequences (« Chemin MQA-Absorbé »; « Le mécanisme d'attention »).
  * For each (b, t, h), over the visible positions j:

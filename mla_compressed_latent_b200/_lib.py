@@ -55,6 +55,9 @@ SIGNATURES = {
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "mla_absorb_q": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, PI, c_void_p,
                                c_void_p]),
+    "mla_append_cache_absorb_q": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_int32, c_void_p, c_void_p,
+                                            c_void_p, c_void_p, c_void_p, PI, PI, c_int32,
+                                            POINTER(MlaLatentCache), c_void_p, c_void_p, c_size_t, c_void_p]),
     "mla_decode_workspace_size": (c_size_t, [PD, c_int32, c_int32, c_int32, c_int32]),
     "mla_decode_absorbed": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, POINTER(MlaLatentCache), PI,
                                       c_int32, PI, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),

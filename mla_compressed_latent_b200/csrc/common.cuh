@@ -87,6 +87,18 @@ __device__ __forceinline__ void rope_cos_sin_at(int pos, double inv_freq, float*
 __device__ __forceinline__ void rope_cos_sin(int pos, int i, int d_r, float base, float* c, float* s) {
   rope_cos_sin_at(pos, rope_inv_freq(i, d_r, base), c, s);
 }
+// The same angle and reduction, the remainder evaluated by the SFU (__sincosf): on |r| <= π its
+// absolute error is a few 1e-7, far below one rounding of a bf16 output (2^-9 relative), at a few
+// instructions instead of sincosf's polynomial. For the bf16-only tensor-core paths.
+__device__ __forceinline__ void rope_cos_sin_at_sfu(int pos, double inv_freq, float* c, float* s) {
+  constexpr double kTwoPiHi = 6.283185307179586;
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;
+  constexpr double kInvTwoPi = 0.15915494309189535;
+  const double a = (double)pos * inv_freq;
+  const double k = rint(a * kInvTwoPi);
+  const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
+  __sincosf((float)r, s, c);
+}
 
 // ---- reductions --------------------------------------------------------------------------------
 __device__ __forceinline__ float warp_sum(float v) {

@@ -61,10 +61,21 @@ struct Params {
   // set by run(): every output row start is 16-byte aligned (base and strides), so the epilogue may
   // store 16-byte pieces
   int vec_out;
+  // set by run(): the grid of CTAs (x = head * CTAs per head [+ the second problem's m-tiles],
+  // y = token block, z = K split)
+  int gx, gy, gz;
+  // 1: the weights are not written by the kernel launched before this one on the stream, so a CTA
+  // issues its first weight tiles before it waits for that kernel (everything else after)
+  int w_early;
+  // m-tiles (128 output features each) per CTA, 1..4: a head's tiles side by side in TMEM, fed by
+  // one token box per K chunk (1 with a second problem or K-major weights)
+  int m_sub;
 };
 
-__host__ __device__ constexpr int stage_bytes(int tn) { return kABytes + tn * 128; }
-__host__ __device__ constexpr int smem_bytes(int tn, int stages) { return 1024 + kBarBytes + stages * stage_bytes(tn); }
+__host__ __device__ constexpr int stage_bytes(int tn, int msub = 1) { return msub * kABytes + tn * 128; }
+__host__ __device__ constexpr int smem_bytes(int tn, int stages, int msub = 1) {
+  return 1024 + kBarBytes + stages * stage_bytes(tn, msub);
+}
 
 #ifdef MLA_TEST_HOOKS
 // Test builds only: with g_test_stall set, each CTA's MMA issuer first waits for a barrier phase that
@@ -89,24 +100,28 @@ __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, const volati
   }
 }
 
-// grid: x = head * m_tiles + m_tile (then, with kTwo, the second problem's m-tiles), y = token block,
-// z = K split. The tensor maps stay kernel parameters (TMA reads them from parameter space); the
-// body is instantiated once with a single weight map, and once with a second one.
+// Tile (bx, by, bz): x = head * m_tiles + m_tile (then, with kTwo, the second problem's m-tiles),
+// y = token block, z = K split. The tensor maps stay kernel parameters (TMA reads them from parameter
+// space); the body is instantiated once with a single weight map, and once with a second one.
 template <bool kTwo>
 __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
-                                               const CUtensorMap& tm_w2, const Params p) {
+                                               const CUtensorMap& tm_w2, const Params p, const int bx,
+                                               const int by, const int bz) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = (p.M + kBM - 1) / kBM;
-  const bool second = kTwo && (int)blockIdx.x >= p.H * m_tiles;   // a CTA of the second problem
-  const int h = second ? 0 : blockIdx.x / m_tiles;
-  const int mt = second ? blockIdx.x - p.H * m_tiles : blockIdx.x % m_tiles;
+  const int msub = kTwo ? 1 : max(1, p.m_sub);
+  const int cph = (m_tiles + msub - 1) / msub;      // CTAs per head
+  const bool second = kTwo && bx >= p.H * cph;      // a CTA of the second problem
+  const int h = second ? 0 : bx / cph;
+  const int mc = second ? 0 : bx % cph;             // the CTA's place among its head's CTAs
+  const int mt = second ? bx - p.H * cph : mc * msub;   // its first m-tile
   const int M = second ? p.M2 : p.M;
   const CUtensorMap* tw = second ? &tm_w2 : &tm_w;
-  const int tok0 = blockIdx.y * p.tn;
-  const int split = blockIdx.z;
+  const int tok0 = by * p.tn;
+  const int split = bz;
   const int kc0 = split * p.chunks_per_split;
   const int nk = max(0, min(p.K / kBK, kc0 + p.chunks_per_split) - kc0);
   const int S = p.stages;
@@ -114,8 +129,10 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
   const uint32_t slot = done + 8u;
   volatile int* abort = reinterpret_cast<volatile int*>(smem_raw + (done + 16u - raw));   // the issuer gave up
   const uint32_t ring = base + kBarBytes;
-  const uint32_t sbytes = (uint32_t)stage_bytes(p.tn);
-  const uint32_t tmem_cols = p.tn <= 32 ? 32u : (p.tn <= 64 ? 64u : 128u);
+  const uint32_t sbytes = (uint32_t)stage_bytes(p.tn, msub);
+  const uint32_t xoff = (uint32_t)(msub * kABytes);   // the token box after the weight boxes
+  const uint32_t acc_cols = (uint32_t)(msub * p.tn);   // m-subtile j's accumulator: columns [j*tn, (j+1)*tn)
+  const uint32_t tmem_cols = acc_cols <= 32 ? 32u : acc_cols <= 64 ? 64u : acc_cols <= 128 ? 128u : acc_cols <= 256 ? 256u : 512u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { ptx::mbar_init(full0 + 8u * s, 1); ptx::mbar_init(empty0 + 8u * s, 1); }
@@ -126,30 +143,58 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
     ptx::prefetch_tmap(&tm_x);
   }
   if (warp == 2) { ptx::tmem_alloc(slot, tmem_cols); ptx::tmem_relinquish(); }
-  grid_dependency_wait();   // the inputs may come from the previous kernel of the stream
+  // the rotated tail's inverse frequencies (one per pair) depend on no input: into shared memory now
+  const bool rope_tail = p.rope_in != nullptr && !second;
+  double* inv_freq = reinterpret_cast<double*>(smem_raw + (base + kInvFreqOff - raw));
+  if (rope_tail && warp >= 4 && (int)threadIdx.x - 128 < p.d_r / 2)
+    inv_freq[threadIdx.x - 128] = rope_inv_freq((int)threadIdx.x - 128, p.d_r, p.rope_base);
   ptx::tc_fence_before();
   __syncthreads();
-  allow_dependents();
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + (slot - raw));
 
+  // per m-subtile, the two weight boxes (64 k x 64 features each) of K chunk i into stage st (a tile
+  // past M reads the fill value: features are the inner coordinate of the MN-major weight map)
+  auto load_w = [&](int i, uint32_t st, uint32_t fb) {
+    const int kk = (kc0 + i) * kBK;
+    for (int j = 0; j < msub; ++j) {
+      const int m0 = (mt + j) * kBM;
+      const uint32_t sj = st + (uint32_t)j * kABytes;
+      if (p.a_kmajor) {   // rows m of W[h]ᵀ: two boxes of 64 rows x 64 k
+        ptx::tma_load_2d(sj, tw, kk, h * M + m0, fb);
+        ptx::tma_load_2d(sj + kABytes / 2, tw, kk, h * M + m0 + 64, fb);
+      } else {
+        ptx::tma_load_2d(sj, tw, m0, h * p.K + kk, fb);
+        ptx::tma_load_2d(sj + kABytes / 2, tw, m0 + 64, h * p.K + kk, fb);
+      }
+    }
+  };
+  // Weights that no earlier kernel of the stream writes fill the ring's first two stages while that
+  // kernel finishes; the token rows (and everything else) wait for it. (Two, not the whole ring: a
+  // token box issued behind every stage's weights would hold back the first MMA.)
+  const int pre = p.w_early ? min(min(nk, S), 2) : 0;
   if (warp == 0 && lane == 0) {
-    // ---- TMA producer: per K chunk two weight boxes (64 k x 64 features) and one token box
+    for (int i = 0; i < pre; ++i) {
+      ptx::mbar_arrive_expect_tx(full0 + 8u * i, sbytes);
+      load_w(i, ring + i * sbytes, full0 + 8u * i);
+    }
+  }
+  grid_dependency_wait();   // the inputs may come from the previous kernel of the stream
+  allow_dependents();
+
+  if (warp == 0 && lane == 0) {
+    // ---- TMA producer: per K chunk two weight boxes and one token box (64 tokens x 64 k)
     int i = 0;
     for (; i < nk; ++i) {
       const int s = i % S;
-      if (!wait(empty0 + 8u * s, ((i / S) & 1u) ^ 1u, abort)) break;
       const uint32_t st = ring + s * sbytes;
-      const int kk = (kc0 + i) * kBK, k = h * p.K + kk;
-      ptx::mbar_arrive_expect_tx(full0 + 8u * s, sbytes);
-      if (p.a_kmajor) {   // rows m of W[h]ᵀ: two boxes of 64 rows x 64 k
-        ptx::tma_load_2d(st, tw, kk, h * M + mt * kBM, full0 + 8u * s);
-        ptx::tma_load_2d(st + kABytes / 2, tw, kk, h * M + mt * kBM + 64, full0 + 8u * s);
-      } else {
-        ptx::tma_load_2d(st, tw, mt * kBM, k, full0 + 8u * s);
-        ptx::tma_load_2d(st + kABytes / 2, tw, mt * kBM + 64, k, full0 + 8u * s);
+      if (i >= pre) {   // a pre-issued stage is on its first use: free
+        if (!wait(empty0 + 8u * s, ((i / S) & 1u) ^ 1u, abort)) break;
+        ptx::mbar_arrive_expect_tx(full0 + 8u * s, sbytes);
+        load_w(i, st, full0 + 8u * s);
       }
-      ptx::tma_load_2d(st + kABytes, &tm_x, p.x_shared ? kk : k, tok0, full0 + 8u * s);
+      const int kk = (kc0 + i) * kBK;
+      ptx::tma_load_2d(st + xoff, &tm_x, p.x_shared ? kk : h * p.K + kk, tok0, full0 + 8u * s);
     }
     // every load issued must land before the CTA may exit (waited for even after a give-up)
     for (int k = (i > S ? i - S : 0); k < i; ++k) wait(full0 + 8u * (k % S), (k / S) & 1u);
@@ -172,71 +217,117 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
         // a K step of 16 moves 16 rows = 2048 B. A, K-major: 8-feature groups 1024 B apart (the two
         // 64-row boxes are contiguous); a K step moves 32 B inside the swizzle row.
         // B, K-major: 8-token groups 1024 B apart; a K step of 16 moves 32 B inside the swizzle row.
-        const uint64_t ad = p.a_kmajor ? ptx::smem_desc_sw128(st, 16, 1024) : ptx::smem_desc_sw128(st, kABytes / 2, 1024);
         const uint64_t a_step = p.a_kmajor ? 2u : (uint64_t)(2048 >> 4);
-        const uint64_t bd = ptx::smem_desc_sw128(st + kABytes, 16, 1024);
+        const uint64_t bd = ptx::smem_desc_sw128(st + xoff, 16, 1024);
+        for (int j = 0; j < msub; ++j) {
+          const uint32_t sj = st + (uint32_t)j * kABytes;
+          const uint64_t ad = p.a_kmajor ? ptx::smem_desc_sw128(sj, 16, 1024) : ptx::smem_desc_sw128(sj, kABytes / 2, 1024);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          ptx::mma_ss(tmem, ad + (uint64_t)k * a_step, bd + (uint64_t)(2 * k), idesc, (i | k) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k)
+            ptx::mma_ss(tmem + (uint32_t)(j * p.tn), ad + (uint64_t)k * a_step, bd + (uint64_t)(2 * k), idesc,
+                        (i | k) ? 1u : 0u);
+        }
         ptx::mma_commit(empty0 + 8u * s);
       }
     }
     if (!live) *abort = 1;   // the producer stops waiting for stages that will not be freed
     ptx::mma_commit(done);
-  } else if (warp >= 4) {
-    // ---- epilogue: thread = output feature (TMEM lane), 32 tokens (TMEM columns) per load
-    const int row = threadIdx.x - 128;
-    const int m = mt * kBM + row;
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    if (p.rope_in != nullptr && !second) {
+  } else if (warp >= 4 && rope_tail) {
+    {
+      const int row = threadIdx.x - 128;
       // the rotated tail does not depend on the GEMM: done while the main loop runs, the token
-      // block's tokens dealt out over the head's m-tiles (token j of the block goes to m-tile j % m_tiles);
-      // the pairs' inverse frequencies are computed once, into shared memory
+      // block's tokens dealt out over the head's CTAs (token j of the block goes to CTA j % cph)
       const int half = p.d_r / 2;
-      double* inv_freq = reinterpret_cast<double*>(smem_raw + (base + kInvFreqOff - raw));
-      if (row < half) inv_freq[row] = rope_inv_freq(row, p.d_r, p.rope_base);
-      ptx::named_bar_sync(1, 128);
-      const int my_tok = (p.tn - mt + m_tiles - 1) / m_tiles;
-      // four pairs per round, their loads issued together
-      for (int i0 = row; i0 < my_tok * half; i0 += 4 * 128) {
-        __nv_bfloat162 r2[4];
-        int tok[4], q[4], pos[4];
+      const int my_tok = (p.tn - mc + cph - 1) / cph;
+      auto token = [&](int j) { return tok0 + j * cph + mc; };
+      auto out_row = [&](int tok) { return p.y + (int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + p.M; };
+      if (p.vec_out && (half & 3) == 0) {
+        // four pairs (16 bytes) per item, four items per thread per round, all loads issued first
+        const int quads = half / 4, items = my_tok * quads;
+        for (int i0 = row; i0 < items; i0 += 4 * 128) {
+          uint4 v[4];
+          int tok[4], pos[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = i0 + 128 * u;
-          tok[u] = tok0 + (i / half) * m_tiles + mt;
-          q[u] = i % half;
-          const bool live = i < my_tok * half && tok[u] < p.n_tok;
-          if (!live) tok[u] = -1;
-          r2[u] = live ? *reinterpret_cast<const __nv_bfloat162*>(p.rope_in + ((int64_t)tok[u] * p.H + h) * p.d_r + 2 * q[u])
-                       : __floats2bfloat162_rn(0.f, 0.f);
-          pos[u] = live ? p.seqlens[tok[u] / p.s_q] - p.s_q + tok[u] % p.s_q : 0;
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + 128 * u;
+            tok[u] = i < items ? token(i / quads) : p.n_tok;
+            const bool live = tok[u] < p.n_tok;
+            const int g = i % quads;
+            v[u] = live ? *reinterpret_cast<const uint4*>(p.rope_in + ((int64_t)tok[u] * p.H + h) * p.d_r + 8 * g)
+                        : make_uint4(0u, 0u, 0u, 0u);
+            pos[u] = live ? p.seqlens[tok[u] / p.s_q] - p.s_q + tok[u] % p.s_q : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (tok[u] >= p.n_tok) continue;
+            const int g = (i0 + 128 * u) % quads;
+            __nv_bfloat162* x2 = reinterpret_cast<__nv_bfloat162*>(&v[u]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float cs, sn;
+              rope_cos_sin_at_sfu(pos[u], inv_freq[4 * g + e], &cs, &sn);
+              const float x0 = __low2float(x2[e]), x1 = __high2float(x2[e]);
+              x2[e] = __floats2bfloat162_rn(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+            }
+            *reinterpret_cast<uint4*>(out_row(tok[u]) + 8 * g) = v[u];
+          }
         }
+      } else {
+        // one pair per item, four items per thread per round
+        for (int i0 = row; i0 < my_tok * half; i0 += 4 * 128) {
+          __nv_bfloat162 r2[4];
+          int tok[4], q[4], pos[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (tok[u] < 0) continue;
-          float cs, sn;
-          rope_cos_sin_at(pos[u], inv_freq[q[u]], &cs, &sn);
-          const float x0 = __low2float(r2[u]), x1 = __high2float(r2[u]);
-          __nv_bfloat16* o = p.y + (int64_t)tok[u] * p.y_tok_stride + (int64_t)h * p.y_head_stride + p.M;
-          *reinterpret_cast<__nv_bfloat162*>(o + 2 * q[u]) = __floats2bfloat162_rn(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + 128 * u;
+            tok[u] = token(i / half);
+            q[u] = i % half;
+            const bool live = i < my_tok * half && tok[u] < p.n_tok;
+            if (!live) tok[u] = -1;
+            r2[u] = live ? *reinterpret_cast<const __nv_bfloat162*>(p.rope_in + ((int64_t)tok[u] * p.H + h) * p.d_r + 2 * q[u])
+                         : __floats2bfloat162_rn(0.f, 0.f);
+            pos[u] = live ? p.seqlens[tok[u] / p.s_q] - p.s_q + tok[u] % p.s_q : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (tok[u] < 0) continue;
+            float cs, sn;
+            rope_cos_sin_at_sfu(pos[u], inv_freq[q[u]], &cs, &sn);
+            const float x0 = __low2float(r2[u]), x1 = __high2float(r2[u]);
+            *reinterpret_cast<__nv_bfloat162*>(out_row(tok[u]) + 2 * q[u]) =
+                __floats2bfloat162_rn(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+          }
         }
       }
     }
+  }
+  // ---- epilogue: thread = output feature (TMEM lane (warp % 4) * 32 + lane), 32 tokens (TMEM
+  // columns) per load. Warps 4-7 take the even m-subtiles; with two or more, warps 0-3 (their roles
+  // done) take the odd ones.
+  if (warp >= 4 || msub > 1) {
+    __syncwarp();
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const bool ok = __all_sync(0xffffffffu, wait(done, 0));
     ptx::tc_fence_after();
-    if (ok && p.vec_out) {
+    const int jstep = msub > 1 ? 2 : 1;
+    for (int j = warp >= 4 ? 0 : 1; j < msub && ok; j += jstep) {
+    const int mj = mt + j;                        // the m-tile of subtile j
+    if (mj * kBM >= M) break;
+    const uint32_t col0 = (uint32_t)(j * p.tn);   // its accumulator's first TMEM column
+    const int m = mj * kBM + row;
+    if (p.vec_out) {
       // 32 features (the warp's TMEM lanes) x 32 tokens at a time: each thread puts its feature's
       // values in column `lane` of a [token][feature] tile in shared memory (the ring, free once the
       // accumulator is done: 4 KB per warp), then the warp stores the tile's token rows in 16-byte
       // pieces (features are contiguous in every output; M and the strides are multiples of 8).
-      uint8_t* tile = smem_raw + (ring - raw) + (uint32_t)(warp - 4) * 4096u;
-      const uint32_t tile_s = ring + (uint32_t)(warp - 4) * 4096u;
-      const int f0 = mt * kBM + (warp & 3) * 32;   // the warp's first feature
+      uint8_t* tile = smem_raw + (ring - raw) + (uint32_t)(warp ^ 4) * 4096u;
+      const uint32_t tile_s = ring + (uint32_t)(warp ^ 4) * 4096u;
+      const int f0 = mj * kBM + (warp & 3) * 32;   // the warp's first feature
       const bool f32_out = !second && p.mode != 0;
       for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
         uint32_t r[32];
-        ptx::tmem_ld32(tmem + lane_off + (uint32_t)c, r);
+        ptx::tmem_ld32(tmem + lane_off + col0 + (uint32_t)c, r);
         ptx::tmem_wait_ld();
         const int kn = min(32, p.n_tok - tok0 - c);
         if (f32_out) {
@@ -262,10 +353,10 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
         }
         __syncwarp();
       }
-    } else if (ok) {   // any other output layout: one value per store
+    } else {   // any other output layout: one value per store
       for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
         uint32_t r[32];
-        ptx::tmem_ld32(tmem + lane_off + (uint32_t)c, r);
+        ptx::tmem_ld32(tmem + lane_off + col0 + (uint32_t)c, r);
         ptx::tmem_wait_ld();
         if (m >= M) continue;
         const int kn = min(32, p.n_tok - tok0 - c);
@@ -283,6 +374,7 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
         }
       }
     }
+    }
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -294,13 +386,13 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
 
 __global__ void __launch_bounds__(kThreads, 1)
 head_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const Params p) {
-  head_gemm_body<false>(tm_w, tm_x, tm_w, p);
+  head_gemm_body<false>(tm_w, tm_x, tm_w, p, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 head_gemm2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                   const __grid_constant__ CUtensorMap tm_w2, const Params p) {
-  head_gemm_body<true>(tm_w, tm_x, tm_w2, p);
+  head_gemm_body<true>(tm_w, tm_x, tm_w2, p, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // ---- host ----------------------------------------------------------------------------------------
@@ -331,10 +423,20 @@ struct Problem {
   int num_sms = 0;           // SMs of the device (0: unknown)
   bool a_kmajor = false;     // w is [H * M, K] (each head's weight transposed), read K-major
   bool x_shared = false;     // x is [n_tok, K], the same row for every head
+  int m_per_cta = 1;         // m-tiles per CTA (1..4; more than 1 needs MN-major weights, no w2)
 };
 
-// Launches on `st`; returns MLA_OK, or an error status with nothing launched.
-inline int run(const Problem& pr, Params p, cudaStream_t st) {
+constexpr int kSmemMax = 232448;   // 227 KB per CTA
+
+// One problem ready to launch: its parameters with every derived field set, and its tensor maps.
+struct Prepared {
+  Params p;
+  CUtensorMap tm_w, tm_x, tm_w2;
+  int ctas;
+};
+
+// Checks the problem and fills `out` (ring depth at most max_stages); MLA_OK, or an error status.
+inline int prepare(const Problem& pr, Params p, int max_stages, Prepared* out) {
   if (!supported(pr.K, pr.M) || pr.n_tok <= 0 || pr.H <= 0 || pr.splits <= 0) return MLA_ERR_UNSUPPORTED;
   const bool two = pr.w2 != nullptr;
   if ((pr.a_kmajor || pr.x_shared) && (two || p.rope_in != nullptr)) return MLA_ERR_UNSUPPORTED;
@@ -356,39 +458,58 @@ inline int run(const Problem& pr, Params p, cudaStream_t st) {
   p.n_tok = pr.n_tok;
   p.H = pr.H;
   p.tn = tokens_per_cta(pr.n_tok);
+  const int m_tiles = (pr.M + kBM - 1) / kBM;
+  if (pr.m_per_cta < 1 || pr.m_per_cta > 4 || (pr.m_per_cta > 1 && (two || pr.a_kmajor))) return MLA_ERR_UNSUPPORTED;
+  p.m_sub = std::min({pr.m_per_cta, m_tiles, 512 / p.tn});   // the accumulators fit TMEM's 512 columns
   const int chunks = pr.K / kBK;
   p.chunks_per_split = (chunks + pr.splits - 1) / pr.splits;
-  constexpr int kSmemMax = 232448;   // 227 KB per CTA
-  p.stages = std::min({kMaxStages, p.chunks_per_split, (kSmemMax - 2048) / stage_bytes(p.tn)});
-  const int m_ctas = pr.H * ((pr.M + kBM - 1) / kBM) + (two ? (pr.M2 + kBM - 1) / kBM : 0);
-  const int ctas = m_ctas * ((pr.n_tok + p.tn - 1) / p.tn) * pr.splits;
-  // more CTAs than SMs: a ring that lets two CTAs share an SM keeps the whole grid in one wave
-  if (pr.num_sms > 0 && ctas > pr.num_sms)
-    p.stages = std::max(1, std::min(p.stages, (kSmemMax / 2 - 2048) / stage_bytes(p.tn)));
-  CUtensorMap tm_w, tm_x, tm_w2;
+  p.stages = std::max(1, std::min({max_stages, kMaxStages, p.chunks_per_split,
+                                   (kSmemMax - 2048) / stage_bytes(p.tn, p.m_sub)}));
+  p.gx = pr.H * ((m_tiles + p.m_sub - 1) / p.m_sub) + (two ? (pr.M2 + kBM - 1) / kBM : 0);
+  p.gy = (pr.n_tok + p.tn - 1) / p.tn;
+  p.gz = pr.splits;
+  out->ctas = p.gx * p.gy * p.gz;
   if (pr.a_kmajor) {
-    if (!tmap::make_bf16_sw128(&tm_w, pr.w, pr.K, (int64_t)pr.H * pr.M, pr.K, kBK)) return MLA_ERR_INVALID_ARG;
-  } else if (!tmap::make_bf16_sw128(&tm_w, pr.w, pr.M, (int64_t)pr.H * pr.K, pr.M, kBK)) {
+    if (!tmap::make_bf16_sw128(&out->tm_w, pr.w, pr.K, (int64_t)pr.H * pr.M, pr.K, kBK)) return MLA_ERR_INVALID_ARG;
+  } else if (!tmap::make_bf16_sw128(&out->tm_w, pr.w, pr.M, (int64_t)pr.H * pr.K, pr.M, kBK)) {
     return MLA_ERR_INVALID_ARG;
   }
-  if (two && !tmap::make_bf16_sw128(&tm_w2, pr.w2, pr.M2, pr.K, pr.M2, kBK)) return MLA_ERR_INVALID_ARG;
+  out->tm_w2 = out->tm_w;
+  if (two && !tmap::make_bf16_sw128(&out->tm_w2, pr.w2, pr.M2, pr.K, pr.M2, kBK)) return MLA_ERR_INVALID_ARG;
   const int64_t x_cols = pr.x_shared ? (int64_t)pr.K : (int64_t)pr.H * pr.K;
-  if (!tmap::make_bf16_sw128(&tm_x, pr.x, x_cols, pr.n_tok, x_cols, p.tn)) return MLA_ERR_INVALID_ARG;
+  if (!tmap::make_bf16_sw128(&out->tm_x, pr.x, x_cols, pr.n_tok, x_cols, p.tn)) return MLA_ERR_INVALID_ARG;
+  out->p = p;
+  return MLA_OK;
+}
+
+// The kernels' shared-memory limit, raised once per device.
+inline int set_attributes() {
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-    if (cudaFuncSetAttribute(head_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess ||
-        cudaFuncSetAttribute(head_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess)
-      return MLA_ERR_CUDA;
-    if (dev >= 0 && dev < 64) attr_done[dev] = true;
-  }
-  const dim3 grid(m_ctas, (pr.n_tok + p.tn - 1) / p.tn, pr.splits);
-  const size_t smem = (size_t)smem_bytes(p.tn, p.stages);
-  if (two)
-    mla::launch_pdl(head_gemm2_kernel, grid, dim3(kThreads), smem, st, tm_w, tm_x, tm_w2, p);
+  if (dev >= 0 && dev < 64 && attr_done[dev]) return MLA_OK;
+  if (cudaFuncSetAttribute(head_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess ||
+      cudaFuncSetAttribute(head_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (dev >= 0 && dev < 64) attr_done[dev] = true;
+  return MLA_OK;
+}
+
+// Launches on `st`; returns MLA_OK, or an error status with nothing launched.
+inline int run(const Problem& pr, Params p, cudaStream_t st) {
+  Prepared a;
+  int rc = prepare(pr, p, kMaxStages, &a);
+  if (rc) return rc;
+  // more CTAs than SMs: a ring that lets two CTAs share an SM keeps the whole grid in one wave
+  if (pr.num_sms > 0 && a.ctas > pr.num_sms)
+    a.p.stages = std::max(1, std::min(a.p.stages, (kSmemMax / 2 - 2048) / stage_bytes(a.p.tn, a.p.m_sub)));
+  if ((rc = set_attributes())) return rc;
+  const dim3 grid(a.p.gx, a.p.gy, a.p.gz);
+  const size_t smem = (size_t)smem_bytes(a.p.tn, a.p.stages, a.p.m_sub);
+  if (pr.w2 != nullptr)
+    mla::launch_pdl(head_gemm2_kernel, grid, dim3(kThreads), smem, st, a.tm_w, a.tm_x, a.tm_w2, a.p);
   else
-    mla::launch_pdl(head_gemm_kernel, grid, dim3(kThreads), smem, st, tm_w, tm_x, p);
+    mla::launch_pdl(head_gemm_kernel, grid, dim3(kThreads), smem, st, a.tm_w, a.tm_x, a.p);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -99,6 +99,21 @@ mla::gemm::Problem with_sms(mla::gemm::Problem pr) {
 bool append_on_tc(int32_t dtype, int C, int N) { return dtype == MLA_BF16 && mla::gemm::supported(C, N); }
 int append_tc_splits(int n_tok, int C, int N) { return mla::gemm::plan_splits(N, C, n_tok, num_sms(), 64); }
 
+// Launch shape of the a1 finish (one block per new token): with N a multiple of 4 and 16-byte aligned
+// slices, readers of float4 pieces (`groups` slices at a time) plus one warp that finds the row's place
+// meanwhile; otherwise one thread per column.
+struct FinishShape {
+  int threads, groups;
+  size_t smem;
+};
+FinishShape finish_shape(int N, int d_r, const void* part) {
+  if (N % 4 == 0 && aligned16(part) && N / 4 <= 496) {
+    const int groups = std::min(8, 992 / (N / 4));
+    return {mla::simt::finish_readers(N, groups) + 32, groups, ((size_t)(1 + groups) * N + d_r) * sizeof(float)};
+  }
+  return {std::min(1024, (N + 31) / 32 * 32), 0, (size_t)N * sizeof(float)};
+}
+
 // ---- a3 split choice for the CUDA-core decode ---------------------------------------------------
 struct SimtSplit { int nsplit, chunk; };
 SimtSplit simt_split(int n_tok, int H, int max_pages) {
@@ -195,10 +210,11 @@ size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q,
   return (size_t)ks * n_tok * N * sizeof(float);
 }
 
-int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x,
-                     int32_t C, const void* w_dkv_kr, const void* gamma, const int32_t* seqlens,
-                     const int32_t* block_table, int32_t max_pages, const mla_latent_cache_t* cache,
-                     void* workspace, size_t ws_bytes, void* stream) {
+namespace {
+// The arguments of a1 (everything but the workspace); MLA_OK or the error status.
+int append_args(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x, int32_t C,
+                const void* w_dkv_kr, const void* gamma, const int32_t* seqlens, const int32_t* block_table,
+                int32_t max_pages, const mla_latent_cache_t* cache) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
@@ -210,6 +226,16 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     return MLA_ERR_INVALID_ARG;
   if (!stride_ok(cache->latent_stride, dtype, dims->d_c) || !stride_ok(cache->rope_stride, dtype, dims->d_r))
     return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+}  // namespace
+
+int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x,
+                     int32_t C, const void* w_dkv_kr, const void* gamma, const int32_t* seqlens,
+                     const int32_t* block_table, int32_t max_pages, const mla_latent_cache_t* cache,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  int rc = append_args(dims, dtype, B, s_q, x, C, w_dkv_kr, gamma, seqlens, block_table, max_pages, cache);
+  if (rc) return rc;
   const int n_tok = B * s_q, N = dims->d_c + dims->d_r;
   const bool tc = append_on_tc(dtype, C, N);
   const int ks = tc ? append_tc_splits(n_tok, C, N) : append_ksplit(n_tok, C, N);
@@ -217,21 +243,21 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
   if (!workspace || ws_bytes < need) return MLA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MLA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t fin_smem = (size_t)N * sizeof(float);
+  const FinishShape fs = finish_shape(N, dims->d_r, workspace);
   // attributes first: a failure here leaves nothing enqueued
-  if ((rc = dtype == MLA_F32 ? set_smem(mla::simt::append_finish_kernel<float>, fin_smem)
-                             : set_smem(mla::simt::append_finish_kernel<__nv_bfloat16>, fin_smem)))
+  if ((rc = dtype == MLA_F32 ? set_smem(mla::simt::append_finish_kernel<float>, fs.smem)
+                             : set_smem(mla::simt::append_finish_kernel<__nv_bfloat16>, fs.smem)))
     return rc;
   if (tc) {
     using T = __nv_bfloat16;
     mla::gemm::Params p{};
     p.mode = 1;
     p.part = reinterpret_cast<float*>(workspace);
+    p.w_early = 1;
     if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, ks}), p, st))) return rc;
-    const int fin_threads = std::min(1024, (N + 31) / 32 * 32);   // one thread per output column
-    mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)p.part, ks, n_tok, s_q,
+    mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fs.threads), fs.smem, st, (const float*)p.part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
-           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0);
+           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0, fs.groups);
     return launch_status();
   }
   const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
@@ -242,18 +268,18 @@ int mla_append_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s
     using T = float;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, 
         (const T*)x, n_tok, C, (const T*)w_dkv_kr, N, k_chunk, part, nullptr);
-    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, 
+    launch(mla::simt::append_finish_kernel<T>, n_tok, fs.threads, fs.smem, st, 
         part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
         block_table, max_pages, (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride,
-        cache->num_pages, 0);
+        cache->num_pages, 0, fs.groups);
   } else {
     using T = __nv_bfloat16;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, 
         (const T*)x, n_tok, C, (const T*)w_dkv_kr, N, k_chunk, part, nullptr);
-    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, 
+    launch(mla::simt::append_finish_kernel<T>, n_tok, fs.threads, fs.smem, st, 
         part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
         block_table, max_pages, (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride,
-        cache->num_pages, 0);
+        cache->num_pages, 0, fs.groups);
   }
   return launch_status();
 }
@@ -311,6 +337,7 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
     mla::gemm::Params p{};
     p.mode = 1;
     p.part = part;
+    p.w_early = 1;
     if ((rc = mla::gemm::run(with_sms({w_dq, x, 1, C, d_q, n_tok, ks}), p, st))) return rc;
     mla::launch_pdl(mla::simt::rms_rows_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)part, ks,
                     n_tok, d_q, (const T*)gamma_q, dims->rms_eps, (T*)c_q);
@@ -321,6 +348,7 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
     pu.y_tok_stride = (int64_t)H * D;
     pu.y2 = reinterpret_cast<T*>(q_rope_raw);
     pu.y2_tok_stride = (int64_t)H * d_r;
+    pu.w_early = 1;
     mla::gemm::Problem up{w_uq, c_q, 1, d_q, H * D, n_tok, 1};
     up.w2 = w_qr;
     up.M2 = H * d_r;
@@ -350,29 +378,58 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
 // ------------------------------------------------------------------------------------------------
 // a2
 // ------------------------------------------------------------------------------------------------
-int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_nope,
-                 const void* q_rope_raw, const void* w_uk, const int32_t* seqlens, void* q_abs, void* stream) {
+namespace {
+// The arguments of a2; MLA_OK or the error status.
+int absorb_args(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_nope,
+                const void* q_rope_raw, const void* w_uk, const int32_t* seqlens, const void* q_abs) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
   if (!tokens_ok(B, s_q) || !q_nope || !q_rope_raw || !w_uk || !seqlens || !q_abs) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_nope) || !aligned16(q_rope_raw) || !aligned16(w_uk) || !aligned16(q_abs) || !aligned16(seqlens))
     return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+// a2 on the tensor cores: bf16, whole 64-wide K chunks, 16-byte weight rows, a RoPE tail that fits.
+bool absorb_on_tc(const mla_dims_t* dims, int32_t dtype) {
+  return dtype == MLA_BF16 && mla::gemm::supported(dims->D, dims->d_c) && mla::gemm::supported_rope(dims->d_r);
+}
+
+// The tensor-core problem of a2: per head, q_nope[:, h, :] · W_UK[h] into q_abs[:, h, 0:d_c], with the
+// rotated tail q_abs[:, h, d_c:] written by the m-tile-0 CTAs.
+void absorb_problem(const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_nope, const void* q_rope_raw,
+                    const void* w_uk, const int32_t* seqlens, void* q_abs, mla::gemm::Problem* pr,
+                    mla::gemm::Params* p) {
+  const int H = dims->H, d_c = dims->d_c, d_r = dims->d_r;
+  *p = mla::gemm::Params{};
+  p->mode = 0;
+  p->y = reinterpret_cast<__nv_bfloat16*>(q_abs);
+  p->y_tok_stride = (int64_t)H * (d_c + d_r);
+  p->y_head_stride = d_c + d_r;
+  p->rope_in = reinterpret_cast<const __nv_bfloat16*>(q_rope_raw);
+  p->d_r = d_r;
+  p->s_q = s_q;
+  p->seqlens = seqlens;
+  p->rope_base = dims->rope_base;
+  p->w_early = 1;
+  *pr = with_sms({w_uk, q_nope, H, dims->D, d_c, B * s_q, 1});
+  pr->m_per_cta = 2;   // two CTAs per head and token block, each streaming half of W_UK[h]
+}
+}  // namespace
+
+int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_nope,
+                 const void* q_rope_raw, const void* w_uk, const int32_t* seqlens, void* q_abs, void* stream) {
+  int rc = absorb_args(dims, dtype, B, s_q, q_nope, q_rope_raw, w_uk, seqlens, q_abs);
+  if (rc) return rc;
   const int n_tok = B * s_q;
   const int D = dims->D, H = dims->H, d_c = dims->d_c, d_r = dims->d_r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == MLA_BF16 && mla::gemm::supported(D, d_c) && mla::gemm::supported_rope(d_r)) {
-    mla::gemm::Params p{};
-    p.mode = 0;
-    p.y = reinterpret_cast<__nv_bfloat16*>(q_abs);
-    p.y_tok_stride = (int64_t)H * (d_c + d_r);
-    p.y_head_stride = d_c + d_r;
-    p.rope_in = reinterpret_cast<const __nv_bfloat16*>(q_rope_raw);
-    p.d_r = d_r;
-    p.s_q = s_q;
-    p.seqlens = seqlens;
-    p.rope_base = dims->rope_base;
-    return mla::gemm::run(with_sms({w_uk, q_nope, H, D, d_c, n_tok, 1}), p, st);
+  if (absorb_on_tc(dims, dtype)) {
+    mla::gemm::Problem pr;
+    mla::gemm::Params p;
+    absorb_problem(dims, B, s_q, q_nope, q_rope_raw, w_uk, seqlens, q_abs, &pr, &p);
+    return mla::gemm::run(pr, p, st);
   }
   dim3 grid(H, (n_tok + mla::simt::HG_TOK - 1) / mla::simt::HG_TOK);
   const size_t smem = (size_t)mla::simt::HG_TOK * D * sizeof(float);
@@ -390,6 +447,26 @@ int mla_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
         seqlens, s_q, dims->rope_base);
   }
   return launch_status();
+}
+
+// ------------------------------------------------------------------------------------------------
+// a1 + a2 in one call
+// ------------------------------------------------------------------------------------------------
+int mla_append_cache_absorb_q(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* x,
+                              int32_t C, const void* w_dkv_kr, const void* gamma, const void* q_nope,
+                              const void* q_rope_raw, const void* w_uk, const int32_t* seqlens,
+                              const int32_t* block_table, int32_t max_pages, const mla_latent_cache_t* cache,
+                              void* q_abs, void* workspace, size_t ws_bytes, void* stream) {
+  // every argument of both halves is checked before anything is launched
+  int rc = append_args(dims, dtype, B, s_q, x, C, w_dkv_kr, gamma, seqlens, block_table, max_pages, cache);
+  if (rc) return rc;
+  if ((rc = absorb_args(dims, dtype, B, s_q, q_nope, q_rope_raw, w_uk, seqlens, q_abs))) return rc;
+  if (mla_append_workspace_size(dims, B, s_q, C) > ws_bytes || !workspace) return MLA_ERR_WORKSPACE;
+  // the append first: the absorption's CTAs then stream W_UK while the append's finish runs
+  if ((rc = mla_append_cache(dims, dtype, B, s_q, x, C, w_dkv_kr, gamma, seqlens, block_table, max_pages, cache,
+                             workspace, ws_bytes, stream)))
+    return rc;
+  return mla_absorb_q(dims, dtype, B, s_q, q_nope, q_rope_raw, w_uk, seqlens, q_abs, stream);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -538,6 +615,7 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
     p.y = reinterpret_cast<__nv_bfloat16*>(out);
     p.y_tok_stride = (int64_t)H * d_v;
     p.y_head_stride = d_v;
+    p.w_early = 1;
     if ((rc = mla::gemm::run(with_sms({w_uv, o_lat, H, d_c, d_v, n_tok, 1}), p, st))) return rc;
     if (w_o) {
       if (mla::gemm::supported(K, C)) {   // the heads concatenated, times W_O, on the tensor cores
@@ -546,6 +624,7 @@ int mla_out_proj(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, 
         po.y = reinterpret_cast<__nv_bfloat16*>(out_model);
         po.y_tok_stride = C;
         po.y_head_stride = 0;
+        po.w_early = 1;
         if ((rc = mla::gemm::run(with_sms({w_o, out, 1, K, C, n_tok, 1}), po, st))) return rc;
       } else {
         using T = __nv_bfloat16;
@@ -702,8 +781,8 @@ int mla_append_gqa_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32
   T* kbuf = reinterpret_cast<T*>(ws + lay.kbuf);
   T* vbuf = reinterpret_cast<T*>(ws + lay.vbuf);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t fin_smem = (size_t)N * sizeof(float);
-  if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fin_smem))) return rc;
+  const FinishShape fs = finish_shape(N, dims->d_r, part);
+  if ((rc = set_smem(mla::simt::append_finish_kernel<T>, fs.smem))) return rc;
   // 1. z = x · [W_DKV | W_KR] (split-K partial sums)
   mla::gemm::Params p{};
   p.mode = 1;
@@ -711,11 +790,10 @@ int mla_append_gqa_cache(const mla_dims_t* dims, int32_t dtype, int32_t B, int32
   if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, lay.ks}), p, st))) return rc;
   // 2. c = RMSNorm(z_c)·gamma into a plain buffer (rounded to the storage type, as a latent cache row
   //    would be); k_r = RoPE(z_r) into the cache's RoPE rows
-  const int fin_threads = std::min(1024, (N + 31) / 32 * 32);
-  mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)part,
+  mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fs.threads), fs.smem, st, (const float*)part,
                   lay.ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens,
                   block_table, max_pages, cbuf, (int64_t)dims->d_c, (T*)cache->rope, cache->rope_stride,
-                  cache->num_pages, 1);
+                  cache->num_pages, 1, fs.groups);
   // 3. K_g = W_UK[g] · c (W_UK stored [g, D, d_c]: read K-major), V_g = c · W_UV[g], every group
   mla::gemm::Problem pk{w_uk_g, cbuf, g, dims->d_c, dims->D, n_tok, 1};
   pk.a_kmajor = true;
@@ -863,13 +941,13 @@ extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, i
   const int cap = (int)(kAppendScratchFloats / per_slice);
   const bool tc = append_on_tc(dtype, C, N);
   const int ks = std::min(tc ? append_tc_splits(n_tok, C, N) : append_ksplit(n_tok, C, N), cap);
-  const size_t fin_smem = (size_t)N * sizeof(float);
-  // attributes first: a failure here leaves nothing enqueued
-  if ((rc = dtype == MLA_F32 ? set_smem(mla::simt::append_finish_kernel<float>, fin_smem)
-                             : set_smem(mla::simt::append_finish_kernel<__nv_bfloat16>, fin_smem)))
-    return rc;
   float* part = nullptr;
   if ((rc = append_scratch_address(&part))) return rc;
+  const FinishShape fs = finish_shape(N, dims->d_r, part);
+  // attributes first: a failure here leaves nothing enqueued
+  if ((rc = dtype == MLA_F32 ? set_smem(mla::simt::append_finish_kernel<float>, fs.smem)
+                             : set_smem(mla::simt::append_finish_kernel<__nv_bfloat16>, fs.smem)))
+    return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (tc) {
     // the tensor-core projection writes one fp32 slice per K split (an empty split writes zeros)
@@ -878,11 +956,10 @@ extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, i
     p.mode = 1;
     p.part = part;
     if ((rc = mla::gemm::run(with_sms({w_dkv_kr, x, 1, C, N, n_tok, ks}), p, st))) return rc;
-    const int fin_threads = std::min(1024, (N + 31) / 32 * 32);
-    mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st,
+    mla::launch_pdl(mla::simt::append_finish_kernel<T>, dim3(n_tok), dim3(fs.threads), fs.smem, st,
                     (const float*)part, ks, n_tok, s_q, dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps,
                     dims->rope_base, seqlens, block_table, max_pages, (T*)cache->latent, cache->latent_stride,
-                    (T*)cache->rope, cache->rope_stride, cache->num_pages, 0);
+                    (T*)cache->rope, cache->rope_stride, cache->num_pages, 0, fs.groups);
     return launch_status();
   }
   const int k_chunk = ((C + ks - 1) / ks + 63) / 64 * 64;
@@ -892,16 +969,16 @@ extern "C" int mla_append_cache_noalloc(const mla_dims_t* dims, int32_t dtype, i
     using T = float;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, (const T*)x, n_tok, C,
            (const T*)w_dkv_kr, N, k_chunk, part, (T*)nullptr);
-    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)part, ks, n_tok, s_q,
+    launch(mla::simt::append_finish_kernel<T>, n_tok, fs.threads, fs.smem, st, (const float*)part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
-           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0);
+           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0, fs.groups);
   } else {
     using T = __nv_bfloat16;
     launch(mla::simt::proj_partial_kernel<T>, grid, mla::simt::PROJ_COLS, 0, st, (const T*)x, n_tok, C,
            (const T*)w_dkv_kr, N, k_chunk, part, (T*)nullptr);
-    launch(mla::simt::append_finish_kernel<T>, n_tok, 256, fin_smem, st, (const float*)part, ks, n_tok, s_q,
+    launch(mla::simt::append_finish_kernel<T>, n_tok, fs.threads, fs.smem, st, (const float*)part, ks, n_tok, s_q,
            dims->d_c, dims->d_r, (const T*)gamma, dims->rms_eps, dims->rope_base, seqlens, block_table, max_pages,
-           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0);
+           (T*)cache->latent, cache->latent_stride, (T*)cache->rope, cache->rope_stride, cache->num_pages, 0, fs.groups);
   }
   return launch_status();
 }

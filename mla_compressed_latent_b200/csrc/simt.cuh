@@ -72,10 +72,15 @@ __device__ __forceinline__ float sum_slices(const float* src, int ksplit, int64_
 
 // =============================================================================================
 // a1 epilogue: sum the K slices, RMSNorm the latent part, rotate the RoPE part, store the row.
-// One block per new token (a thread per column sums that column's K slices, many loads in flight);
-// the latent row is written 16 bytes at a time. With
-// latent_by_token the latent row of token tok goes to latent + tok * lat_stride (a plain buffer)
-// instead of its cache slot; the RoPE key always goes to its cache slot.
+// One block per new token. With groups > 0 (N % 4 == 0, 16-byte aligned slices; blockDim.x =
+// L + 32 where L = groups * N/4 rounded up to a warp; dynamic shared memory (1 + groups) * N + d_r
+// floats) the first groups * N/4 threads read the slices in 16-byte pieces: thread (g, q) sums
+// columns 4q..4q+3 over slices g, g + groups, ... (all of its loads in flight together), and the
+// groups' sums are then added in a fixed order; meanwhile the last warp finds the token's cache row
+// and the rotation's cos/sin, so that no dependent load is left after the sums. With groups == 0 a
+// thread per column sums that column's slices and the row is found afterwards. The latent row is
+// written 16 bytes at a time. With latent_by_token the latent row of token tok goes to latent + tok *
+// lat_stride (a plain buffer) instead of its cache slot; the RoPE key always goes to its cache slot.
 // =============================================================================================
 template <typename T> struct Vec16;
 template <> struct Vec16<float> {
@@ -98,34 +103,86 @@ template <> struct Vec16<__nv_bfloat16> {
   }
 };
 
+// threads of the slice readers in the groups > 0 layout (the place-finding warp follows them)
+__host__ __device__ inline int finish_readers(int N, int groups) { return (groups * (N / 4) + 31) / 32 * 32; }
+
 template <typename T>
 __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit, int n_tok, int s_q,
                                      int d_c, int d_r, const T* __restrict__ gamma, float eps,
                                      float rope_base, const int32_t* __restrict__ seqlens,
                                      const int32_t* __restrict__ block_table, int max_pages,
                                      T* latent, int64_t lat_stride, T* rope, int64_t rope_stride,
-                                     int num_pages, int latent_by_token) {
+                                     int num_pages, int latent_by_token, int groups) {
   extern __shared__ float z[];
   __shared__ float red[32];
+  __shared__ long long s_row;   // the token's cache row; -1: none (reported)
+  __shared__ int s_pos;
   grid_dependency_wait();   // launched with programmatic dependent launch after the projection
   allow_dependents();
   const int tok = blockIdx.x;
   const int b = tok / s_q, t = tok % s_q;
-  const int N = d_c + d_r;
-  // one column per thread, up to 32 slices' loads in flight per thread
-  for (int i = threadIdx.x; i < N; i += blockDim.x)
-    z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
+  const int N = d_c + d_r, half = d_r / 2;
+  float* cs_sn = z + (1 + groups) * N;   // groups > 0: cos, sin of pair i at [2i], [2i + 1]
+  if (groups > 0) {
+    const int Q = N / 4, readers = finish_readers(N, groups);
+    float* acc = z + N;   // [groups][N]
+    if ((int)threadIdx.x >= readers) {
+      // the place-finding warp: position, cache row, then the rotation of every pair
+      const int lane = threadIdx.x - readers;
+      int pos = 0;
+      if (lane == 0) {
+        long long row = -1;
+        pos = seqlens[b] - s_q + t;
+        if (pos < 0 || (pos >> 6) >= max_pages) report(MLA_ERR_DEVICE_CHECK);
+        else row = cache_row(block_table + (int64_t)b * max_pages, pos, num_pages);
+        s_row = row;
+        s_pos = pos;
+      }
+      pos = __shfl_sync(0xffffffffu, pos, 0);
+      for (int i = lane; i < half; i += 32) rope_cos_sin(pos, i, d_r, rope_base, &cs_sn[2 * i], &cs_sn[2 * i + 1]);
+    } else if ((int)threadIdx.x < groups * Q) {
+      const int q = threadIdx.x % Q, g = threadIdx.x / Q;
+      const float4* src = reinterpret_cast<const float4*>(part + (int64_t)tok * N) + q;
+      const int64_t step = (int64_t)n_tok * Q;   // one slice, in float4
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = g; s0 < ksplit; s0 += 8 * groups) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int sl = s0 + u * groups;
+          v[u] = sl < ksplit ? __ldcg(src + sl * step) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) { a.x += v[u].x; a.y += v[u].y; a.z += v[u].z; a.w += v[u].w; }
+      }
+      reinterpret_cast<float4*>(acc + g * N)[q] = a;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+      float v = 0.f;
+      for (int g = 0; g < groups; ++g) v += acc[g * N + i];
+      z[i] = v;
+    }
+  } else {
+    // one column per thread, up to 32 slices' loads in flight per thread
+    for (int i = threadIdx.x; i < N; i += blockDim.x)
+      z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
+    if (threadIdx.x == 0) {
+      long long row = -1;
+      const int pos = seqlens[b] - s_q + t;
+      if (pos < 0 || (pos >> 6) >= max_pages) report(MLA_ERR_DEVICE_CHECK);
+      else row = cache_row(block_table + (int64_t)b * max_pages, pos, num_pages);
+      s_row = row;
+      s_pos = pos;
+    }
+  }
   __syncthreads();
   float ss = 0.f;
   for (int i = threadIdx.x; i < d_c; i += blockDim.x) ss = fmaf(z[i], z[i], ss);
   ss = block_sum(ss, red);
   const float inv = 1.0f / sqrtf(ss / (float)d_c + eps);
-  const int pos = seqlens[b] - s_q + t;
-  if (pos < 0 || (pos >> 6) >= max_pages) {
-    if (threadIdx.x == 0) report(MLA_ERR_DEVICE_CHECK);
-    return;
-  }
-  const int64_t row = cache_row(block_table + (int64_t)b * max_pages, pos, num_pages);
+  const int64_t row = s_row;
+  const int pos = s_pos;
   if (row < 0) return;
   T* lrow = latent + (latent_by_token ? (int64_t)tok : row) * lat_stride;
   constexpr int V = Vec16<T>::n;
@@ -139,9 +196,14 @@ __global__ void append_finish_kernel(const float* __restrict__ part, int ksplit,
   } else {
     for (int i = threadIdx.x; i < d_c; i += blockDim.x) st(lrow + i, z[i] * inv * (gamma ? ld(gamma + i) : 1.f));
   }
-  for (int i = threadIdx.x; i < d_r / 2; i += blockDim.x) {
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
     float cs, sn;
-    rope_cos_sin(pos, i, d_r, rope_base, &cs, &sn);
+    if (groups > 0) {
+      cs = cs_sn[2 * i];
+      sn = cs_sn[2 * i + 1];
+    } else {
+      rope_cos_sin(pos, i, d_r, rope_base, &cs, &sn);
+    }
     const float a = z[d_c + 2 * i], bb = z[d_c + 2 * i + 1];
     st(rope + row * rope_stride + 2 * i, a * cs - bb * sn);
     st(rope + row * rope_stride + 2 * i + 1, a * sn + bb * cs);

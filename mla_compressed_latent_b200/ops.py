@@ -186,6 +186,26 @@ def mla_absorb_q(dims: Dims, q_nope, q_rope_raw, w_uk, seqlens, q_abs=None, stre
     return q_abs
 
 
+def mla_append_cache_absorb_q(dims: Dims, x, w_dkv_kr, gamma, q_nope, q_rope_raw, w_uk, seqlens, block_table,
+                              cache: LatentCache, q_abs=None, workspace=None, stream=None):
+    """mla_append_cache and mla_absorb_q of one step in one call (their projections share a launch);
+    returns q_abs."""
+    lib = L.load()
+    B, s_q, C = x.shape
+    if q_abs is None:
+        q_abs = torch.empty(B, s_q, dims.H, dims.d_c + dims.d_r, dtype=q_nope.dtype, device=q_nope.device)
+    d = dims.c()
+    need = lib.mla_append_workspace_size(ctypes.byref(d), B, s_q, C)
+    workspace, wsb = _workspace(need, x.device, workspace)
+    cc = cache.c()
+    rc = lib.mla_append_cache_absorb_q(ctypes.byref(d), _dt(x), B, s_q, _ptr(x), C, _ptr(w_dkv_kr), _ptr(gamma),
+                                       _ptr(q_nope), _ptr(q_rope_raw), _ptr(w_uk), _ptr(_i32(seqlens)),
+                                       _ptr(_i32(block_table)), block_table.shape[1], ctypes.byref(cc), _ptr(q_abs),
+                                       _ptr(workspace) if workspace is not None else None, wsb, _stream(stream))
+    _check("mla_append_cache_absorb_q", rc)
+    return q_abs
+
+
 def mla_decode_workspace_size(dims: Dims, dtype, B, s_q, max_pages) -> int:
     d = dims.c()
     return L.load().mla_decode_workspace_size(ctypes.byref(d), _DTYPES[dtype], B, s_q, max_pages)

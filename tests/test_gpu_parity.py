@@ -214,6 +214,42 @@ def test_absorb_q(name, s_q):
         _assert_close(got[b][..., w.d_c:], ref[..., w.d_c:], w.dtype, f"rotated query seq {b}")
 
 
+@pytest.mark.parametrize("name,B,s_q", [("dsv3_b64_l4096", 64, 1), ("dsv3_b64_l4096", 5, 3),
+                                        ("dsv3_b64_l4096", 300, 1), ("smallem_fp32", 3, 2)])
+def test_append_cache_absorb_q(name, B, s_q):
+    """a1 and a2 in one call: the new rows and q_abs against the oracle, q_abs identical to
+    mla_absorb_q's, every other pool row untouched."""
+    w = synth.workload(name, B=B, s_q=s_q, lengths=("list", tuple(4096 - 3 * i for i in range(B))))
+    case = Case(w)
+    dev = case.to_device()
+    cache = _cache(dev, case)
+    before = dev["pool"].clone()
+    dims = Dims.of(w)
+    q_abs = ops.mla_append_cache_absorb_q(dims, dev["x"], dev["w_dkv_kr"], None, dev["q_nope"], dev["q_rope_raw"],
+                                          dev["W_UK"], dev["seqlens"], dev["table"], cache)
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    assert torch.equal(q_abs, ops.mla_absorb_q(dims, dev["q_nope"], dev["q_rope_raw"], dev["W_UK"], dev["seqlens"]))
+    got_q = q_abs.to(torch.float64).cpu().numpy()
+    for b in sorted({0, B // 2, B - 1}):
+        pos = O.token_positions(int(case.lens[b]), s_q)
+        ref = O.absorb_query(case.q_nope64[b], case.q_rope_raw64[b], case.W64["W_UK"], pos, w.rope_base)
+        _assert_close(got_q[b], ref, w.dtype, f"q_abs seq {b}")
+    # token (b, t) is at position L_b - s_q + t
+    pos = (case.lens[:, None] - s_q + np.arange(s_q)[None, :]).reshape(-1).astype(np.int64)
+    seq = np.repeat(np.arange(B), s_q)
+    c_ref, kr_ref = O.latent_rows(case.x64.reshape(B * s_q, w.C), case.W64["W_DKV"], case.W64["W_KR"], pos, None,
+                                  w.rms_eps, w.rope_base)
+    rows = case.table[seq, pos // 64].astype(np.int64) * 64 + pos % 64
+    pool = dev["pool"].cpu()
+    got = pool[torch.from_numpy(rows)].to(torch.float64).numpy()
+    _assert_close(got[:, :w.d_c], c_ref, w.dtype, "appended latent")
+    _assert_close(got[:, w.d_c:], kr_ref, w.dtype, "appended rope key")
+    mask = torch.ones(pool.shape[0], dtype=torch.bool)
+    mask[torch.from_numpy(rows)] = False
+    assert torch.equal(pool[mask], before.cpu()[mask])
+
+
 @pytest.mark.parametrize("name", ["dsv3_b64_l4096", "smallem_fp32"])
 def test_out_proj(name):
     w = synth.workload(name, B=5, s_q=2)

@@ -73,6 +73,10 @@ CALLS = {
     # B, s_q, q_abs, cache, table, max_pages, seqlens, o_lat, lse, ws, ws_bytes, stream
     "mla_decode_absorbed": ([64, 1, P, "LC", P, 64, P, P, P, P, BIG_WS, None],
                             [2, 4, 6, 7, 8], [0, 1, 5], 9, []),
+    # B, s_q, x, C, w_dkv_kr, gamma, q_nope, q_rope_raw, w_uk, seqlens, table, max_pages, cache, q_abs,
+    # ws, ws_bytes, stream
+    "mla_append_cache_absorb_q": ([64, 1, P, 7168, P, P, P, P, P, P, P, 64, "LC", P, P, BIG_WS, None],
+                                  [2, 4, 6, 7, 8, 9, 10, 13], [0, 1, 3, 11], 14, [5]),
     # B, s_q, o_lat, w_uv, out, w_o, C, out_model, stream
     "mla_out_proj": ([64, 1, P, P, P, P, 7168, P, None], [2, 3, 4, 7], [0, 1, 6], None, [5]),
     # B, s_q, q_nope, q_rope_raw, cache, table, max_pages, seqlens, out, lse, ws, ws_bytes, stream
@@ -176,6 +180,9 @@ def test_bad_latent_cache_is_rejected(lib, field, value):
     assert rc == L.MLA_ERR_INVALID_ARG
     rc = lib.mla_append_cache(ctypes.byref(d), 1, 64, 1, g, 7168, g, None, g, g, 64, ctypes.byref(cache), g,
                               BIG_WS, None)
+    assert rc == L.MLA_ERR_INVALID_ARG
+    rc = lib.mla_append_cache_absorb_q(ctypes.byref(d), 1, 64, 1, g, 7168, g, None, g, g, g, g, g, 64,
+                                       ctypes.byref(cache), g, g, BIG_WS, None)
     assert rc == L.MLA_ERR_INVALID_ARG
 
 
