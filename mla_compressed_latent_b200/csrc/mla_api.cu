@@ -99,6 +99,21 @@ mla::gemm::Problem with_sms(mla::gemm::Problem pr) {
 bool append_on_tc(int32_t dtype, int C, int N) { return dtype == MLA_BF16 && mla::gemm::supported(C, N); }
 int append_tc_splits(int n_tok, int C, int N) { return mla::gemm::plan_splits(N, C, n_tok, num_sms(), 64); }
 
+// Launch shape of the query chain's RMS step (one block per token): float4 slice reads in `groups`
+// interleaved sets when N is a multiple of 4 and the slices are 16-byte aligned.
+struct RmsShape {
+  int threads, groups;
+  size_t smem;
+};
+RmsShape rms_shape(int N, const void* part) {
+  if (N % 4 == 0 && aligned16(part) && N / 4 <= mla::simt::RMS_THREADS) {
+    const int groups = std::min(8, mla::simt::RMS_THREADS / (N / 4));
+    return {std::min(mla::simt::RMS_THREADS, (groups * (N / 4) + 31) / 32 * 32), groups,
+            (size_t)(1 + groups) * N * sizeof(float)};
+  }
+  return {std::min(mla::simt::RMS_THREADS, (N + 31) / 32 * 32), 0, (size_t)N * sizeof(float)};
+}
+
 // Launch shape of the a1 finish (one block per new token): with N a multiple of 4 and 16-byte aligned
 // slices, readers of float4 pieces (`groups` slices at a time) plus one warp that finds the row's place
 // meanwhile; otherwise one thread per column.
@@ -326,11 +341,10 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* part = reinterpret_cast<float*>(workspace);
   void* c_q = reinterpret_cast<char*>(workspace) + pb;
-  const size_t fin_smem = (size_t)d_q * sizeof(float);
-  const int fin_threads = std::min(mla::simt::RMS_THREADS, (d_q + 31) / 32 * 32);
+  const RmsShape rs = rms_shape(d_q, part);
   // attributes first: a failure here leaves nothing enqueued
-  if ((rc = dtype == MLA_F32 ? set_smem(mla::simt::rms_rows_kernel<float>, fin_smem)
-                             : set_smem(mla::simt::rms_rows_kernel<__nv_bfloat16>, fin_smem)))
+  if ((rc = dtype == MLA_F32 ? set_smem(mla::simt::rms_rows_kernel<float>, rs.smem)
+                             : set_smem(mla::simt::rms_rows_kernel<__nv_bfloat16>, rs.smem)))
     return rc;
   if (tc) {
     using T = __nv_bfloat16;
@@ -339,8 +353,8 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
     p.part = part;
     p.w_early = 1;
     if ((rc = mla::gemm::run(with_sms({w_dq, x, 1, C, d_q, n_tok, ks}), p, st))) return rc;
-    mla::launch_pdl(mla::simt::rms_rows_kernel<T>, dim3(n_tok), dim3(fin_threads), fin_smem, st, (const float*)part, ks,
-                    n_tok, d_q, (const T*)gamma_q, dims->rms_eps, (T*)c_q);
+    mla::launch_pdl(mla::simt::rms_rows_kernel<T>, dim3(n_tok), dim3(rs.threads), rs.smem, st, (const float*)part, ks,
+                    n_tok, d_q, (const T*)gamma_q, dims->rms_eps, (T*)c_q, rs.groups);
     // both up-projections in one launch, each a single-"head" GEMM over its whole output width
     mla::gemm::Params pu{};
     pu.mode = 0;
@@ -363,8 +377,8 @@ int mla_project_query(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t 
     using T = decltype(zero);
     launch(mla::simt::proj_partial_kernel<T>, dim3(cols(d_q), tok_blocks, ks), mla::simt::PROJ_COLS, 0, st,
            (const T*)x, n_tok, C, (const T*)w_dq, d_q, k_chunk, part, (T*)nullptr);
-    launch(mla::simt::rms_rows_kernel<T>, n_tok, fin_threads, fin_smem, st, (const float*)part, ks, n_tok, d_q,
-           (const T*)gamma_q, dims->rms_eps, (T*)c_q);
+    launch(mla::simt::rms_rows_kernel<T>, n_tok, rs.threads, rs.smem, st, (const float*)part, ks, n_tok, d_q,
+           (const T*)gamma_q, dims->rms_eps, (T*)c_q, rs.groups);
     // one K slice: the kernel writes the finished dot products straight to its output
     launch(mla::simt::proj_partial_kernel<T>, dim3(cols(H * D), tok_blocks, 1), mla::simt::PROJ_COLS, 0, st,
            (const T*)c_q, n_tok, d_q, (const T*)w_uq, H * D, d_q, (float*)nullptr, (T*)q_nope);

@@ -264,29 +264,68 @@ __global__ void reduce_slices_kernel(const float* __restrict__ part, int ksplit,
 
 // =============================================================================================
 // Query chain, middle step: c_q = RMSNorm(sum of the K slices of x·W_DQ) · gamma_q, one row of N
-// values per token, stored in T. One block per token (blockDim a multiple of 32, at most
-// RMS_THREADS: the launch bound keeps the block's registers within the SM's).
+// values per token, stored in T. One block per token. With groups > 0 (N % 4 == 0, 16-byte aligned
+// slices, blockDim.x >= groups * N/4, dynamic shared memory (1 + groups) * N floats) thread (g, q)
+// sums columns 4q..4q+3 over slices g, g + groups, ... with all of its loads in flight, and the
+// groups' sums are added in a fixed order; with groups == 0 a thread per column sums its slices.
+// Rows of N % 8 == 0 bf16 values (or N % 4 fp32) are stored 16 bytes at a time.
 // =============================================================================================
-constexpr int RMS_THREADS = 512;
+constexpr int RMS_THREADS = 1024;
 
 template <typename T>
 __global__ void __launch_bounds__(RMS_THREADS) rms_rows_kernel(const float* __restrict__ part, int ksplit, int n_tok, int N,
-                                const T* __restrict__ gamma, float eps, T* __restrict__ out) {
+                                const T* __restrict__ gamma, float eps, T* __restrict__ out, int groups) {
   extern __shared__ float z[];
   __shared__ float red[32];
   grid_dependency_wait();   // launched with programmatic dependent launch after the projection
   allow_dependents();
   const int tok = blockIdx.x;
-  for (int i = threadIdx.x; i < N; i += blockDim.x)
-    z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
+  if (groups > 0) {
+    const int Q = N / 4;
+    float* acc = z + N;   // [groups][N]
+    if ((int)threadIdx.x < groups * Q) {
+      const int q = threadIdx.x % Q, g = threadIdx.x / Q;
+      const float4* src = reinterpret_cast<const float4*>(part + (int64_t)tok * N) + q;
+      const int64_t step = (int64_t)n_tok * Q;   // one slice, in float4
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = g; s0 < ksplit; s0 += 8 * groups) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int sl = s0 + u * groups;
+          v[u] = sl < ksplit ? __ldcg(src + sl * step) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) { a.x += v[u].x; a.y += v[u].y; a.z += v[u].z; a.w += v[u].w; }
+      }
+      reinterpret_cast<float4*>(acc + g * N)[q] = a;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+      float v = 0.f;
+      for (int g = 0; g < groups; ++g) v += acc[g * N + i];
+      z[i] = v;
+    }
+  } else {
+    for (int i = threadIdx.x; i < N; i += blockDim.x)
+      z[i] = sum_slices(part + (int64_t)tok * N + i, ksplit, (int64_t)n_tok * N);
+  }
   __syncthreads();
   float ss = 0.f;
   for (int i = threadIdx.x; i < N; i += blockDim.x) ss = fmaf(z[i], z[i], ss);
   ss = block_sum(ss, red);
   const float inv = 1.0f / sqrtf(ss / (float)N + eps);
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
-    const float gm = gamma ? ld(gamma + i) : 1.f;
-    st(out + (int64_t)tok * N + i, z[i] * inv * gm);
+  T* row = out + (int64_t)tok * N;
+  constexpr int V = Vec16<T>::n;
+  if (N % V == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+    for (int i = threadIdx.x * V; i < N; i += blockDim.x * V) {
+      float v[V];
+#pragma unroll
+      for (int u = 0; u < V; ++u) v[u] = z[i + u] * inv * (gamma ? ld(gamma + i + u) : 1.f);
+      Vec16<T>::store(row + i, v);
+    }
+  } else {
+    for (int i = threadIdx.x; i < N; i += blockDim.x) st(row + i, z[i] * inv * (gamma ? ld(gamma + i) : 1.f));
   }
 }
 
