@@ -23,6 +23,7 @@
 // Every wait is bounded in time; on expiry the kernel records MLA_ERR_TIMEOUT and drains.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda.h>
 
 #include "common.cuh"
@@ -101,8 +102,8 @@ enum Bar : int {
 };
 constexpr int kOffTmemSlot = kOffBar + NUM_BARS * 8;
 constexpr int kOffAbort = kOffTmemSlot + 8;
-constexpr int kOffWork = kOffAbort + 8;                // long long start, end, off_b, b, total tiles
-constexpr int kSmemUsed = kOffWork + 40;
+constexpr int kOffWork = kOffAbort + 8;                // long long start, end, off_b, b, total tiles, whole
+constexpr int kSmemUsed = kOffWork + 48;
 constexpr int kSmemBytes = kSmemUsed + 1024;           // + alignment slack of the dynamic base
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert((kOffBar % 8) == 0 && (kOffWork % 8) == 0 && (kOffEpi % 1024) == 0 && (kOffStaging % 16) == 0, "alignment");
@@ -124,6 +125,9 @@ struct Params {
   float* part_o;               // [2 * pairs, 128, 512]
   float* part_lse;             // [2 * pairs, 128]
   float sm_scale_log2;         // sm_scale * log2(e)
+  // 1: launched cooperatively; the kernel then merges cut sequences itself after a grid-wide barrier
+  // (taken only when something was cut) and no merge kernel follows
+  int merge_in_kernel;
 };
 
 // ---- work split -----------------------------------------------------------------------------------
@@ -189,8 +193,8 @@ __device__ void plan_range(const int32_t* seqlens, int B, int s_q, int max_tiles
   }
   const long long T = __shfl_sync(0xffffffffu, incl, 31);
   const long long excl = incl - local;
-  if (lane == 0) out[4] = T;
   const int G = npairs / s_q, grp = pair / s_q;
+  if (lane == 0) { out[4] = T; out[5] = (G > 0 && whole_sequences(B, G, T, max_tb)) ? 1 : 0; }
   if (grp >= G) {   // left over when s_q does not divide the pairs: no work
     if (lane == 0) { out[0] = 0; out[1] = 0; out[2] = 0; out[3] = B; }
     return;
@@ -220,6 +224,74 @@ __device__ void plan_range(const int32_t* seqlens, int B, int s_q, int max_tiles
     }
   }
   if (lane == 0 && start >= end) { out[0] = 0; out[1] = 0; out[2] = 0; out[3] = B; }
+}
+
+// ---- merge of split sequences ------------------------------------------------------------------------
+// group g covers global tiles [g*T/G, (g+1)*T/G); the group holding tile x is floor(((x+1)*G - 1) / T).
+__device__ __forceinline__ int pair_of(long long x, long long T, int P) { return (int)(((x + 1) * P - 1) / T); }
+
+// One warp combines the parts of new token v (= b * s_q + tok) and head h, if its sequence was cut:
+// the parts come from pair (group, tok) of the groups that covered the sequence's tiles. T = total
+// tiles, G = groups; lane l holds sequences [b0, b1) for the prefix of tiles before b.
+__device__ __forceinline__ void merge_token_head(const int32_t* __restrict__ seqlens, int s_q, int max_tiles, int G,
+                                                 long long T, int b0, int b1, int v, int h,
+                                                 const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                                                 __nv_bfloat16* __restrict__ o_lat, float* __restrict__ lse) {
+  const int lane = threadIdx.x & 31;
+  const int b = v / s_q, tok = v % s_q;
+  long long before = 0;
+  for (int x = b0; x < min(b1, b); ++x) before += tiles_of(__ldg(seqlens + x), max_tiles);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+  const long long off = before, tb = tiles_of(__ldg(seqlens + b), max_tiles);
+  if (tb == 0) return;
+  const int p0 = pair_of(off, T, G), p1 = pair_of(off + tb - 1, T, G);   // groups
+  if (p0 == p1) return;                       // written whole by one group
+  // a group with an empty range wrote nothing; the others' parts in order, lane q holds group p0 + q's lse
+  auto slot = [&](int q) -> int {
+    const long long start_q = (long long)q * T / G;
+    if ((long long)(q + 1) * T / G <= start_q) return -1;
+    return (q * s_q + tok) * 2 + (start_q < off ? 1 : 0);
+  };
+  float mx = -INFINITY;
+  for (int q0 = p0; q0 <= p1; q0 += 32) {
+    const int q = q0 + lane;
+    const int idx = q <= p1 ? slot(q) : -1;
+    mx = fmaxf(mx, warp_max(idx >= 0 ? part_lse[(size_t)idx * kH + h] : -INFINITY));
+  }
+  float tot = 0.f;
+  float acc[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+  // lane covers columns [4 lane + 128 k, +4) for k < 4: every load instruction reads 512 contiguous bytes
+  for (int q = p0; q <= p1; q += 2) {
+    const int i0 = slot(q), i1 = q + 1 <= p1 ? slot(q + 1) : -1;
+    float4 x0[4], x1[4];
+    const float w0 = i0 >= 0 ? exp2f((part_lse[(size_t)i0 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
+    const float w1 = i1 >= 0 ? exp2f((part_lse[(size_t)i1 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
+    const float4* s0 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i0, 0) * kH + h) * kDC) + lane;
+    const float4* s1 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i1, 0) * kH + h) * kDC) + lane;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x0[k] = i0 >= 0 ? s0[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+      x1[k] = i1 >= 0 ? s1[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    tot += w0 + w1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc[4 * k] += w0 * x0[k].x + w1 * x1[k].x;
+      acc[4 * k + 1] += w0 * x0[k].y + w1 * x1[k].y;
+      acc[4 * k + 2] += w0 * x0[k].z + w1 * x1[k].z;
+      acc[4 * k + 3] += w0 * x0[k].w + w1 * x1[k].w;
+    }
+  }
+  const float inv = 1.f / tot;
+  uint2* dst = reinterpret_cast<uint2*>(o_lat + ((size_t)v * kH + h) * kDC) + lane;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    dst[32 * k] = make_uint2(ptx::pack_bf16x2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
+                             ptx::pack_bf16x2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
+  if (lane == 0) lse[(size_t)v * kH + h] = mx + logf(tot);
 }
 
 // ---- bounded waits ---------------------------------------------------------------------------------
@@ -801,21 +873,35 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
   }
 
   // teardown: TMEM back, then leave together so no remote access can target an exited CTA. The
-  // merge that follows may be scheduled from here on (it waits for this grid's completion and its
-  // writes before reading anything), so its launch overlaps the last CTAs' exit.
+  // merge kernel that follows (when there is one) may be scheduled from here on (it waits for this
+  // grid's completion and its writes before reading anything), so its launch overlaps the last
+  // CTAs' exit.
   ptx::tc_fence_before();
   __syncthreads();
-  allow_dependents();
+  if (!p.merge_in_kernel) allow_dependents();
   if (warp == 2) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
   ptx::cluster_sync();
+  if (p.merge_in_kernel) {
+    // Launched cooperatively: when a sequence was cut (the same decision in every CTA, from the same
+    // totals) every CTA passes one grid-wide barrier, after which all parts are written and visible,
+    // and the grid's warps take the (token, head) units in turn. Every path of the kernel arrives
+    // here (all waits above are bounded), so the barrier always completes.
+    if (work[4] > 0 && work[5] == 0) {
+      cooperative_groups::this_grid().sync();
+      const int per = (p.B + 31) / 32;
+      const int b0 = min(p.B, lane * per), b1 = min(p.B, b0 + per);
+      const int warps = kThreads / 32;
+      const long long units = (long long)p.B * p.s_q * kH;
+      for (long long u = (long long)blockIdx.x * warps + warp; u < units; u += (long long)gridDim.x * warps)
+        merge_token_head(p.seqlens, p.s_q, p.max_tiles, npairs / p.s_q, work[4], b0, b1, (int)(u / kH), (int)(u % kH),
+                         p.part_o, p.part_lse, p.o_lat, p.lse);
+    }
+    allow_dependents();
+  }
 }
-
-// ---- merge of split sequences ------------------------------------------------------------------------
-// group g covers global tiles [g*T/G, (g+1)*T/G); the group holding tile x is floor(((x+1)*G - 1) / T).
-__device__ __forceinline__ int pair_of(long long x, long long T, int P) { return (int)(((x + 1) * P - 1) / T); }
 
 // One warp per (sequence, head), 4 heads per block of 128 threads (about 1.4 waves at 48 registers).
 // Each warp finds the sequence's tile range itself (no block barrier), then issues all its
@@ -849,63 +935,8 @@ merge_kernel(const int32_t* __restrict__ seqlens, int B, int s_q, int max_tiles,
   }
   const long long T = local;
   if (T == 0 || G == 0 || whole_sequences(B, G, T, max_tb)) return;   // nothing was cut
-  for (int v = blockIdx.x; v < B * s_q; v += gridDim.x) {
-    const int b = v / s_q, tok = v % s_q;
-    long long before = 0;
-    for (int x = b0; x < min(b1, b); ++x) before += tiles_of(__ldg(seqlens + x), max_tiles);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
-    const long long off = before, tb = tiles_of(__ldg(seqlens + b), max_tiles);
-    if (tb == 0) continue;
-    const int p0 = pair_of(off, T, G), p1 = pair_of(off + tb - 1, T, G);   // groups
-    if (p0 == p1) continue;                     // written whole by one group
-    const int h = blockIdx.y * kMergeHeads + warp;
-    // a group with an empty range wrote nothing; the others' parts in order, lane q holds group p0 + q's lse
-    auto slot = [&](int q) -> int {
-      const long long start_q = (long long)q * T / G;
-      if ((long long)(q + 1) * T / G <= start_q) return -1;
-      return (q * s_q + tok) * 2 + (start_q < off ? 1 : 0);
-    };
-    float mx = -INFINITY;
-    for (int q0 = p0; q0 <= p1; q0 += 32) {
-      const int q = q0 + lane;
-      const int idx = q <= p1 ? slot(q) : -1;
-      mx = fmaxf(mx, warp_max(idx >= 0 ? part_lse[(size_t)idx * kH + h] : -INFINITY));
-    }
-    float tot = 0.f;
-    float acc[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    // lane covers columns [4 lane + 128 k, +4) for k < 4: every load instruction reads 512 contiguous bytes
-    for (int q = p0; q <= p1; q += 2) {
-      const int i0 = slot(q), i1 = q + 1 <= p1 ? slot(q + 1) : -1;
-      float4 x0[4], x1[4];
-      const float w0 = i0 >= 0 ? exp2f((part_lse[(size_t)i0 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
-      const float w1 = i1 >= 0 ? exp2f((part_lse[(size_t)i1 * kH + h] - mx) * 1.4426950408889634f) : 0.f;
-      const float4* s0 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i0, 0) * kH + h) * kDC) + lane;
-      const float4* s1 = reinterpret_cast<const float4*>(part_o + ((size_t)max(i1, 0) * kH + h) * kDC) + lane;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        x0[k] = i0 >= 0 ? s0[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
-        x1[k] = i1 >= 0 ? s1[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      tot += w0 + w1;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        acc[4 * k] += w0 * x0[k].x + w1 * x1[k].x;
-        acc[4 * k + 1] += w0 * x0[k].y + w1 * x1[k].y;
-        acc[4 * k + 2] += w0 * x0[k].z + w1 * x1[k].z;
-        acc[4 * k + 3] += w0 * x0[k].w + w1 * x1[k].w;
-      }
-    }
-    const float inv = 1.f / tot;
-    uint2* dst = reinterpret_cast<uint2*>(o_lat + ((size_t)v * kH + h) * kDC) + lane;
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      dst[32 * k] = make_uint2(ptx::pack_bf16x2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
-                               ptx::pack_bf16x2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
-    if (lane == 0) lse[(size_t)v * kH + h] = mx + logf(tot);
-  }
+  for (int v = blockIdx.x; v < B * s_q; v += gridDim.x)
+    merge_token_head(seqlens, s_q, max_tiles, G, T, b0, b1, v, blockIdx.y * kMergeHeads + warp, part_o, part_lse, o_lat, lse);
 }
 
 // ---- host side -----------------------------------------------------------------------------------------
@@ -981,9 +1012,42 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   prm.part_o = reinterpret_cast<float*>(workspace);
   prm.part_lse = prm.part_o + (size_t)2 * max_pairs(num_sms) * kH * kDC;
   prm.sm_scale_log2 = d->sm_scale * 1.4426950408889634f;
-  launch_pdl(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
-  launch_pdl(merge_kernel, dim3(std::min(B * s_q, kMergeTokenBlocks), kH / kMergeHeads), dim3(32 * kMergeHeads), 0, st, seqlens, (int)B, (int)s_q, (int)max_pages, P, (const float*)prm.part_o,
-         (const float*)prm.part_lse, prm.o_lat, lse);
+  // First choice: one cooperative launch that merges cut sequences itself (no merge kernel, no
+  // kernel boundary after the decode). If the runtime does not take a cooperative launch of this
+  // clustered grid (with programmatic dependent launch, then without), the decode and the merge
+  // kernel go as two launches. The outcome is remembered per device.
+  static int coop_mode[64] = {0};   // 0 unknown, 1 cooperative + PDL, 2 cooperative, 3 two launches
+  const int di = (dev >= 0 && dev < 64) ? dev : 0;
+  for (int mode = coop_mode[di] ? coop_mode[di] : 1; mode <= 3; ++mode) {
+    if (mode == 3) {
+      prm.merge_in_kernel = 0;
+      launch_pdl(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
+      launch_pdl(merge_kernel, dim3(std::min(B * s_q, kMergeTokenBlocks), kH / kMergeHeads), dim3(32 * kMergeHeads), 0,
+                 st, seqlens, (int)B, (int)s_q, (int)max_pages, P, (const float*)prm.part_o,
+                 (const float*)prm.part_lse, prm.o_lat, lse);
+      coop_mode[di] = 3;
+      break;
+    }
+    prm.merge_in_kernel = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * P);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = mode == 1 ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, decode_kernel, tm_lat, tm_rope, tm_q, prm) == cudaSuccess) {
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      coop_mode[di] = mode;
+      break;
+    }
+    (void)cudaGetLastError();   // a configuration the runtime refused: nothing was launched
+  }
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
