@@ -692,6 +692,7 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
+    import numpy as np
     import torch
     import torch.distributed as dist
     import synth
@@ -753,6 +754,8 @@ def main():
         ws_q = torch.empty(max(16, L.load().mla_query_workspace_size(ctypes.byref(dc), w.B, w.s_q, w.C, w.d_q)),
                            dtype=torch.uint8, device=device)
 
+    lens_host = np.ascontiguousarray(dev["lens"], dtype=np.int32)
+
     def step(x, q_nope, q_rope, events=None, out_t=None):
         """One decode step. events: None; "decode" (two events around the decode call, which is all
         the timed region carries, so the other kernels keep overlapping their launches); or "all"
@@ -777,7 +780,10 @@ def main():
                                       dev["table"], cache, q_abs=q_abs, workspace=ws_app)
         if events:
             mark("append_absorb")
-        ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"], o_lat=o_lat, lse=lse, workspace=ws_dec)
+        # a3 + a4, with the host's copy of the lengths (a serving host has it): no split machinery
+        # when nothing is cut
+        ops.mla_decode_absorbed(dims, q_abs, cache, dev["table"], dev["seqlens"], o_lat=o_lat, lse=lse, workspace=ws_dec,
+                                seqlens_host=lens_host)
         if events:
             mark("decode")
         ops.mla_out_proj(dims, o_lat, dev["W_UV"], out=out if out_t is None else out_t)

@@ -202,6 +202,18 @@ MLA_API int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B
                         const void* q_abs, const mla_latent_cache_t* cache,
                         const int32_t* block_table, int32_t max_pages, const int32_t* seqlens,
                         void* o_lat, float* lse, void* workspace, size_t ws_bytes, void* stream);
+/* The same call given a host copy of the lengths (seqlens_host: B int32 in host memory, equal to
+ * seqlens; NULL is mla_decode_absorbed). The tensor-core decode cuts sequences between its worker
+ * pairs only when the batch is unbalanced; the copy lets the host see beforehand that nothing will
+ * be cut, and the decode then goes as one plain launch without the split merge machinery (at the
+ * bench shape a few microseconds less per call). If the device's seqlens nevertheless make the
+ * kernel cut a sequence (the copy was stale), that sequence's outputs are left unmerged and
+ * MLA_ERR_DEVICE_CHECK is recorded. The copy is read during the call only. */
+MLA_API int mla_decode_absorbed_hinted(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q,
+                               const void* q_abs, const mla_latent_cache_t* cache,
+                               const int32_t* block_table, int32_t max_pages, const int32_t* seqlens,
+                               const int32_t* seqlens_host, void* o_lat, float* lse, void* workspace,
+                               size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
  * a5. Output projection (« Ce que DeepSeek fait de plus »: the weighted latent sum is projected

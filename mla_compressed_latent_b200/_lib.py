@@ -61,6 +61,9 @@ SIGNATURES = {
     "mla_decode_workspace_size": (c_size_t, [PD, c_int32, c_int32, c_int32, c_int32]),
     "mla_decode_absorbed": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, POINTER(MlaLatentCache), PI,
                                       c_int32, PI, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "mla_decode_absorbed_hinted": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, POINTER(MlaLatentCache), PI,
+                                             c_int32, PI, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                             c_void_p]),
     "mla_out_proj": (c_int32, [PD, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_int32,
                                c_void_p, c_void_p]),
     "mla_gqla_workspace_size": (c_size_t, [PD, c_int32, c_int32, c_int32, c_int32]),

@@ -128,10 +128,13 @@ struct Params {
   // 1: launched cooperatively; the kernel then merges cut sequences itself after a grid-wide barrier
   // (taken only when something was cut) and no merge kernel follows
   int merge_in_kernel;
+  // 1: launched without any merge because the host's copy of seqlens cut no sequence; a cut found
+  // here from the device's seqlens is then reported (its parts would stay unmerged)
+  int expect_whole;
 };
 
 // ---- work split -----------------------------------------------------------------------------------
-__device__ __forceinline__ int tiles_of(int L, int max_tiles) { return L > 0 ? min((L + kTile - 1) / kTile, max_tiles) : 0; }
+__host__ __device__ __forceinline__ int tiles_of(int L, int max_tiles) { return L > 0 ? min((L + kTile - 1) / kTile, max_tiles) : 0; }
 
 // Walks the segments (sequence, tile range) of one pair's contiguous range of the global tile list.
 struct SegIter {
@@ -165,7 +168,7 @@ struct SegIter {
 // balanced share, each group takes one whole sequence instead (group g takes sequence g; nothing is
 // cut). Both the decode and the merge kernel decide it the same way from seqlens.
 constexpr int kSplitSlack = 12;
-__device__ __forceinline__ bool whole_sequences(int B, int npairs, long long T, int max_tb) {
+__host__ __device__ __forceinline__ bool whole_sequences(int B, int npairs, long long T, int max_tb) {
   return B <= npairs && (long long)max_tb <= (T + npairs - 1) / npairs + kSplitSlack;
 }
 
@@ -884,6 +887,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant_
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
   ptx::cluster_sync();
+  if (p.expect_whole && work[4] > 0 && work[5] == 0 && threadIdx.x == 0 && blockIdx.x == 0) report(MLA_ERR_DEVICE_CHECK);
   if (p.merge_in_kernel) {
     // Launched cooperatively: when a sequence was cut (the same decision in every CTA, from the same
     // totals) every CTA passes one grid-wide barrier, after which all parts are written and visible,
@@ -980,7 +984,7 @@ inline int active_pairs(int num_sms) {
 
 inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void* q_abs, const mla_latent_cache_t* cache,
                          const int32_t* block_table, int32_t max_pages, const int32_t* seqlens, void* o_lat, float* lse,
-                         void* workspace, size_t ws_bytes, int num_sms, cudaStream_t st) {
+                         void* workspace, size_t ws_bytes, int num_sms, const int32_t* seqlens_host, cudaStream_t st) {
   if (!workspace || ws_bytes < decode_workspace_bytes(d, MLA_BF16, B, s_q, num_sms)) return MLA_ERR_WORKSPACE;
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -1012,6 +1016,24 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   prm.part_o = reinterpret_cast<float*>(workspace);
   prm.part_lse = prm.part_o + (size_t)2 * max_pairs(num_sms) * kH * kDC;
   prm.sm_scale_log2 = d->sm_scale * 1.4426950408889634f;
+  prm.expect_whole = 0;
+  if (seqlens_host) {
+    // the host's copy of the lengths decides the split as the kernel will: when nothing is cut, the
+    // decode goes as a plain launch (programmatic dependent launch, no merge at all)
+    long long T = 0;
+    int max_tb = 0;
+    for (int b = 0; b < B; ++b) {
+      const int tb = tiles_of(seqlens_host[b], max_pages);
+      T += tb;
+      max_tb = std::max(max_tb, tb);
+    }
+    if (T == 0 || whole_sequences(B, P / s_q, T, max_tb)) {
+      prm.merge_in_kernel = 0;
+      prm.expect_whole = 1;
+      launch_pdl(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
+      return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    }
+  }
   // First choice: one cooperative launch that merges cut sequences itself (no merge kernel, no
   // kernel boundary after the decode). If the runtime does not take a cooperative launch of this
   // clustered grid (with programmatic dependent launch, then without), the decode and the merge

@@ -493,10 +493,10 @@ size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t dtype, int32_t 
   return ws;
 }
 
-int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_abs,
-                        const mla_latent_cache_t* cache, const int32_t* block_table, int32_t max_pages,
-                        const int32_t* seqlens, void* o_lat, float* lse, void* workspace, size_t ws_bytes,
-                        void* stream) {
+int mla_decode_absorbed_hinted(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_abs,
+                               const mla_latent_cache_t* cache, const int32_t* block_table, int32_t max_pages,
+                               const int32_t* seqlens, const int32_t* seqlens_host, void* o_lat, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_dtype(dtype))) return rc;
@@ -514,7 +514,7 @@ int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_
   if (mla::sm100::decode_supported(dims, dtype, B, s_q)) {
     const mla_dims_t dd = with_scale(dims);
     return mla::sm100::launch_decode(&dd, B, s_q, q_abs, cache, block_table, max_pages, seqlens, o_lat, lse,
-                                     workspace, ws_bytes, num_sms(), st);
+                                     workspace, ws_bytes, num_sms(), seqlens_host, st);
   }
 
   if (dims->H % mla::simt::DEC_HEADS || dims->d_c % 32 || dims->d_c > 32 * mla::simt::DEC_MAX_OV)
@@ -535,6 +535,14 @@ int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_
   A.nsplit = sp.nsplit; A.chunk = sp.chunk;
   return dtype == MLA_F32 ? launch_decode_simt<float>(A, n_tok, workspace, ws_bytes, st)
                           : launch_decode_simt<__nv_bfloat16>(A, n_tok, workspace, ws_bytes, st);
+}
+
+int mla_decode_absorbed(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_abs,
+                        const mla_latent_cache_t* cache, const int32_t* block_table, int32_t max_pages,
+                        const int32_t* seqlens, void* o_lat, float* lse, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  return mla_decode_absorbed_hinted(dims, dtype, B, s_q, q_abs, cache, block_table, max_pages, seqlens, nullptr, o_lat,
+                                    lse, workspace, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------------------------------------

@@ -212,7 +212,10 @@ def mla_decode_workspace_size(dims: Dims, dtype, B, s_q, max_pages) -> int:
 
 
 def mla_decode_absorbed(dims: Dims, q_abs, cache: LatentCache, block_table, seqlens, o_lat=None, lse=None,
-                        workspace=None, stream=None):
+                        workspace=None, stream=None, seqlens_host=None):
+    """a3 + a4. seqlens_host: optional host copy of seqlens (int32, B values; a numpy array or a CPU
+    tensor) that lets the library launch the decode without the split machinery when nothing is
+    cut (mla_decode_absorbed_hinted)."""
     lib = L.load()
     B, s_q, H, _ = q_abs.shape
     if o_lat is None:
@@ -224,10 +227,20 @@ def mla_decode_absorbed(dims: Dims, q_abs, cache: LatentCache, block_table, seql
     need = lib.mla_decode_workspace_size(ctypes.byref(d), _dt(q_abs), B, s_q, max_pages)
     workspace, wsb = _workspace(need, q_abs.device, workspace)
     cc = cache.c()
-    rc = lib.mla_decode_absorbed(ctypes.byref(d), _dt(q_abs), B, s_q, _ptr(q_abs), ctypes.byref(cc),
-                                 _ptr(_i32(block_table)), max_pages, _ptr(_i32(seqlens)), _ptr(o_lat), _ptr(lse),
-                                 _ptr(workspace) if workspace is not None else None, wsb, _stream(stream))
-    _check("mla_decode_absorbed", rc)
+    if seqlens_host is None:
+        rc = lib.mla_decode_absorbed(ctypes.byref(d), _dt(q_abs), B, s_q, _ptr(q_abs), ctypes.byref(cc),
+                                     _ptr(_i32(block_table)), max_pages, _ptr(_i32(seqlens)), _ptr(o_lat), _ptr(lse),
+                                     _ptr(workspace) if workspace is not None else None, wsb, _stream(stream))
+        _check("mla_decode_absorbed", rc)
+    else:
+        host = torch.as_tensor(seqlens_host, dtype=torch.int32).contiguous()
+        if host.is_cuda or host.numel() != B:
+            raise ValueError("seqlens_host: B int32 values in host memory")
+        rc = lib.mla_decode_absorbed_hinted(ctypes.byref(d), _dt(q_abs), B, s_q, _ptr(q_abs), ctypes.byref(cc),
+                                            _ptr(_i32(block_table)), max_pages, _ptr(_i32(seqlens)),
+                                            ctypes.c_void_p(host.data_ptr()), _ptr(o_lat), _ptr(lse),
+                                            _ptr(workspace) if workspace is not None else None, wsb, _stream(stream))
+        _check("mla_decode_absorbed_hinted", rc)
     return o_lat, lse
 
 

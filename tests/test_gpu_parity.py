@@ -669,6 +669,36 @@ def test_gqla_full_size_sampled():
 # errors
 # ------------------------------------------------------------------------------------------------
 
+@pytest.mark.parametrize("lens,s_q", [([4096] * 64, 1), ([4096, 129, 2049, 64, 5000], 1), ([131072], 1),
+                                      ([65, 66, 4, 64 * 3 + 2, 64 * 3 + 3], 4), ([1, 2], 1)])
+def test_decode_with_host_lengths_equals_plain(lens, s_q):
+    """mla_decode_absorbed_hinted (a host copy of seqlens) gives the outputs of mla_decode_absorbed
+    bit for bit, whether the copy shows nothing cut (a plain launch, no merge) or a cut (the merging
+    launch), and records nothing."""
+    w = synth.workload("dsv3_b64_l4096", B=len(lens), s_q=s_q, lengths=("list", tuple(lens)), pages="random")
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    dims = Dims.of(w)
+    o_ref, l_ref = ops.mla_decode_absorbed(dims, dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"])
+    o, l = ops.mla_decode_absorbed(dims, dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"],
+                                   seqlens_host=case.lens.astype(np.int32))
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    assert torch.equal(o, o_ref) and torch.equal(l, l_ref)
+
+
+def test_stale_host_lengths_are_reported():
+    """A host copy that shows nothing cut while the device's lengths cut a sequence: the plain launch
+    cannot merge it, so the call records MLA_ERR_DEVICE_CHECK."""
+    w = synth.workload("dsv3_b64_l4096", B=1, lengths=("list", (131072,)), pages="random")
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), dev["table"], dev["seqlens"],
+                            seqlens_host=np.array([64], dtype=np.int32))
+    assert ops.mla_check_status() == L.MLA_ERR_DEVICE_CHECK
+    assert ops.mla_check_status() == 0
+
+
 def test_page_id_outside_pool_is_reported_not_read():
     w = synth.workload("dsv3_b64_l4096", B=2, lengths=("list", (200, 70)))
     case = Case(w, with_weights=False)

@@ -73,6 +73,9 @@ CALLS = {
     # B, s_q, q_abs, cache, table, max_pages, seqlens, o_lat, lse, ws, ws_bytes, stream
     "mla_decode_absorbed": ([64, 1, P, "LC", P, 64, P, P, P, P, BIG_WS, None],
                             [2, 4, 6, 7, 8], [0, 1, 5], 9, []),
+    # ... the same with the host copy of seqlens (NULL here: a host pointer is never faked)
+    "mla_decode_absorbed_hinted": ([64, 1, P, "LC", P, 64, P, None, P, P, P, BIG_WS, None],
+                                   [2, 4, 6, 8, 9], [0, 1, 5], 10, []),
     # B, s_q, x, C, w_dkv_kr, gamma, q_nope, q_rope_raw, w_uk, seqlens, table, max_pages, cache, q_abs,
     # ws, ws_bytes, stream
     "mla_append_cache_absorb_q": ([64, 1, P, 7168, P, P, P, P, P, P, P, 64, "LC", P, P, BIG_WS, None],
