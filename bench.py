@@ -32,9 +32,6 @@ UNIT = "positions/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # nominal B200 figures (context for the measured fractions): HBM3e ~8 TB/s, dense bf16 2.25 PFLOP/s
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
-# fp32 FMA throughput of the CUDA cores (the roof of a kernel that does its contractions there):
-# 148 SMs x 128 fp32 lanes x 2 FLOPs per FMA x 1965 MHz (the maximum SM clock)
-ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def parse():
@@ -515,7 +512,7 @@ def time_decode_alone(name, device, steps, warmup, peaks):
 
             def call():
                 ops.mla_decode_absorbed_fp8(dims, q_abs, cache8, tbl, seqlens, o_lat=o_lat, lse=lse, workspace=ws)
-            kernel = "mla_decode_absorbed_fp8 (CUDA-core decode + split merge)"
+            kernel = "mla_decode_absorbed_fp8 (pages dequantised to a bf16 scratch, then the tensor-core decode)"
         else:
             ws = torch.empty(max(16, ops.mla_decode_workspace_size(dims, torch.bfloat16, w.B, w.s_q, table.shape[1])),
                              dtype=torch.uint8, device=device)
@@ -538,11 +535,7 @@ def time_decode_alone(name, device, steps, warmup, peaks):
     sec = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
     gbs, tfs = bytes_ / sec / 1e9, flops / sec / 1e12
     t_hbm, t_tc = bytes_ / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)
-    if getattr(w, "latent_bits", 16) == 8:   # the 8-bit decode runs its contractions on the CUDA cores
-        roof = {"bound": "alu", "achieved": tfs, "peak": ALU_FP32_TFLOPS, "unit": "TFLOP/s",
-                "frac": tfs / ALU_FP32_TFLOPS, "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
-                "peak_note": "fp32 FMA of 148 SMs x 128 lanes at 1965 MHz"}
-    elif t_tc > t_hbm:
+    if t_tc > t_hbm:
         roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": tfs / peaks["bf16_tflops"],
                 "frac_sustained": tfs / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),

@@ -297,9 +297,12 @@ MLA_API int mla_out_proj_preabsorbed(const mla_dims_t* dims, int32_t dtype, int3
  *   of 16).
  * mla_decode_absorbed_fp8: a3 + a4 over that cache. The cache descriptor names the codes, the
  *   scales and the dtype RoPE keys of the same num_pages*64 rows. workspace: at least
- *   mla_decode_fp8_workspace_size(...) bytes (split partials; no initialisation needed). Runs on the
- *   CUDA cores (fp32 arithmetic); requires every seqlens[b] >= s_q. Same errors as
- *   mla_decode_absorbed.
+ *   mla_decode_fp8_workspace_size(...) bytes, no initialisation needed. In bf16 at the shapes of
+ *   the tensor-core decode (H = 128, d_c = 512, d_r = 64, s_q <= 8) the pages the batch reads are
+ *   first dequantised into the workspace (bf16 rows s * value(code), rounded once, and the RoPE keys:
+ *   B * max_pages * 64 * (d_c + d_r) * 2 bytes, plus a dense page table and the decode's own
+ *   workspace), and the tensor-core decode runs over them; otherwise the decode runs on the CUDA
+ *   cores (fp32 arithmetic). Requires every seqlens[b] >= s_q. Same errors as mla_decode_absorbed.
  * ------------------------------------------------------------------------------------------- */
 typedef struct mla_latent_cache_fp8 {
   const uint8_t* codes;   /* device, [num_pages*64, >= d_c] E4M3 codes of the latent rows */

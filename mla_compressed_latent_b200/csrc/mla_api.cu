@@ -569,9 +569,33 @@ int mla_quantize_latent_fp8(const mla_dims_t* dims, int32_t dtype, const void* l
   return launch_status();
 }
 
+namespace {
+// The tensor-core route of the 8-bit decode: the batch's pages dequantised into a dense bf16 scratch
+// (latent rows, RoPE rows, a dense page table), then the bf16 tensor-core decode over it.
+struct Fp8Scratch {
+  size_t lat, rope, table, dec, total;
+};
+bool fp8_on_tc(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q) {
+  return mla::sm100::decode_supported(dims, dtype, B, s_q) && dims->d_c % 16 == 0 && dims->d_r % 8 == 0;
+}
+Fp8Scratch fp8_scratch(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t max_pages) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t rows = (size_t)B * max_pages * 64;
+  Fp8Scratch f;
+  f.lat = 0;
+  f.rope = up(rows * dims->d_c * 2);
+  f.table = f.rope + up(rows * dims->d_r * 2);
+  f.dec = f.table + up((size_t)B * max_pages * 4);
+  f.total = f.dec + mla::sm100::decode_workspace_bytes(dims, MLA_BF16, B, s_q, num_sms());
+  return f;
+}
+}  // namespace
+
 size_t mla_decode_fp8_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t max_pages) {
   if (check_dims(dims) || !tokens_ok(B, s_q) || max_pages <= 0) return 0;
-  return simt_decode_ws(B * s_q, dims->H, dims->d_c, max_pages);
+  const size_t simt = simt_decode_ws(B * s_q, dims->H, dims->d_c, max_pages);
+  const bool tc = fp8_on_tc(dims, MLA_BF16, B, s_q) && (int64_t)B * max_pages * 64 <= INT32_MAX;
+  return tc ? std::max(simt, fp8_scratch(dims, B, s_q, max_pages).total) : simt;
 }
 
 int mla_decode_absorbed_fp8(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q, const void* q_abs,
@@ -590,9 +614,26 @@ int mla_decode_absorbed_fp8(const mla_dims_t* dims, int32_t dtype, int32_t B, in
     return MLA_ERR_INVALID_ARG;
   if (cache->code_stride < dims->d_c || cache->code_stride % 16 || !stride_ok(cache->rope_stride, dtype, dims->d_r))
     return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (fp8_on_tc(dims, dtype, B, s_q) && (int64_t)B * max_pages * 64 <= INT32_MAX) {
+    // dequantise the pages the decode reads into bf16 (one rounding of s * value), then decode them
+    // on the tensor cores through a dense page table
+    const Fp8Scratch f = fp8_scratch(dims, B, s_q, max_pages);
+    if (!workspace || ws_bytes < f.total) return MLA_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    using T = __nv_bfloat16;
+    mla::launch_pdl(mla::simt::dequant_pages_kernel, dim3(max_pages, B), dim3(256), 0, st,
+                    (const uint8_t*)cache->codes, cache->code_stride, (const float*)cache->scales, (const T*)cache->rope,
+                    cache->rope_stride, cache->num_pages, seqlens, block_table, max_pages, dims->d_c, dims->d_r,
+                    (T*)(ws + f.lat), (T*)(ws + f.rope), (int32_t*)(ws + f.table));
+    if ((rc = launch_status())) return rc;
+    mla_latent_cache_t dense{ws + f.lat, dims->d_c, ws + f.rope, dims->d_r, B * max_pages};
+    const mla_dims_t dd = with_scale(dims);
+    return mla::sm100::launch_decode(&dd, B, s_q, q_abs, &dense, (const int32_t*)(ws + f.table), max_pages, seqlens,
+                                     o_lat, lse, ws + f.dec, ws_bytes - f.dec, num_sms(), nullptr, st);
+  }
   if (dims->H % mla::simt::DEC_HEADS || dims->d_c % 32 || dims->d_c > 32 * mla::simt::DEC_MAX_OV)
     return MLA_ERR_UNSUPPORTED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int n_tok = B * s_q;
   DecodeArgs A{};
   A.q = q_abs;

@@ -423,6 +423,62 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
   return (c & 0x80u) ? -v : v;
 }
 
+// =============================================================================================
+// f4 on the tensor cores, first pass: the pages a decode reads, dequantised into a dense bf16
+// scratch. Block (p, b) takes page p of sequence b (p below the sequence's tile count): latent row r
+// becomes s_r · value(code) rounded once to bf16 (value from the E4M3 table above), the RoPE key is
+// copied; dense_table[b][p] = b * max_pages + p names the scratch page, for the decode that follows.
+// A page id outside the pool is reported and its rows are zeros. d_c % 16 == 0, d_r % 8 == 0.
+// =============================================================================================
+__global__ void __launch_bounds__(256)
+dequant_pages_kernel(const uint8_t* __restrict__ codes, int64_t code_stride, const float* __restrict__ scales,
+                     const __nv_bfloat16* __restrict__ rope, int64_t rope_stride, int num_pages,
+                     const int32_t* __restrict__ seqlens, const int32_t* __restrict__ block_table, int max_pages,
+                     int d_c, int d_r, __nv_bfloat16* __restrict__ lat_out, __nv_bfloat16* __restrict__ rope_out,
+                     int32_t* __restrict__ dense_table) {
+  __shared__ float lut[256];
+  grid_dependency_wait();   // the inputs may come from the previous kernel of the stream
+  allow_dependents();
+  lut[threadIdx.x] = e4m3_value(threadIdx.x);   // 256 threads, one code each
+  const int p = blockIdx.x, b = blockIdx.y;
+  if (threadIdx.x == 0) dense_table[(int64_t)b * max_pages + p] = b * max_pages + p;
+  const int L = seqlens[b];
+  const int tiles = L > 0 ? min((L + 63) / 64, max_pages) : 0;
+  __syncthreads();
+  if (p >= tiles) return;
+  const int page = block_table[(int64_t)b * max_pages + p];
+  const bool ok = page >= 0 && page < num_pages;
+  if (!ok && threadIdx.x == 0) report(MLA_ERR_DEVICE_CHECK);
+  const int64_t dst0 = ((int64_t)b * max_pages + p) * 64;
+  const int per_row = d_c / 16;
+  for (int i = threadIdx.x; i < 64 * per_row; i += blockDim.x) {
+    const int r = i / per_row, c = i % per_row;
+    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (ok) {
+      const int64_t src = (int64_t)page * 64 + r;
+      const uint4 v = *reinterpret_cast<const uint4*>(codes + src * code_stride + 16 * c);
+      const float sc = scales[src];
+      const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t word = q[k >> 1] >> (16 * (k & 1));
+        const __nv_bfloat162 h = __floats2bfloat162_rn(lut[word & 0xffu] * sc, lut[(word >> 8) & 0xffu] * sc);
+        w[k] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(lat_out + (dst0 + r) * d_c + 16 * c);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+  const int per_rope = d_r / 8;
+  for (int i = threadIdx.x; i < 64 * per_rope; i += blockDim.x) {
+    const int r = i / per_rope, c = i % per_rope;
+    const uint4 v = ok ? *reinterpret_cast<const uint4*>(rope + ((int64_t)page * 64 + r) * rope_stride + 8 * c)
+                       : make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(rope_out + (dst0 + r) * d_r + 8 * c) = v;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 decode_simt_kernel(DecodeArgs A) {
