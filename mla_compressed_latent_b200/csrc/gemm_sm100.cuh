@@ -312,68 +312,68 @@ __device__ __forceinline__ void head_gemm_body(const CUtensorMap& tm_w, const CU
     ptx::tc_fence_after();
     const int jstep = msub > 1 ? 2 : 1;
     for (int j = warp >= 4 ? 0 : 1; j < msub && ok; j += jstep) {
-    const int mj = mt + j;                        // the m-tile of subtile j
-    if (mj * kBM >= M) break;
-    const uint32_t col0 = (uint32_t)(j * p.tn);   // its accumulator's first TMEM column
-    const int m = mj * kBM + row;
-    if (p.vec_out) {
-      // 32 features (the warp's TMEM lanes) x 32 tokens at a time: each thread puts its feature's
-      // values in column `lane` of a [token][feature] tile in shared memory (the ring, free once the
-      // accumulator is done: 4 KB per warp), then the warp stores the tile's token rows in 16-byte
-      // pieces (features are contiguous in every output; M and the strides are multiples of 8).
-      uint8_t* tile = smem_raw + (ring - raw) + (uint32_t)(warp ^ 4) * 4096u;
-      const uint32_t tile_s = ring + (uint32_t)(warp ^ 4) * 4096u;
-      const int f0 = mj * kBM + (warp & 3) * 32;   // the warp's first feature
-      const bool f32_out = !second && p.mode != 0;
-      for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
-        uint32_t r[32];
-        ptx::tmem_ld32(tmem + lane_off + col0 + (uint32_t)c, r);
-        ptx::tmem_wait_ld();
-        const int kn = min(32, p.n_tok - tok0 - c);
-        if (f32_out) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            reinterpret_cast<float*>(tile)[k * 32 + lane] = nk > 0 ? __uint_as_float(r[k]) : 0.f;
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            reinterpret_cast<__nv_bfloat16*>(tile)[k * 32 + lane] = __float2bfloat16_rn(nk > 0 ? __uint_as_float(r[k]) : 0.f);
+      const int mj = mt + j;                        // the m-tile of subtile j
+      if (mj * kBM >= M) break;
+      const uint32_t col0 = (uint32_t)(j * p.tn);   // its accumulator's first TMEM column
+      const int m = mj * kBM + row;
+      if (p.vec_out) {
+        // 32 features (the warp's TMEM lanes) x 32 tokens at a time: each thread puts its feature's
+        // values in column `lane` of a [token][feature] tile in shared memory (the ring, free once the
+        // accumulator is done: 4 KB per warp), then the warp stores the tile's token rows in 16-byte
+        // pieces (features are contiguous in every output; M and the strides are multiples of 8).
+        uint8_t* tile = smem_raw + (ring - raw) + (uint32_t)(warp ^ 4) * 4096u;
+        const uint32_t tile_s = ring + (uint32_t)(warp ^ 4) * 4096u;
+        const int f0 = mj * kBM + (warp & 3) * 32;   // the warp's first feature
+        const bool f32_out = !second && p.mode != 0;
+        for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tmem + lane_off + col0 + (uint32_t)c, r);
+          ptx::tmem_wait_ld();
+          const int kn = min(32, p.n_tok - tok0 - c);
+          if (f32_out) {
+  #pragma unroll
+            for (int k = 0; k < 32; ++k)
+              reinterpret_cast<float*>(tile)[k * 32 + lane] = nk > 0 ? __uint_as_float(r[k]) : 0.f;
+          } else {
+  #pragma unroll
+            for (int k = 0; k < 32; ++k)
+              reinterpret_cast<__nv_bfloat16*>(tile)[k * 32 + lane] = __float2bfloat16_rn(nk > 0 ? __uint_as_float(r[k]) : 0.f);
+          }
+          __syncwarp();
+          const int pieces = f32_out ? 8 : 4;   // 16-byte pieces per 32-feature token row
+          for (int i = lane; i < 32 * pieces; i += 32) {
+            const int t = i / pieces, f = f0 + (i % pieces) * (f32_out ? 4 : 8);
+            if (t >= kn || f >= M) continue;
+            const uint4 v = ptx::ld_shared_v4(tile_s + (uint32_t)i * 16u);
+            const int tok = tok0 + c + t;
+            void* dst = second ? (void*)(p.y2 + (int64_t)tok * p.y2_tok_stride + f)
+                      : p.mode == 0 ? (void*)(p.y + (int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + f)
+                                    : (void*)(p.part + ((int64_t)split * p.n_tok + tok) * p.M + f);
+            *reinterpret_cast<uint4*>(dst) = v;
+          }
+          __syncwarp();
         }
-        __syncwarp();
-        const int pieces = f32_out ? 8 : 4;   // 16-byte pieces per 32-feature token row
-        for (int i = lane; i < 32 * pieces; i += 32) {
-          const int t = i / pieces, f = f0 + (i % pieces) * (f32_out ? 4 : 8);
-          if (t >= kn || f >= M) continue;
-          const uint4 v = ptx::ld_shared_v4(tile_s + (uint32_t)i * 16u);
-          const int tok = tok0 + c + t;
-          void* dst = second ? (void*)(p.y2 + (int64_t)tok * p.y2_tok_stride + f)
-                    : p.mode == 0 ? (void*)(p.y + (int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + f)
-                                  : (void*)(p.part + ((int64_t)split * p.n_tok + tok) * p.M + f);
-          *reinterpret_cast<uint4*>(dst) = v;
+      } else {   // any other output layout: one value per store
+        for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tmem + lane_off + col0 + (uint32_t)c, r);
+          ptx::tmem_wait_ld();
+          if (m >= M) continue;
+          const int kn = min(32, p.n_tok - tok0 - c);
+  #pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            if (k >= kn) break;
+            const int tok = tok0 + c + k;
+            const float v = nk > 0 ? __uint_as_float(r[k]) : 0.f;
+            if (second)
+              p.y2[(int64_t)tok * p.y2_tok_stride + m] = __float2bfloat16_rn(v);
+            else if (p.mode == 0)
+              p.y[(int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + m] = __float2bfloat16_rn(v);
+            else
+              p.part[((int64_t)split * p.n_tok + tok) * p.M + m] = v;
+          }
         }
-        __syncwarp();
       }
-    } else {   // any other output layout: one value per store
-      for (int c = 0; c < p.tn && tok0 + c < p.n_tok; c += 32) {
-        uint32_t r[32];
-        ptx::tmem_ld32(tmem + lane_off + col0 + (uint32_t)c, r);
-        ptx::tmem_wait_ld();
-        if (m >= M) continue;
-        const int kn = min(32, p.n_tok - tok0 - c);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          if (k >= kn) break;
-          const int tok = tok0 + c + k;
-          const float v = nk > 0 ? __uint_as_float(r[k]) : 0.f;
-          if (second)
-            p.y2[(int64_t)tok * p.y2_tok_stride + m] = __float2bfloat16_rn(v);
-          else if (p.mode == 0)
-            p.y[(int64_t)tok * p.y_tok_stride + (int64_t)h * p.y_head_stride + m] = __float2bfloat16_rn(v);
-          else
-            p.part[((int64_t)split * p.n_tok + tok) * p.M + m] = v;
-        }
-      }
-    }
     }
   }
   ptx::tc_fence_before();
