@@ -81,7 +81,7 @@ def load_peaks():
 # DRAM traffic of one decode_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum) from an
 # ncu capture at dsv3_b64_l4096; reported only while the kernel's sources are the ones it was taken
 # on (their hash), otherwise the roofline's traffic is null.
-DECODE_TRAFFIC = {"workload": "dsv3_b64_l4096", "bytes": 311_842_816 + 3_818_752, "sources_sha256_16": "d1b0f91158f9d6a6"}
+DECODE_TRAFFIC = {"workload": "dsv3_b64_l4096", "bytes": 311_842_816 + 3_818_752, "sources_sha256_16": "4c5ed38ef3a23a6b"}
 DECODE_SOURCES = ("decode_sm100.cuh", "ptx_sm100.cuh", "common.cuh")
 # the same for one gqla_kernel launch at gqla_g8_b32_l8192
 GQLA_TRAFFIC = {"workload": "gqla_g8_b32_l8192", "bytes": 1_115_266_304 + 11_254_784, "sources_sha256_16": "76601daee2d83ab6"}

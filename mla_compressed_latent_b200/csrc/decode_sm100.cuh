@@ -982,6 +982,12 @@ inline int active_pairs(int num_sms) {
   return cached[dev];
 }
 
+#ifdef MLA_TEST_HOOKS
+// Test builds only: launch the decode and the merge kernel as two launches (the path taken when the
+// runtime refuses the cooperative launch), so that a test keeps that path covered.
+inline bool g_test_two_launches = false;
+#endif
+
 inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void* q_abs, const mla_latent_cache_t* cache,
                          const int32_t* block_table, int32_t max_pages, const int32_t* seqlens, void* o_lat, float* lse,
                          void* workspace, size_t ws_bytes, int num_sms, const int32_t* seqlens_host, cudaStream_t st) {
@@ -1040,14 +1046,18 @@ inline int launch_decode(const mla_dims_t* d, int32_t B, int32_t s_q, const void
   // kernel go as two launches. The outcome is remembered per device.
   static int coop_mode[64] = {0};   // 0 unknown, 1 cooperative + PDL, 2 cooperative, 3 two launches
   const int di = (dev >= 0 && dev < 64) ? dev : 0;
-  for (int mode = coop_mode[di] ? coop_mode[di] : 1; mode <= 3; ++mode) {
+  bool forced = false;
+#ifdef MLA_TEST_HOOKS
+  forced = g_test_two_launches;
+#endif
+  for (int mode = forced ? 3 : (coop_mode[di] ? coop_mode[di] : 1); mode <= 3; ++mode) {
     if (mode == 3) {
       prm.merge_in_kernel = 0;
       launch_pdl(decode_kernel, dim3(2 * P), dim3(kThreads), kSmemBytes, st, tm_lat, tm_rope, tm_q, prm);
       launch_pdl(merge_kernel, dim3(std::min(B * s_q, kMergeTokenBlocks), kH / kMergeHeads), dim3(32 * kMergeHeads), 0,
                  st, seqlens, (int)B, (int)s_q, (int)max_pages, P, (const float*)prm.part_o,
                  (const float*)prm.part_lse, prm.o_lat, lse);
-      coop_mode[di] = 3;
+      if (!forced) coop_mode[di] = 3;
       break;
     }
     prm.merge_in_kernel = 1;

@@ -196,6 +196,11 @@ uint64_t mla_launch_count(void) { return mla::g_launches.load(std::memory_order_
 MLA_API int mla_test_set_stall(int on) {
   return cudaMemcpyToSymbol(mla::gemm::g_test_stall, &on, sizeof(int)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
+// Test builds only: the decode goes as two launches (decode, then the merge kernel) while on is set.
+MLA_API int mla_test_set_two_launches(int on) {
+  mla::sm100::g_test_two_launches = on != 0;
+  return MLA_OK;
+}
 #endif
 
 const char* mla_build_info(void) {

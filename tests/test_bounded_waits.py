@@ -34,6 +34,8 @@ def _load_test_lib():
         fn.argtypes = args
     lib.mla_test_set_stall.restype = ctypes.c_int32
     lib.mla_test_set_stall.argtypes = [ctypes.c_int32]
+    lib.mla_test_set_two_launches.restype = ctypes.c_int32
+    lib.mla_test_set_two_launches.argtypes = [ctypes.c_int32]
     return lib
 
 
@@ -65,3 +67,40 @@ def test_wait_that_runs_out_reports_timeout_then_next_call_is_clean():
         ref = O.absorb_query(case.q_nope64[b], case.q_rope_raw64[b], case.W64["W_UK"], O.token_positions(L_b, 1))
         err = max_rel_err(got[b], ref)
         assert err <= TOL["bf16"]["out"], f"seq {b}: max|Δ|/max|ref| = {err:.3e}"
+
+
+@pytest.mark.parametrize("lens", [[131072], list(np.random.default_rng(11).integers(1, 2000, 200))])
+def test_decode_as_two_launches_merges_cut_sequences(lens):
+    """The decode's fallback when the runtime refuses its cooperative launch: the decode, then the
+    merge kernel. Cut sequences (one spanning every pair; 200 ragged ones) against the oracle."""
+    lib = _load_test_lib()
+    w = synth.workload("dsv3_b64_l4096", B=len(lens), lengths=("list", tuple(int(x) for x in lens)), pages="random")
+    case = Case(w, with_weights=False)
+    dev = case.to_device()
+    d = Dims.of(w).c()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    max_pages = dev["table"].shape[1]
+    ws = torch.empty(lib.mla_decode_workspace_size(ctypes.byref(d), L.MLA_BF16, w.B, 1, max_pages), dtype=torch.uint8,
+                     device="cuda")
+    o_lat = torch.empty(w.B, 1, w.H, w.d_c, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(w.B, 1, w.H, dtype=torch.float32, device="cuda")
+    pool = dev["pool"]
+    cache = L.MlaLatentCache(pool.data_ptr(), pool.stride(0), pool[:, w.d_c:].data_ptr(), pool.stride(0), case.num_pages)
+    assert lib.mla_test_set_two_launches(1) == L.MLA_OK
+    try:
+        rc = lib.mla_decode_absorbed(ctypes.byref(d), L.MLA_BF16, w.B, 1, ctypes.c_void_p(dev["q_abs"].data_ptr()),
+                                     ctypes.byref(cache), ctypes.c_void_p(dev["table"].data_ptr()), max_pages,
+                                     ctypes.c_void_p(dev["seqlens"].data_ptr()), ctypes.c_void_p(o_lat.data_ptr()),
+                                     ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                     ws.numel(), stream)
+    finally:
+        lib.mla_test_set_two_launches(0)
+    assert rc == L.MLA_OK
+    assert lib.mla_check_status(stream) == L.MLA_OK
+    got_o, got_l = o_lat.double().cpu().numpy(), lse.double().cpu().numpy()
+    for b in range(w.B):
+        c, kr = case.seq_rows64(b)
+        ref_o, ref_l = O.absorbed_decode(case.q_abs64[b], c, kr, int(case.lens[b]), w.sm_scale)
+        err = max_rel_err(got_o[b], ref_o)
+        assert err <= TOL["bf16"]["out"], f"seq {b}: max|Δ|/max|ref| = {err:.3e}"
+        assert float(np.abs(got_l[b] - ref_l).max()) <= TOL["bf16"]["lse"], f"seq {b}: lse"
