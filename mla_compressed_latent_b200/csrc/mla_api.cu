@@ -581,7 +581,9 @@ struct Fp8Scratch {
   size_t lat, rope, table, dec, total;
 };
 bool fp8_on_tc(const mla_dims_t* dims, int32_t dtype, int32_t B, int32_t s_q) {
-  return mla::sm100::decode_supported(dims, dtype, B, s_q) && dims->d_c % 16 == 0 && dims->d_r % 8 == 0;
+  // (the dequantising pass takes one block row per sequence: B within a grid's y extent)
+  return mla::sm100::decode_supported(dims, dtype, B, s_q) && dims->d_c % 16 == 0 && dims->d_r % 8 == 0 &&
+         B <= 65535;
 }
 Fp8Scratch fp8_scratch(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t max_pages) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
