@@ -84,7 +84,7 @@ def load_peaks():
 DECODE_TRAFFIC = {"workload": "dsv3_b64_l4096", "bytes": 311_842_816 + 3_818_752, "sources_sha256_16": "4c5ed38ef3a23a6b"}
 DECODE_SOURCES = ("decode_sm100.cuh", "ptx_sm100.cuh", "common.cuh")
 # the same for one gqla_kernel launch at gqla_g8_b32_l8192
-GQLA_TRAFFIC = {"workload": "gqla_g8_b32_l8192", "bytes": 1_115_266_304 + 11_254_784, "sources_sha256_16": "76601daee2d83ab6"}
+GQLA_TRAFFIC = {"workload": "gqla_g8_b32_l8192", "bytes": 1_115_248_640 + 10_563_072, "sources_sha256_16": "c67edddacfb49765"}
 GQLA_SOURCES = ("gqla_sm100.cuh", "ptx_sm100.cuh", "common.cuh")
 
 
