@@ -768,7 +768,8 @@ def main():
                                                    q_nope=qn_buf, q_rope_raw=qr_buf, workspace=ws_q)
             if every:
                 mark("project_q")
-        # a1 + a2: the cache append and the query absorption, their projections in one launch
+        # a1 + a2 in one call: the cache append, then the query absorption (whose CTAs stream W_UK
+        # while the append's finish runs)
         ops.mla_append_cache_absorb_q(dims, x, dev["w_dkv_kr"], None, q_nope, q_rope, dev["W_UK"], dev["seqlens"],
                                       dev["table"], cache, q_abs=q_abs, workspace=ws_app)
         if events:
