@@ -200,6 +200,27 @@ def test_append_cache(name, B):
     assert torch.equal(pool[mask], before.cpu()[mask])
 
 
+def test_append_cache_row_width_not_a_multiple_of_four():
+    """d_c + d_r = 39 (separate latent and RoPE pools, 16-byte strides): the finish sums its split-K
+    slices one column per thread instead of in 16-byte pieces. Rows against the oracle."""
+    w = synth.workload("smallem_fp32", d_c=33, d_r=6, B=3, lengths=("list", (77, 5, 130)))
+    case = Case(w)
+    dev = case.to_device()
+    rows_total = case.num_pages * 64
+    latent = torch.zeros(rows_total, 36, dtype=torch.float32, device="cuda")[:, :w.d_c]
+    rope = torch.zeros(rows_total, 8, dtype=torch.float32, device="cuda")[:, :w.d_r]
+    cache = LatentCache(latent, rope, case.num_pages)
+    ops.mla_append_cache(Dims.of(w), dev["x"], dev["w_dkv_kr"], None, dev["seqlens"], dev["table"], cache)
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    pos = (case.lens - 1).astype(np.int64)
+    c_ref, kr_ref = O.latent_rows(case.x64[:, 0], case.W64["W_DKV"], case.W64["W_KR"], pos, None, w.rms_eps,
+                                  w.rope_base)
+    rows = torch.from_numpy(case.table[np.arange(w.B), pos // 64].astype(np.int64) * 64 + pos % 64)
+    _assert_close(latent.cpu()[rows].double().numpy(), c_ref, w.dtype, "appended latent")
+    _assert_close(rope.cpu()[rows].double().numpy(), kr_ref, w.dtype, "appended rope key")
+
+
 @pytest.mark.parametrize("name,s_q", [("dsv3_b64_l4096", 1), ("dsv3_b64_l4096", 3), ("smallem_fp32", 1)])
 def test_absorb_q(name, s_q):
     w = synth.workload(name, s_q=s_q, B=7, lengths=("list", (7, 100, 4096, 65, 64, 9999, 131072)))
@@ -375,6 +396,7 @@ def test_smallem_layer_fp32_from_hidden_states(queries):
 @pytest.mark.parametrize("name,over", [
     ("smallem_fp32", {}),
     ("smallem_fp32", dict(B=3, s_q=2)),
+    ("smallem_fp32", dict(d_q=254)),          # a width the float4 RMS step does not take
     ("dsv3_b64_l4096", dict(d_q=1536, lengths=("fixed", 64))),
     ("dsv3_b64_l4096", dict(d_q=1536, B=50, s_q=3, lengths=("fixed", 64))),
 ])
