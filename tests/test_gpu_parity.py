@@ -221,6 +221,22 @@ def test_append_cache_row_width_not_a_multiple_of_four():
     _assert_close(rope.cpu()[rows].double().numpy(), kr_ref, w.dtype, "appended rope key")
 
 
+def test_absorb_q_width_not_a_multiple_of_two_tiles():
+    """d_c = 384: the absorption's CTAs hold two 128-feature m-tiles each, so a head's second CTA has
+    one tile past the weight's last column (its loads read the fill value, its epilogue skips it)."""
+    w = synth.workload("dsv3_b64_l4096", d_c=384, B=5, lengths=("list", (7, 100, 4096, 65, 131072)))
+    case = Case(w)
+    dev = case.to_device()
+    q_abs = ops.mla_absorb_q(Dims.of(w), dev["q_nope"], dev["q_rope_raw"], dev["W_UK"], dev["seqlens"])
+    torch.cuda.synchronize()
+    assert ops.mla_check_status() == 0
+    got = q_abs.to(torch.float64).cpu().numpy()
+    for b in range(w.B):
+        pos = O.token_positions(int(case.lens[b]), 1)
+        ref = O.absorb_query(case.q_nope64[b], case.q_rope_raw64[b], case.W64["W_UK"], pos, w.rope_base)
+        _assert_close(got[b], ref, w.dtype, f"q_abs seq {b}")
+
+
 @pytest.mark.parametrize("name,s_q", [("dsv3_b64_l4096", 1), ("dsv3_b64_l4096", 3), ("smallem_fp32", 1)])
 def test_absorb_q(name, s_q):
     w = synth.workload(name, s_q=s_q, B=7, lengths=("list", (7, 100, 4096, 65, 64, 9999, 131072)))
