@@ -780,6 +780,38 @@ def test_sequence_without_its_new_token_is_reported():
     assert ops.mla_check_status() == 0
 
 
+@pytest.mark.parametrize("combined", [False, True])
+def test_append_to_a_page_outside_the_pool_is_reported_not_written(combined):
+    """A new token whose page id lies outside the pool: the append records MLA_ERR_DEVICE_CHECK and
+    writes nothing for it; the other sequence's row is written as usual (alone and in the combined
+    append + absorb call)."""
+    w = synth.workload("dsv3_b64_l4096", B=2, lengths=("list", (200, 70)))
+    case = Case(w)
+    dev = case.to_device()
+    cache = _cache(dev, case)
+    bad = dev["table"].clone()
+    bad[1, (70 - 1) // 64] = case.num_pages + 3
+    before = dev["pool"].clone()
+    dims = Dims.of(w)
+    if combined:
+        ops.mla_append_cache_absorb_q(dims, dev["x"], dev["w_dkv_kr"], None, dev["q_nope"], dev["q_rope_raw"],
+                                      dev["W_UK"], dev["seqlens"], bad, cache)
+    else:
+        ops.mla_append_cache(dims, dev["x"], dev["w_dkv_kr"], None, dev["seqlens"], bad, cache)
+    assert ops.mla_check_status() == L.MLA_ERR_DEVICE_CHECK
+    pos = (case.lens - 1).astype(np.int64)
+    c_ref, kr_ref = O.latent_rows(case.x64[:, 0], case.W64["W_DKV"], case.W64["W_KR"], pos, None, w.rms_eps,
+                                  w.rope_base)
+    row0 = int(case.table[0, pos[0] // 64]) * 64 + int(pos[0] % 64)
+    pool = dev["pool"].cpu()
+    got = pool[row0].double().numpy()
+    _assert_close(got[None, :w.d_c], c_ref[:1], w.dtype, "appended latent of the valid sequence")
+    mask = torch.ones(pool.shape[0], dtype=torch.bool)
+    mask[row0] = False
+    assert torch.equal(pool[mask], before.cpu()[mask])   # nothing else moved
+    assert ops.mla_check_status() == 0
+
+
 def test_invalid_arguments_raise():
     w = synth.workload("dsv3_b64_l4096", B=1, lengths=("list", (64,)))
     case = Case(w, with_weights=False)
