@@ -746,6 +746,13 @@ def test_page_id_outside_pool_is_reported_not_read():
     ops.mla_decode_absorbed(Dims.of(w), dev["q_abs"], _cache(dev, case), bad, dev["seqlens"])
     assert ops.mla_check_status() == L.MLA_ERR_DEVICE_CHECK
     assert ops.mla_check_status() == 0       # cleared by the previous read
+    # the 8-bit decode's dequantising pass checks the same ids (its decode reads a dense table)
+    codes, scales = _fp8_rows(case)
+    cache8 = LatentCacheFp8(torch.from_numpy(codes).cuda(), torch.from_numpy(scales.astype(np.float32)).cuda(),
+                            dev["pool"][:, w.d_c:], case.num_pages)
+    ops.mla_decode_absorbed_fp8(Dims.of(w), dev["q_abs"], cache8, bad, dev["seqlens"])
+    assert ops.mla_check_status() == L.MLA_ERR_DEVICE_CHECK
+    assert ops.mla_check_status() == 0
 
 
 def test_sequence_without_its_new_token_is_reported():
